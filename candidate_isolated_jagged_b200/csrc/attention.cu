@@ -1,0 +1,782 @@
+// Jagged candidate-isolated attention on sm_100a (tcgen05 + TMEM + TMA).
+//
+// What it computes (候选隔离注意力掩码, sections 段 ID：掩码的表达方式 and 掩码长什么样): every
+// non-padding query of user b attends to the segment-1 keys of its own row (prefix + history),
+// and each candidate also attends to itself; padding queries output 0. The mask is never
+// materialised: per user, the keys a query can see (besides itself) are exactly the segment-1
+// positions inside [hist_lo, hist_hi), so the work of a user is a dense, non-causal rectangle of
+// (row tiles) x (history key tiles). Key tiles over the candidate range are never visited
+// (history x candidate and candidate x other-candidate pairs are skipped wholesale), and the
+// candidate's self term is merged into the online softmax as a diagonal epilogue on CUDA cores.
+//
+// Kernel structure (one persistent CTA per SM, 6 warps):
+//   warp 0      TMA producer: Q tile (2 buffers), K and V tiles (2-stage rings each).
+//   warp 1      TMEM allocator and single-thread MMA issuer: S = Q K^T into one of two TMEM
+//               S buffers, O += P V into the TMEM O accumulator; completion via tcgen05.commit.
+//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row): masked online
+//               softmax in the log2 domain with fp32 m, l in registers, P written as bf16 to a
+//               128-byte-swizzled shared tile, lazy O rescaling (only when the running max grows
+//               by more than 2^8), then the diagonal merge, 1/l and the store.
+// Work items (user, head, 128-row query tile) come from the cost-sorted queue; CTA c takes items
+// c, c + grid, c + 2 grid, ... so the longest items start first.
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "jca_device.cuh"
+#include "jca_internal.h"
+
+namespace jca {
+namespace {
+
+struct AttnArgs {
+  const __nv_bfloat16* q;   // [Tq, H, D] query rows (read again for the diagonal term)
+  const __nv_bfloat16* dk;  // [Tq, H, D] diagonal keys: the query row's own key
+  const __nv_bfloat16* dv;  // [Tq, H, D] diagonal values
+  const int8_t* q_seg;      // [Tq] segment of each query row, or null = every row is a candidate
+  const int8_t* kv_seg;     // [Tkv] segment of each key row (read only for users with holes)
+  void* out;                // [Tq, H, D] bf16 or fp32
+  const int4* items;
+  const int32_t* n_items;
+  int32_t* status;
+  int H;
+  int out_fp32;
+  float scale_log2;         // softmax scale * log2(e)
+};
+
+template <int D>
+struct Cfg {
+  static constexpr int BM = kTileM;
+  static constexpr int BN = kTileN;
+  static constexpr int ROW_BYTES = D * 2;                          // one head of one token
+  static constexpr int SW = ROW_BYTES >= 128 ? 128 : ROW_BYTES;    // swizzle span (bytes)
+  static constexpr int NBLK = ROW_BYTES / SW;                      // column blocks per tile
+  static constexpr int BOX_X = SW / 2;                             // elements per TMA box row
+  static constexpr int TILE_BYTES = BM * ROW_BYTES;
+  static constexpr int BLK_BYTES = BM * SW;
+  static constexpr uint32_t LAYOUT = SW == 128 ? 2u : (SW == 64 ? 4u : 6u);
+  static constexpr int KSTEPS_QK = D / 16;
+  static constexpr int KSTEPS_PER_BLK = SW / 32;
+  static constexpr int KSTEPS_PV = BN / 16;
+  static constexpr int P_BLK_BYTES = BM * 128;                     // P: two 64-key blocks
+  static constexpr int P_BYTES = 2 * P_BLK_BYTES;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
+  static constexpr int OFF_P = OFF_V + 2 * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int NUM_BARS = 20;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_USED = OFF_MISC + 16;
+  static constexpr int SMEM_RAW = SMEM_USED + 1024;                // slack for 1 KB alignment
+  // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
+  static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+  static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256, TMEM_COLS = 512;
+  static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
+};
+
+// Barrier slots.
+enum : int {
+  kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = 6, kVFull = 8, kVEmpty = 10,
+  kSFull = 12, kSEmpty = 14, kPFull = 16, kPVDone = 17, kDrain = 18
+};
+
+constexpr int kThreads = 192;
+constexpr int kSoftmaxThreads = 128;
+
+struct Item {
+  int q_row0, h, nrows, kv_lo, kv_len, holes, n_kv;
+};
+
+__device__ __forceinline__ Item decode_item(int4 v) {
+  Item w;
+  w.q_row0 = v.x;
+  w.h = v.y >> 8;
+  w.nrows = v.y & 255;
+  w.kv_lo = v.z;
+  w.kv_len = v.w & 0x7fffffff;
+  w.holes = (int)((unsigned)v.w >> 31);
+  w.n_kv = (w.kv_len + kTileN - 1) / kTileN;
+  return w;
+}
+
+// ------------------------------------------------------------------------------------------
+// Producer
+// ------------------------------------------------------------------------------------------
+template <int D>
+__device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                              const CUtensorMap* tmV, const AttnArgs& a, uint32_t sbase,
+                              uint32_t bars, int n_items, volatile int* abort_flag) {
+  using C = Cfg<D>;
+  uint32_t armed[6] = {0, 0, 0, 0, 0, 0};  // q0 q1 k0 k1 v0 v1
+  uint32_t g = 0, qi = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+    const Item w = decode_item(a.items[it]);
+    if (w.n_kv == 0) continue;
+    const int qs = qi & 1;
+    ok = mbar_wait(bars + 8 * (kQEmpty + qs), ((qi >> 1) & 1) ^ 1, abort_flag, a.status);
+    if (!ok) break;
+    mbar_arrive_expect_tx(bars + 8 * (kQFull + qs), C::TILE_BYTES);
+    ++armed[qs];
+#pragma unroll
+    for (int c = 0; c < C::NBLK; ++c)
+      tma_load_3d(sbase + C::OFF_Q + qs * C::TILE_BYTES + c * C::BLK_BYTES, tmQ,
+                  bars + 8 * (kQFull + qs), c * C::BOX_X, w.h, w.q_row0);
+    ++qi;
+    for (int j = 0; j < w.n_kv; ++j, ++g) {
+      const int s = g & 1;
+      const uint32_t ph = (g >> 1) & 1;
+      const int row = w.kv_lo + j * C::BN;
+      ok = mbar_wait(bars + 8 * (kKEmpty + s), ph ^ 1, abort_flag, a.status);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bars + 8 * (kKFull + s), C::TILE_BYTES);
+      ++armed[2 + s];
+#pragma unroll
+      for (int c = 0; c < C::NBLK; ++c)
+        tma_load_3d(sbase + C::OFF_K + s * C::TILE_BYTES + c * C::BLK_BYTES, tmK,
+                    bars + 8 * (kKFull + s), c * C::BOX_X, w.h, row);
+      ok = mbar_wait(bars + 8 * (kVEmpty + s), ph ^ 1, abort_flag, a.status);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bars + 8 * (kVFull + s), C::TILE_BYTES);
+      ++armed[4 + s];
+#pragma unroll
+      for (int c = 0; c < C::NBLK; ++c)
+        tma_load_3d(sbase + C::OFF_V + s * C::TILE_BYTES + c * C::BLK_BYTES, tmV,
+                    bars + 8 * (kVFull + s), c * C::BOX_X, w.h, row);
+    }
+  }
+  if (!ok) {
+    // Aborting: let every copy this thread started land before the CTA exits.
+    const int full_slot[6] = {kQFull, kQFull + 1, kKFull, kKFull + 1, kVFull, kVFull + 1};
+    for (int i = 0; i < 6; ++i)
+      if (armed[i]) mbar_wait_drain(bars + 8 * full_slot[i], (armed[i] - 1) & 1);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// MMA issuer
+// ------------------------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ bool issue_pv(uint32_t gg, bool first, uint32_t sbase, uint32_t bars,
+                                         uint32_t tmem, const AttnArgs& a,
+                                         volatile int* abort_flag) {
+  using C = Cfg<D>;
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(C::BM, D, false, true);
+  const int s = gg & 1;
+  const uint32_t ph = (gg >> 1) & 1;
+  if (!mbar_wait(bars + 8 * (kVFull + s), ph, abort_flag, a.status)) return false;
+  if (!mbar_wait(bars + 8 * kPFull, gg & 1, abort_flag, a.status)) return false;
+  tc_fence_after();
+  const uint32_t p_base = sbase + C::OFF_P;
+  const uint32_t v_base = sbase + C::OFF_V + s * C::TILE_BYTES;
+#pragma unroll
+  for (int kk = 0; kk < C::KSTEPS_PV; ++kk) {
+    // P: K-major, 128-byte swizzle, two 64-key blocks; V: MN-major (head dim contiguous).
+    const uint64_t adesc =
+        smem_desc(p_base + (kk / 4) * C::P_BLK_BYTES + (kk % 4) * 32, 16, 1024, 2u);
+    const uint64_t bdesc =
+        smem_desc(v_base + kk * 16 * C::SW, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
+    tc_mma(tmem + C::TMEM_O, adesc, bdesc, kIdescPV, (first && kk == 0) ? 0u : 1u);
+  }
+  tc_commit(bars + 8 * (kVEmpty + s));
+  tc_commit(bars + 8 * kPVDone);
+  return true;
+}
+
+template <int D>
+__device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                         int n_items, volatile int* abort_flag) {
+  using C = Cfg<D>;
+  constexpr uint32_t kIdescQK = idesc_bf16_f32(C::BM, C::BN, false, false);
+  uint32_t g = 0, qi = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+    const Item w = decode_item(a.items[it]);
+    if (w.n_kv == 0) continue;
+    const int qs = qi & 1;
+    ok = mbar_wait(bars + 8 * (kQFull + qs), (qi >> 1) & 1, abort_flag, a.status);
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t q_base = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+    for (int j = 0; j < w.n_kv; ++j, ++g) {
+      const int s = g & 1;
+      const uint32_t ph = (g >> 1) & 1;
+      ok = mbar_wait(bars + 8 * (kKFull + s), ph, abort_flag, a.status) &&
+           mbar_wait(bars + 8 * (kSEmpty + s), ph ^ 1, abort_flag, a.status);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t k_base = sbase + C::OFF_K + s * C::TILE_BYTES;
+      const uint32_t d_tmem = tmem + (s ? C::TMEM_S1 : C::TMEM_S0);
+#pragma unroll
+      for (int kk = 0; kk < C::KSTEPS_QK; ++kk) {
+        const uint32_t off =
+            (kk / C::KSTEPS_PER_BLK) * C::BLK_BYTES + (kk % C::KSTEPS_PER_BLK) * 32;
+        tc_mma(d_tmem, smem_desc(q_base + off, 16, 8 * C::SW, C::LAYOUT),
+               smem_desc(k_base + off, 16, 8 * C::SW, C::LAYOUT), kIdescQK, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(bars + 8 * (kKEmpty + s));
+      tc_commit(bars + 8 * (kSFull + s));
+      // PV of the previous key tile goes behind this QK, so the tensor core computes the next
+      // S while the softmax warps work on the previous one.
+      if (j > 0) {
+        ok = issue_pv<D>(g - 1, j == 1, sbase, bars, tmem, a, abort_flag);
+        if (!ok) break;
+      }
+    }
+    if (!ok) break;
+    ok = issue_pv<D>(g - 1, w.n_kv == 1, sbase, bars, tmem, a, abort_flag);
+    if (!ok) break;
+    tc_commit(bars + 8 * (kQEmpty + qs));
+    ++qi;
+  }
+  if (!ok) {
+    // Aborting: wait until every MMA this thread issued has completed.
+    tc_commit(bars + 8 * kDrain);
+    mbar_wait_drain(bars + 8 * kDrain, 0);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Softmax + epilogue
+// ------------------------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void load_o_row(uint32_t t_o, float* o) {
+  if constexpr (D == 16) {
+    uint32_t r[16];
+    tmem_ld_x16(t_o, r);
+    tmem_wait_ld();
+    reg_fence16(r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(r[i]);
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; c += 32) {
+      uint32_t r[32];
+      tmem_ld_x32(t_o + c, r);
+      tmem_wait_ld();
+      reg_fence16(r);
+      reg_fence16(r + 16);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[c + i] = __uint_as_float(r[i]);
+    }
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void rescale_o_row(uint32_t t_o, float alpha) {
+  if constexpr (D == 16) {
+    uint32_t r[16];
+    tmem_ld_x16(t_o, r);
+    tmem_wait_ld();
+    reg_fence16(r);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+    tmem_st_x16(t_o, r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; c += 32) {
+      uint32_t r[32];
+      tmem_ld_x32(t_o + c, r);
+      tmem_wait_ld();
+      reg_fence16(r);
+      reg_fence16(r + 16);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+      tmem_st_x32(t_o + c, r);
+    }
+  }
+  tmem_wait_st();
+}
+
+// Diagonal merge (the candidate's own key/value), normalisation and store of one output row.
+template <int D>
+__device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int r, float m,
+                                           float l, float* o) {
+  if (r >= w.nrows) return;
+  const int row = w.q_row0 + r;
+  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
+  const int seg = a.q_seg ? (int)a.q_seg[row] : -1;
+  float inv;
+  if (seg == 0) {
+    inv = 0.f;  // padding query: no visible key
+  } else {
+    if (seg == -1) {
+      const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
+      const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 qa = ld_global_nc_v4(qp + c);
+        const uint4 ka = ld_global_nc_v4(kp + c);
+        acc[0] = fmaf(bf16_lo(qa.x), bf16_lo(ka.x), fmaf(bf16_hi(qa.x), bf16_hi(ka.x), acc[0]));
+        acc[1] = fmaf(bf16_lo(qa.y), bf16_lo(ka.y), fmaf(bf16_hi(qa.y), bf16_hi(ka.y), acc[1]));
+        acc[2] = fmaf(bf16_lo(qa.z), bf16_lo(ka.z), fmaf(bf16_hi(qa.z), bf16_hi(ka.z), acc[2]));
+        acc[3] = fmaf(bf16_lo(qa.w), bf16_lo(ka.w), fmaf(bf16_hi(qa.w), bf16_hi(ka.w), acc[3]));
+      }
+      const float sd = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * a.scale_log2;
+      const float m_new = fmaxf(m, sd);
+      const float alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+      const float beta = fast_exp2(sd - m_new);
+      l = l * alpha + beta;
+      const uint4* vp = reinterpret_cast<const uint4*>(a.dv + base);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c) {
+        const uint4 va = ld_global_nc_v4(vp + c);
+        const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          o[8 * c + 2 * i] = fmaf(o[8 * c + 2 * i], alpha, beta * bf16_lo(vw[i]));
+          o[8 * c + 2 * i + 1] = fmaf(o[8 * c + 2 * i + 1], alpha, beta * bf16_hi(vw[i]));
+        }
+      }
+    }
+    inv = l > 0.f ? 1.f / l : 0.f;
+  }
+  if (a.out_fp32) {
+    float4* op = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base);
+#pragma unroll
+    for (int c = 0; c < D / 4; ++c)
+      op[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
+                          o[4 * c + 3] * inv);
+  } else {
+    uint4* op = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base);
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c)
+      op[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
+                         pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
+                         pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
+                         pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+  }
+}
+
+template <int D>
+__device__ void softmax_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                             int n_items, volatile int* abort_flag, int warp, int lane) {
+  using C = Cfg<D>;
+  const int quarter = warp & 3;               // TMEM lane quarter this warp may access
+  const int r = quarter * 32 + lane;          // query row of this thread inside the tile
+  const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+  const uint32_t p_row = sbase + C::OFF_P + (uint32_t)r * 128u;
+  const uint32_t sw = (uint32_t)(r & 7);
+  uint32_t g = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+    const Item w = decode_item(a.items[it]);
+    float m = -INFINITY, l = 0.f;
+    for (int j = 0; j < w.n_kv; ++j, ++g) {
+      const int s = g & 1;
+      const uint32_t ph = (g >> 1) & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (kSFull + s), ph, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t x[128];
+      const uint32_t t_s = t_lane + (s ? C::TMEM_S1 : C::TMEM_S0);
+      tmem_ld_x32(t_s + 0, x);
+      tmem_ld_x32(t_s + 32, x + 32);
+      tmem_ld_x32(t_s + 64, x + 64);
+      tmem_ld_x32(t_s + 96, x + 96);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 128; c += 16) reg_fence16(x + c);
+      tc_fence_before();
+      mbar_arrive(bars + 8 * (kSEmpty + s));
+
+      // Masked scores in the log2 domain.
+      const int valid_cols = min(C::BN, w.kv_len - j * C::BN);
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (!w.holes) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          float v = __uint_as_float(x[c]) * a.scale_log2;
+          v = c < valid_cols ? v : -INFINITY;
+          x[c] = __float_as_uint(v);
+          mx[c & 3] = fmaxf(mx[c & 3], v);
+        }
+      } else {
+        const int8_t* kseg = a.kv_seg + (w.kv_lo + j * C::BN);
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          float v = __uint_as_float(x[c]) * a.scale_log2;
+          const bool keep = c < valid_cols && kseg[c] == 1;
+          v = keep ? v : -INFINITY;
+          x[c] = __float_as_uint(v);
+          mx[c & 3] = fmaxf(mx[c & 3], v);
+        }
+      }
+      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float m_new = fmaxf(m, m_tile);
+      // Lazy rescaling: keep the stale reference unless the max grew by more than 2^8.
+      const bool rescale = m_new > m + 8.0f;
+      const float m_use = rescale ? m_new : m;
+      const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 128; c += 2) {
+        const float p0 = fast_exp2(__uint_as_float(x[c]) - m_sub);
+        const float p1 = fast_exp2(__uint_as_float(x[c + 1]) - m_sub);
+        sum[(c >> 1) & 3] += p0 + p1;
+        x[c >> 1] = pack_bf16x2(p0, p1);  // packed P overwrites consumed scores in place
+      }
+      // The previous PV must be complete before P is overwritten and before O is rescaled.
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * kPVDone, (g - 1) & 1, abort_flag,
+                                                 a.status));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
+      if (rescale && j > 0) rescale_o_row<D>(t_lane + C::TMEM_O, alpha);
+      l = (rescale ? l * alpha : l) + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+      m = m_use;
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const int k = cb * 32 + ch * 4;
+          st_shared_v4(p_row + cb * C::P_BLK_BYTES + (((uint32_t)ch ^ sw) << 4), x[k], x[k + 1],
+                       x[k + 2], x[k + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bars + 8 * kPFull);
+    }
+    if (!ok) break;
+    float o[D];
+    if (w.n_kv > 0) {
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bars + 8 * kPVDone, (g - 1) & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      load_o_row<D>(t_lane + C::TMEM_O, o);
+    } else {
+#pragma unroll
+      for (int i = 0; i < D; ++i) o[i] = 0.f;
+    }
+    finish_row<D>(a, w, r, m, l, o);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Kernel
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    jagged_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                       const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  using C = Cfg<D>;
+  if (*a.status != 0) return;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  const uint32_t bars = sbase + C::OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars + 8 * (kQFull + i), 1);
+      mbar_init(bars + 8 * (kQEmpty + i), 1);
+      mbar_init(bars + 8 * (kKFull + i), 1);
+      mbar_init(bars + 8 * (kKEmpty + i), 1);
+      mbar_init(bars + 8 * (kVFull + i), 1);
+      mbar_init(bars + 8 * (kVEmpty + i), 1);
+      mbar_init(bars + 8 * (kSFull + i), 1);
+      mbar_init(bars + 8 * (kSEmpty + i), kSoftmaxThreads);
+    }
+    mbar_init(bars + 8 * kPFull, kSoftmaxThreads);
+    mbar_init(bars + 8 * kPVDone, 1);
+    mbar_init(bars + 8 * kDrain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = *a.n_items;
+
+  if (warp == 0) {
+    if (lane == 0) producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag);
+  } else if (warp == 1) {
+    if (lane == 0) mma_role<D>(a, sbase, bars, tmem, n_items, abort_flag);
+  } else {
+    softmax_role<D>(a, sbase, bars, tmem, n_items, abort_flag, warp, lane);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D map over a token-major [rows, H, D] bf16 tensor; box = {swizzle span, 1 head, 128 rows}.
+template <int D>
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int H) {
+  using C = Cfg<D>;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)C::BOX_X, 1u, (cuuint32_t)C::BM};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle sw = C::SW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : C::SW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_32B;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  bool sm100 = false;
+  bool attr_set[4] = {false, false, false, false};
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+int d_index(int d) { return d == 16 ? 0 : d == 32 ? 1 : d == 64 ? 2 : 3; }
+
+template <int D>
+int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void* k,
+                       const void* v, int64_t Tkv, cudaStream_t stream) {
+  using C = Cfg<D>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return JCA_ERR_CUDA;
+  DeviceInfo* info = &g_dev[dev];
+  {
+    std::lock_guard<std::mutex> lock(g_dev_mu);
+    if (info->sms == 0) {
+      int major = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return JCA_ERR_CUDA;
+      info->sm100 = (major == 10);
+      info->sms = sms;
+    }
+    if (!info->sm100) return JCA_ERR_DEVICE;
+    if (!info->attr_set[d_index(D)]) {
+      if (cudaFuncSetAttribute(jagged_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_ALLOC) != cudaSuccess)
+        return JCA_ERR_CUDA;
+      info->attr_set[d_index(D)] = true;
+    }
+  }
+  CUtensorMap tmQ, tmK, tmV;
+  if (!make_map<D>(&tmQ, q, Tq, a.H) || !make_map<D>(&tmK, k, Tkv, a.H) ||
+      !make_map<D>(&tmV, v, Tkv, a.H))
+    return JCA_ERR_CUDA;
+  jagged_attn_kernel<D><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, a);
+  return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+}
+
+int launch_attention(int d, const AttnArgs& a, const void* q, int64_t Tq, const void* k,
+                     const void* v, int64_t Tkv, cudaStream_t stream) {
+  switch (d) {
+    case 16: return launch_attention_d<16>(a, q, Tq, k, v, Tkv, stream);
+    case 32: return launch_attention_d<32>(a, q, Tq, k, v, Tkv, stream);
+    case 64: return launch_attention_d<64>(a, q, Tq, k, v, Tkv, stream);
+    case 128: return launch_attention_d<128>(a, q, Tq, k, v, Tkv, stream);
+    default: return JCA_ERR_HEAD_DIM;
+  }
+}
+
+bool idx_ok(int idx_bits) { return idx_bits == 32 || idx_bits == 64; }
+
+}  // namespace
+}  // namespace jca
+
+using namespace jca;
+
+extern "C" size_t jca_workspace_bytes(int64_t B, int64_t rows, int H, int d_head) {
+  if (B < 0 || rows < 0 || H < 1 || !head_dim_ok(d_head)) return 0;
+  return workspace_layout(B, rows, H).total;
+}
+
+extern "C" int jagged_cand_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                    int out_fp32, const void* offsets,
+                                    const void* candidate_start, const int8_t* seg, int64_t B,
+                                    int64_t T, int H, int d_head, float scale, int idx_bits,
+                                    void* workspace, size_t workspace_bytes, int32_t* status,
+                                    jca_stream_t stream) {
+  if (!idx_ok(idx_bits)) return JCA_ERR_IDX_BITS;
+  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
+  if (B < 0 || T < 0 || H < 1 || H >= 65536 || T >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX)
+    return JCA_ERR_SHAPE;
+  if (B == 0 && T != 0) return JCA_ERR_SHAPE;
+  if (!status || !offsets || !workspace) return JCA_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !out)) return JCA_ERR_NULL;
+  if (B > 0 && !seg && !candidate_start) return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)))
+    return JCA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+  const WorkspaceLayout L = workspace_layout(B, T, H);
+  if (L.max_items >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  if (workspace_bytes < L.total) return JCA_ERR_WORKSPACE;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int8_t* segp = seg ? const_cast<int8_t*>(seg) : reinterpret_cast<int8_t*>(ws + L.seg);
+  int32_t* kv_count = reinterpret_cast<int32_t*>(ws + L.kv_count);
+  int32_t* items = reinterpret_cast<int32_t*>(ws + L.items);
+  int32_t* n_items = reinterpret_cast<int32_t*>(ws + L.n_items);
+  if (!seg && launch_segment_ids(offsets, candidate_start, nullptr, 0, B, T, idx_bits, segp,
+                                 status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  if (launch_bounds(segp, offsets, B, T, idx_bits, ws + L.hist_lo, ws + L.hist_hi, ws + L.cand_lo,
+                    ws + L.cand_hi, kv_count, 0, status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  if (launch_work_queue(offsets, ws + L.hist_lo, ws + L.hist_hi, kv_count, B, T, T, H, idx_bits,
+                        items, L.max_items, n_items, status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  if (T == 0) return JCA_OK;
+  AttnArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.dk = static_cast<const __nv_bfloat16*>(k);
+  a.dv = static_cast<const __nv_bfloat16*>(v);
+  a.q_seg = segp;
+  a.kv_seg = segp;
+  a.out = out;
+  a.items = reinterpret_cast<const int4*>(items);
+  a.n_items = n_items;
+  a.status = status;
+  a.H = H;
+  a.out_fp32 = out_fp32 ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  return launch_attention(d_head, a, q, T, k, v, T, st);
+}
+
+extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const void* own_v,
+                                  const void* cand_offsets, const void* hist_k,
+                                  const void* hist_v, const void* hist_offsets,
+                                  const int8_t* hist_seg, void* out, int out_fp32, int64_t B,
+                                  int64_t Nc, int64_t Th, int H, int d_head, float scale,
+                                  int idx_bits, void* workspace, size_t workspace_bytes,
+                                  int32_t* status, jca_stream_t stream) {
+  if (!idx_ok(idx_bits)) return JCA_ERR_IDX_BITS;
+  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
+  if (B < 0 || Nc < 0 || Th < 0 || H < 1 || H >= 65536 || Nc >= (int64_t)INT_MAX ||
+      Th >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX)
+    return JCA_ERR_SHAPE;
+  if (B == 0 && (Nc != 0 || Th != 0)) return JCA_ERR_SHAPE;
+  if (!status || !cand_offsets || !hist_offsets || !workspace) return JCA_ERR_NULL;
+  if (Nc > 0 && (!cand_q || !own_k || !own_v || !out)) return JCA_ERR_NULL;
+  if (Th > 0 && (!hist_k || !hist_v)) return JCA_ERR_NULL;
+  if (Nc > 0 && (!aligned(cand_q, 16) || !aligned(own_k, 16) || !aligned(own_v, 16) ||
+                 !aligned(out, 16)))
+    return JCA_ERR_ALIGN;
+  if (Th > 0 && (!aligned(hist_k, 16) || !aligned(hist_v, 16))) return JCA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+  const WorkspaceLayout L = workspace_layout(B, Nc, H);
+  if (L.max_items >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  if (workspace_bytes < L.total) return JCA_ERR_WORKSPACE;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* items = reinterpret_cast<int32_t*>(ws + L.items);
+  int32_t* n_items = reinterpret_cast<int32_t*>(ws + L.n_items);
+  const void* kv_lo;
+  const void* kv_hi;
+  const int32_t* kv_count = nullptr;
+  if (hist_seg) {
+    int32_t* cnt = reinterpret_cast<int32_t*>(ws + L.kv_count);
+    if (launch_bounds(hist_seg, hist_offsets, B, Th, idx_bits, ws + L.hist_lo, ws + L.hist_hi,
+                      nullptr, nullptr, cnt, 1, status, st) != cudaSuccess)
+      return JCA_ERR_CUDA;
+    kv_lo = ws + L.hist_lo;
+    kv_hi = ws + L.hist_hi;
+    kv_count = cnt;
+  } else {
+    // Every history row is valid: the key interval of user b is [hist_off[b], hist_off[b+1]).
+    kv_lo = hist_offsets;
+    kv_hi = static_cast<const char*>(hist_offsets) + idx_bits / 8;
+  }
+  if (launch_work_queue(cand_offsets, kv_lo, kv_hi, kv_count, B, Nc, Th, H, idx_bits, items,
+                        L.max_items, n_items, status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  if (Nc == 0) return JCA_OK;
+  AttnArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(cand_q);
+  a.dk = static_cast<const __nv_bfloat16*>(own_k);
+  a.dv = static_cast<const __nv_bfloat16*>(own_v);
+  a.q_seg = nullptr;
+  a.kv_seg = hist_seg;
+  a.out = out;
+  a.items = reinterpret_cast<const int4*>(items);
+  a.n_items = n_items;
+  a.status = status;
+  a.H = H;
+  a.out_fp32 = out_fp32 ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  // With no history rows at all, the key maps are never read; they point at the candidates.
+  const void* kp = Th > 0 ? hist_k : own_k;
+  const void* vp = Th > 0 ? hist_v : own_v;
+  return launch_attention(d_head, a, cand_q, Nc, kp, vp, Th > 0 ? Th : Nc, st);
+}
+
+extern "C" const char* jca_status_string(int code) {
+  switch (code) {
+    case JCA_OK: return "ok";
+    case JCA_ERR_NULL: return "a required pointer is NULL";
+    case JCA_ERR_SHAPE: return "invalid or unsupported size (B, rows, H)";
+    case JCA_ERR_HEAD_DIM: return "d_head must be 16, 32, 64 or 128";
+    case JCA_ERR_ALIGN: return "pointer not aligned (tensors: 16 bytes, workspace: 256 bytes)";
+    case JCA_ERR_IDX_BITS: return "idx_bits must be 32 or 64";
+    case JCA_ERR_WORKSPACE: return "workspace smaller than jca_workspace_bytes()";
+    case JCA_ERR_CUDA: return "a CUDA call failed";
+    case JCA_ERR_DEVICE: return "the current device is not sm_100 (B200)";
+    case JCA_STATUS_BAD_LENGTH: return "negative length or offsets overflow the index type";
+    case JCA_STATUS_BAD_OFFSETS: return "offsets do not start at 0, decrease, or do not end at rows";
+    case JCA_STATUS_BAD_CAND_START: return "candidate_start outside [0, row length]";
+    case JCA_STATUS_BAD_SEG_LAYOUT: return "a history token follows a candidate inside a row";
+    case JCA_STATUS_BAD_SEG_VALUE: return "segment ID outside the allowed values";
+    case JCA_STATUS_QUEUE_OVERFLOW: return "work queue overflow";
+    case JCA_STATUS_TIMEOUT: return "an attention pipeline wait timed out";
+    default: return "unknown code";
+  }
+}

@@ -1,0 +1,431 @@
+// Builder kernels of the jagged batch: offsets from lengths, segment IDs, per-user bounds, and the
+// cost-sorted work queue consumed by the attention kernels. All of them are sync-free: errors go
+// to the device status word and every kernel returns at once when that word is already non-zero.
+#include <climits>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "jca_internal.h"
+
+namespace jca {
+namespace {
+
+__device__ __forceinline__ void set_status(int32_t* status, int code) {
+  atomicCAS(status, 0, (int32_t)code);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Offsets: exclusive prefix sum of lengths ('HSTU scale' tutorial, section 手算 padding 的浪费与
+// offset). One block walks the lengths in chunks of blockDim.x, carrying the running total.
+// ---------------------------------------------------------------------------------------------
+template <typename IdxT>
+__global__ void __launch_bounds__(1024) offsets_kernel(const IdxT* __restrict__ len,
+                                                       IdxT* __restrict__ off, int64_t B,
+                                                       int32_t* status) {
+  if (*status != 0) return;
+  __shared__ long long warp_incl[32];
+  __shared__ long long carry;
+  __shared__ int bad;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nwarps = blockDim.x >> 5;
+  if (tid == 0) {
+    carry = 0;
+    bad = 0;
+    off[0] = (IdxT)0;
+  }
+  __syncthreads();
+  for (int64_t base = 0; base < B; base += blockDim.x) {
+    const int64_t i = base + tid;
+    long long x = 0;
+    if (i < B) {
+      x = (long long)len[i];
+      if (x < 0) bad = 1;
+    }
+    long long v = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      long long n = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += n;
+    }
+    if (lane == 31) warp_incl[wid] = v;
+    __syncthreads();
+    if (wid == 0) {
+      long long w = lane < nwarps ? warp_incl[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        long long n = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += n;
+      }
+      if (lane < nwarps) warp_incl[lane] = w;
+    }
+    __syncthreads();
+    const long long incl = v + (wid > 0 ? warp_incl[wid - 1] : 0) + carry;
+    if (i < B) {
+      off[i + 1] = (IdxT)incl;
+      if (sizeof(IdxT) == 4 && incl > (long long)INT_MAX) bad = 1;
+    }
+    __syncthreads();
+    if (tid == (int)blockDim.x - 1) carry = incl;
+    __syncthreads();
+  }
+  if (tid == 0 && bad) set_status(status, JCA_STATUS_BAD_LENGTH);
+}
+
+// Offsets of user b must satisfy 0 <= off[b] <= off[b+1] <= rows, off[0] = 0, off[B] = rows.
+__device__ __forceinline__ bool row_ok(long long s, long long e, int64_t b, int64_t B,
+                                       int64_t rows) {
+  return s >= 0 && s <= e && e <= rows && (b > 0 || s == 0) && (b < B - 1 || e == rows);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Segment IDs (候选隔离注意力掩码, section 段 ID：掩码的表达方式): one block per user row.
+// ---------------------------------------------------------------------------------------------
+template <typename IdxT>
+__global__ void segment_ids_kernel(const IdxT* __restrict__ off, const IdxT* __restrict__ cs,
+                                   const uint8_t* __restrict__ valid, int attend_padded_history,
+                                   int64_t B, int64_t T, int8_t* __restrict__ seg,
+                                   int32_t* status) {
+  if (*status != 0) return;
+  for (int64_t b = blockIdx.x; b < B; b += gridDim.x) {
+    const long long s = (long long)off[b], e = (long long)off[b + 1];
+    if (!row_ok(s, e, b, B, T)) {
+      if (threadIdx.x == 0) set_status(status, JCA_STATUS_BAD_OFFSETS);
+      continue;
+    }
+    const long long c = (long long)cs[b];
+    if (c < 0 || c > e - s) {
+      if (threadIdx.x == 0) set_status(status, JCA_STATUS_BAD_CAND_START);
+      continue;
+    }
+    for (long long i = threadIdx.x; i < e - s; i += blockDim.x) {
+      const bool is_candidate = i >= c;
+      bool ok = valid ? (valid[s + i] != 0) : true;
+      if (attend_padded_history) ok = ok || !is_candidate;
+      seg[s + i] = ok ? (is_candidate ? (int8_t)-1 : (int8_t)1) : (int8_t)0;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Bounds (候选隔离注意力掩码, section 段 ID：掩码的表达方式, bounds_from_segment_ids): one block per
+// user row reduces first/last positions of segment 1 and -1 and counts the segment-1 tokens.
+// ---------------------------------------------------------------------------------------------
+template <typename IdxT>
+__global__ void bounds_kernel(const int8_t* __restrict__ seg, const IdxT* __restrict__ off,
+                              int64_t B, int64_t T, IdxT* __restrict__ hist_lo,
+                              IdxT* __restrict__ hist_hi, IdxT* __restrict__ cand_lo,
+                              IdxT* __restrict__ cand_hi, int32_t* __restrict__ kv_count,
+                              int history_only, int32_t* status) {
+  if (*status != 0) return;
+  __shared__ long long s_hmin, s_hmax, s_cmin, s_cmax;
+  __shared__ int s_count, s_bad;
+  for (int64_t b = blockIdx.x; b < B; b += gridDim.x) {
+    const long long s = (long long)off[b], e = (long long)off[b + 1];
+    if (!row_ok(s, e, b, B, T)) {
+      if (threadIdx.x == 0) set_status(status, JCA_STATUS_BAD_OFFSETS);
+      continue;
+    }
+    if (threadIdx.x == 0) {
+      s_hmin = LLONG_MAX;
+      s_hmax = -1;
+      s_cmin = LLONG_MAX;
+      s_cmax = -1;
+      s_count = 0;
+      s_bad = 0;
+    }
+    __syncthreads();
+    long long hmin = LLONG_MAX, hmax = -1, cmin = LLONG_MAX, cmax = -1;
+    int count = 0, bad = 0;
+    for (long long i = threadIdx.x; i < e - s; i += blockDim.x) {
+      const int x = seg[s + i];
+      if (x == 1) {
+        hmin = min(hmin, i);
+        hmax = max(hmax, i);
+        ++count;
+      } else if (x == -1) {
+        if (history_only) bad = 1;
+        cmin = min(cmin, i);
+        cmax = max(cmax, i);
+      } else if (x != 0) {
+        bad = 1;
+      }
+    }
+    if (hmax >= 0) {
+      atomicMin(&s_hmin, hmin);
+      atomicMax(&s_hmax, hmax);
+    }
+    if (cmax >= 0) {
+      atomicMin(&s_cmin, cmin);
+      atomicMax(&s_cmax, cmax);
+    }
+    if (count) atomicAdd(&s_count, count);
+    if (bad) s_bad = 1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      if (s_bad) {
+        set_status(status, JCA_STATUS_BAD_SEG_VALUE);
+      } else if (s_hmax >= 0 && s_cmax >= 0 && s_hmax > s_cmin) {
+        set_status(status, JCA_STATUS_BAD_SEG_LAYOUT);
+      }
+      const bool has_h = s_hmax >= 0, has_c = s_cmax >= 0;
+      hist_lo[b] = (IdxT)(has_h ? s + s_hmin : s);
+      hist_hi[b] = (IdxT)(has_h ? s + s_hmax + 1 : s);
+      if (cand_lo) cand_lo[b] = (IdxT)(has_c ? s + s_cmin : e);
+      if (cand_hi) cand_hi[b] = (IdxT)(has_c ? s + s_cmax + 1 : e);
+      if (kv_count) kv_count[b] = s_count;
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Work queue: counting sort of (user, head, query tile) items by key-tile count, descending.
+// A single block: pass 1 validates and histograms, a block scan turns bucket sizes into start
+// positions (largest cost first), pass 2 emits each user's items contiguously (head-major, then
+// query tile) at a position claimed with an atomic on its bucket cursor.
+// ---------------------------------------------------------------------------------------------
+template <typename IdxT>
+__global__ void __launch_bounds__(1024) work_queue_kernel(
+    const IdxT* __restrict__ qoff, const IdxT* __restrict__ kvlo, const IdxT* __restrict__ kvhi,
+    const int32_t* __restrict__ kv_count, int64_t B, int64_t q_rows, int64_t kv_rows, int H,
+    int4* __restrict__ items, int64_t max_items, int32_t* n_items, int32_t* status) {
+  __shared__ unsigned long long s_cnt[kQueueBuckets];
+  __shared__ unsigned long long s_cursor[kQueueBuckets];
+  __shared__ unsigned long long s_warp[32];
+  __shared__ unsigned long long s_total;
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (*status != 0) {
+    if (tid == 0) *n_items = 0;
+    return;
+  }
+  for (int i = tid; i < kQueueBuckets; i += blockDim.x) s_cnt[i] = 0;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  for (int64_t b = tid; b < B; b += blockDim.x) {
+    const long long s = (long long)qoff[b], e = (long long)qoff[b + 1];
+    const long long lo = (long long)kvlo[b], hi = (long long)kvhi[b];
+    if (!row_ok(s, e, b, B, q_rows) || lo < 0 || lo > hi || hi > kv_rows) {
+      s_bad = 1;
+      continue;
+    }
+    const long long nq = (e - s + kTileM - 1) / kTileM;
+    const long long nkv = (hi - lo + kTileN - 1) / kTileN;
+    const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
+    if (nq) atomicAdd(&s_cnt[key], (unsigned long long)(nq * H));
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      set_status(status, JCA_STATUS_BAD_OFFSETS);
+      *n_items = 0;
+    }
+    return;
+  }
+  // Exclusive scan over buckets in descending key order (thread t <-> bucket NB-1-t).
+  static_assert(kQueueBuckets == 1024, "scan assumes one bucket per thread");
+  const int kb = kQueueBuckets - 1 - tid;
+  const unsigned long long val = s_cnt[kb];
+  unsigned long long v = val;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    unsigned long long w = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      unsigned long long n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const unsigned long long incl = v + (wid > 0 ? s_warp[wid - 1] : 0ull);
+  s_cursor[kb] = incl - val;
+  if (tid == kQueueBuckets - 1) s_total = incl;
+  __syncthreads();
+  if (s_total > (unsigned long long)max_items) {
+    if (tid == 0) {
+      set_status(status, JCA_STATUS_QUEUE_OVERFLOW);
+      *n_items = 0;
+    }
+    return;
+  }
+  for (int64_t b = tid; b < B; b += blockDim.x) {
+    const long long s = (long long)qoff[b], e = (long long)qoff[b + 1];
+    const long long lo = (long long)kvlo[b], hi = (long long)kvhi[b];
+    const long long nq = (e - s + kTileM - 1) / kTileM;
+    if (nq == 0) continue;
+    const long long nkv = (hi - lo + kTileN - 1) / kTileN;
+    const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
+    const unsigned long long pos = atomicAdd(&s_cursor[key], (unsigned long long)(nq * H));
+    const int holes = (kv_count != nullptr && (long long)kv_count[b] != hi - lo) ? 1 : 0;
+    const int w = (int)(hi - lo) | (holes << 31);
+    for (int h = 0; h < H; ++h) {
+      for (long long t = 0; t < nq; ++t) {
+        const long long row0 = s + t * kTileM;
+        const int rows = (int)min((long long)kTileM, e - row0);
+        items[pos + (unsigned long long)h * nq + t] = make_int4((int)row0, h * 256 + rows, (int)lo, w);
+      }
+    }
+  }
+  if (tid == 0) *n_items = (int32_t)s_total;
+}
+
+inline int grid_for_rows(int64_t B) { return (int)(B < (1 << 20) ? B : (1 << 20)); }
+
+}  // namespace
+
+int64_t max_work_items(int64_t B, int64_t rows, int H) {
+  return ((rows + kTileM - 1) / kTileM + B) * (int64_t)H;
+}
+
+WorkspaceLayout workspace_layout(int64_t B, int64_t rows, int H) {
+  WorkspaceLayout w;
+  size_t p = 0;
+  w.seg = p;
+  p = align_up(p + (size_t)rows, 256);
+  w.hist_lo = p;
+  p = align_up(p + 8 * (size_t)B, 256);
+  w.hist_hi = p;
+  p = align_up(p + 8 * (size_t)B, 256);
+  w.cand_lo = p;
+  p = align_up(p + 8 * (size_t)B, 256);
+  w.cand_hi = p;
+  p = align_up(p + 8 * (size_t)B, 256);
+  w.kv_count = p;
+  p = align_up(p + 4 * (size_t)B, 256);
+  w.max_items = max_work_items(B, rows, H);
+  w.items = p;
+  p = align_up(p + 16 * (size_t)w.max_items, 256);
+  w.n_items = p;
+  p = align_up(p + 4, 256);
+  w.total = p;
+  return w;
+}
+
+cudaError_t launch_segment_ids(const void* offsets, const void* cand_start, const uint8_t* valid,
+                               int attend_padded_history, int64_t B, int64_t T, int idx_bits,
+                               int8_t* seg, int32_t* status, cudaStream_t stream) {
+  if (B == 0) return cudaSuccess;
+  const int grid = grid_for_rows(B);
+  if (idx_bits == 32)
+    segment_ids_kernel<int32_t><<<grid, 256, 0, stream>>>(
+        (const int32_t*)offsets, (const int32_t*)cand_start, valid, attend_padded_history, B, T,
+        seg, status);
+  else
+    segment_ids_kernel<int64_t><<<grid, 256, 0, stream>>>(
+        (const int64_t*)offsets, (const int64_t*)cand_start, valid, attend_padded_history, B, T,
+        seg, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bounds(const int8_t* seg, const void* offsets, int64_t B, int64_t T,
+                          int idx_bits, void* hist_lo, void* hist_hi, void* cand_lo,
+                          void* cand_hi, int32_t* kv_count, int history_only, int32_t* status,
+                          cudaStream_t stream) {
+  if (B == 0) return cudaSuccess;
+  const int grid = grid_for_rows(B);
+  if (idx_bits == 32)
+    bounds_kernel<int32_t><<<grid, 256, 0, stream>>>(
+        seg, (const int32_t*)offsets, B, T, (int32_t*)hist_lo, (int32_t*)hist_hi,
+        (int32_t*)cand_lo, (int32_t*)cand_hi, kv_count, history_only, status);
+  else
+    bounds_kernel<int64_t><<<grid, 256, 0, stream>>>(
+        seg, (const int64_t*)offsets, B, T, (int64_t*)hist_lo, (int64_t*)hist_hi,
+        (int64_t*)cand_lo, (int64_t*)cand_hi, kv_count, history_only, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_work_queue(const void* q_offsets, const void* kv_lo, const void* kv_hi,
+                              const int32_t* kv_count, int64_t B, int64_t q_rows,
+                              int64_t kv_rows, int H, int idx_bits, int32_t* items,
+                              int64_t max_items, int32_t* n_items, int32_t* status,
+                              cudaStream_t stream) {
+  if (idx_bits == 32)
+    work_queue_kernel<int32_t><<<1, kQueueBuckets, 0, stream>>>(
+        (const int32_t*)q_offsets, (const int32_t*)kv_lo, (const int32_t*)kv_hi, kv_count, B,
+        q_rows, kv_rows, H, (int4*)items, max_items, n_items, status);
+  else
+    work_queue_kernel<int64_t><<<1, kQueueBuckets, 0, stream>>>(
+        (const int64_t*)q_offsets, (const int64_t*)kv_lo, (const int64_t*)kv_hi, kv_count, B,
+        q_rows, kv_rows, H, (int4*)items, max_items, n_items, status);
+  return cudaGetLastError();
+}
+
+}  // namespace jca
+
+using namespace jca;
+
+extern "C" int jca_offsets_from_lengths(const void* lengths, void* offsets, int64_t B,
+                                        int idx_bits, int32_t* status, jca_stream_t stream) {
+  if (idx_bits != 32 && idx_bits != 64) return JCA_ERR_IDX_BITS;
+  if (B < 0 || B >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  if (!offsets || !status || (B > 0 && !lengths)) return JCA_ERR_NULL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (idx_bits == 32)
+    offsets_kernel<int32_t><<<1, 1024, 0, s>>>((const int32_t*)lengths, (int32_t*)offsets, B,
+                                                status);
+  else
+    offsets_kernel<int64_t><<<1, 1024, 0, s>>>((const int64_t*)lengths, (int64_t*)offsets, B,
+                                                status);
+  return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+}
+
+extern "C" int jca_build_segment_ids(const void* offsets, const void* candidate_start,
+                                     const uint8_t* valid_mask, int attend_padded_history,
+                                     int64_t B, int64_t T, int idx_bits, int8_t* seg,
+                                     int32_t* status, jca_stream_t stream) {
+  if (idx_bits != 32 && idx_bits != 64) return JCA_ERR_IDX_BITS;
+  if (B < 0 || T < 0 || T >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  if (B == 0 && T != 0) return JCA_ERR_SHAPE;
+  if (!status || !offsets || (B > 0 && !candidate_start) || (T > 0 && !seg)) return JCA_ERR_NULL;
+  cudaError_t e = launch_segment_ids(offsets, candidate_start, valid_mask, attend_padded_history,
+                                     B, T, idx_bits, seg, status,
+                                     reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+}
+
+extern "C" int jca_bounds_from_segment_ids(const int8_t* seg, const void* offsets, int64_t B,
+                                           int64_t T, int idx_bits, void* hist_lo, void* hist_hi,
+                                           void* cand_lo, void* cand_hi, int32_t* status,
+                                           jca_stream_t stream) {
+  if (idx_bits != 32 && idx_bits != 64) return JCA_ERR_IDX_BITS;
+  if (B < 0 || T < 0 || T >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  if (B == 0 && T != 0) return JCA_ERR_SHAPE;
+  if (!status || !offsets || (T > 0 && !seg)) return JCA_ERR_NULL;
+  if (B > 0 && (!hist_lo || !hist_hi || !cand_lo || !cand_hi)) return JCA_ERR_NULL;
+  cudaError_t e = launch_bounds(seg, offsets, B, T, idx_bits, hist_lo, hist_hi, cand_lo, cand_hi,
+                                nullptr, 0, status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+}
+
+extern "C" int jca_build_work_queue(const void* q_offsets, const void* kv_lo, const void* kv_hi,
+                                    const int32_t* kv_count, int64_t B, int64_t q_rows,
+                                    int64_t kv_rows, int H, int idx_bits, int32_t* items,
+                                    int64_t max_items, int32_t* n_items, int32_t* status,
+                                    jca_stream_t stream) {
+  if (idx_bits != 32 && idx_bits != 64) return JCA_ERR_IDX_BITS;
+  if (B < 0 || q_rows < 0 || kv_rows < 0 || H < 1 || H >= 65536 || max_items < 0 ||
+      max_items >= (int64_t)INT_MAX || q_rows >= (int64_t)INT_MAX ||
+      kv_rows >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX)
+    return JCA_ERR_SHAPE;
+  if (B == 0 && q_rows != 0) return JCA_ERR_SHAPE;
+  if (!q_offsets || !n_items || !status || (B > 0 && (!kv_lo || !kv_hi)) ||
+      (max_items > 0 && !items))
+    return JCA_ERR_NULL;
+  if (items && !aligned(items, 16)) return JCA_ERR_ALIGN;
+  cudaError_t e = launch_work_queue(q_offsets, kv_lo, kv_hi, kv_count, B, q_rows, kv_rows, H,
+                                    idx_bits, items, max_items, n_items, status,
+                                    reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+}
+
+extern "C" int64_t jca_max_work_items(int64_t B, int64_t rows, int H) {
+  if (B < 0 || rows < 0 || H < 1) return 0;
+  return max_work_items(B, rows, H);
+}

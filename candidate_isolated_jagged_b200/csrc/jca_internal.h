@@ -1,0 +1,59 @@
+// Host-side pieces shared by the translation units of libjca.so (not part of the public ABI).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "jca.h"
+
+namespace jca {
+
+constexpr int kTileM = 128;          // query rows per work item
+constexpr int kTileN = 128;          // keys per key tile
+constexpr int kQueueBuckets = 1024;  // cost buckets of the work-queue counting sort
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+inline bool aligned(const void* p, size_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+
+inline bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+int64_t max_work_items(int64_t B, int64_t rows, int H);
+
+// Carve-up of the caller's workspace (all offsets 256-byte aligned).
+struct WorkspaceLayout {
+  size_t seg = 0;        // int8  [rows]   segment IDs built from candidate starts
+  size_t hist_lo = 0;    // int64 [B]      (entries in the caller's idx type)
+  size_t hist_hi = 0;
+  size_t cand_lo = 0;
+  size_t cand_hi = 0;
+  size_t kv_count = 0;   // int32 [B]      segment-1 tokens per user
+  size_t items = 0;      // int4  [max_items]
+  size_t n_items = 0;    // int32 [1]
+  size_t total = 0;
+  int64_t max_items = 0;
+};
+
+WorkspaceLayout workspace_layout(int64_t B, int64_t rows, int H);
+
+// Builder launches (no argument checks; callers validate first).
+cudaError_t launch_segment_ids(const void* offsets, const void* cand_start, const uint8_t* valid,
+                               int attend_padded_history, int64_t B, int64_t T, int idx_bits,
+                               int8_t* seg, int32_t* status, cudaStream_t stream);
+
+// history_only != 0: segment -1 is invalid (a frozen history may hold only 1 and 0).
+cudaError_t launch_bounds(const int8_t* seg, const void* offsets, int64_t B, int64_t T,
+                          int idx_bits, void* hist_lo, void* hist_hi, void* cand_lo,
+                          void* cand_hi, int32_t* kv_count, int history_only, int32_t* status,
+                          cudaStream_t stream);
+
+cudaError_t launch_work_queue(const void* q_offsets, const void* kv_lo, const void* kv_hi,
+                              const int32_t* kv_count, int64_t B, int64_t q_rows,
+                              int64_t kv_rows, int H, int idx_bits, int32_t* items,
+                              int64_t max_items, int32_t* n_items, int32_t* status,
+                              cudaStream_t stream);
+
+}  // namespace jca

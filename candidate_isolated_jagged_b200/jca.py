@@ -1,0 +1,233 @@
+"""Thin ctypes binding over libjca.so (the C ABI declared in include/jca.h).
+
+Argument marshalling only: tensors are passed as device pointers with their sizes, the stream is
+torch's current CUDA stream, and every step of the computation runs in the library's kernels.
+PyTorch allocates the outputs, the workspace and the status word. There is no CPU fallback: when
+the library is missing, ``lib()`` raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libjca.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "jca.h")
+
+_lib = None
+
+c_i32, c_i64, c_f32, c_sz, c_vp = (ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t,
+                                   ctypes.c_void_p)
+
+_SIGNATURES = {
+    "jca_status_string": (ctypes.c_char_p, [c_i32]),
+    "jca_offsets_from_lengths": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_vp, c_vp]),
+    "jca_build_segment_ids": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i64, c_i64, c_i32, c_vp, c_vp,
+                                      c_vp]),
+    "jca_bounds_from_segment_ids": (c_i32, [c_vp, c_vp, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp,
+                                            c_vp, c_vp, c_vp]),
+    "jca_build_work_queue": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i32, c_i32,
+                                     c_vp, c_i64, c_vp, c_vp, c_vp]),
+    "jca_max_work_items": (c_i64, [c_i64, c_i64, c_i32]),
+    "jca_workspace_bytes": (c_sz, [c_i64, c_i64, c_i32, c_i32]),
+    "jagged_cand_attn_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_i64, c_i64,
+                                     c_i32, c_i32, c_f32, c_i32, c_vp, c_sz, c_vp, c_vp]),
+    "cand_only_attn_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
+                                   c_i64, c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp, c_sz,
+                                   c_vp, c_vp]),
+}
+
+
+class JcaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = int(code)
+        super().__init__(f"{where}: {status_string(code)} (code {code})")
+
+
+def lib(path: Optional[str] = None):
+    """Load libjca.so (once). Raises when it is missing: there is no fallback."""
+    global _lib
+    if path is not None:
+        return _load(path)
+    if _lib is None:
+        _lib = _load(LIB_PATH)
+    return _lib
+
+
+def _load(path: str):
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           f"`python -m candidate_isolated_jagged_b200.build`")
+    L = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+def header_functions(path: str = HEADER_PATH):
+    """Names of the functions declared in include/jca.h."""
+    text = open(path).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*([a-z_0-9]+)\s*\(", text,
+                                 flags=re.M)))
+
+
+def status_string(code: int) -> str:
+    return lib().jca_status_string(int(code)).decode()
+
+
+# ------------------------------------------------------------------------------------------------
+# Marshalling helpers
+# ------------------------------------------------------------------------------------------------
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return ctypes.c_void_p(handle)
+
+
+def _idx_bits(t: torch.Tensor) -> int:
+    if t.dtype == torch.int32:
+        return 32
+    if t.dtype == torch.int64:
+        return 64
+    raise TypeError(f"index tensors must be int32 or int64, got {t.dtype}")
+
+
+def _check(code: int, where: str) -> int:
+    if code < 0:
+        raise JcaError(code, where)
+    return code
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check_status(status: torch.Tensor, where: str = "device") -> None:
+    """Read the device status word (synchronises) and raise on a recorded data error."""
+    code = int(status.item())
+    if code != 0:
+        raise JcaError(code, where)
+
+
+# ------------------------------------------------------------------------------------------------
+# Entry points (same names as the C ABI)
+# ------------------------------------------------------------------------------------------------
+
+def jca_offsets_from_lengths(lengths: torch.Tensor, offsets: torch.Tensor, status: torch.Tensor,
+                             stream=None) -> int:
+    return _check(lib().jca_offsets_from_lengths(_ptr(lengths), _ptr(offsets), lengths.numel(),
+                                                 _idx_bits(lengths), _ptr(status), _stream(stream)),
+                  "jca_offsets_from_lengths")
+
+
+def jca_build_segment_ids(offsets, candidate_start, valid_mask, attend_padded_history: bool,
+                          seg: torch.Tensor, status: torch.Tensor, stream=None) -> int:
+    B = offsets.numel() - 1
+    return _check(lib().jca_build_segment_ids(
+        _ptr(offsets), _ptr(candidate_start), _ptr(valid_mask), int(bool(attend_padded_history)),
+        B, seg.numel(), _idx_bits(offsets), _ptr(seg), _ptr(status), _stream(stream)),
+        "jca_build_segment_ids")
+
+
+def jca_bounds_from_segment_ids(seg, offsets, hist_lo, hist_hi, cand_lo, cand_hi, status,
+                                stream=None) -> int:
+    B = offsets.numel() - 1
+    return _check(lib().jca_bounds_from_segment_ids(
+        _ptr(seg), _ptr(offsets), B, seg.numel(), _idx_bits(offsets), _ptr(hist_lo), _ptr(hist_hi),
+        _ptr(cand_lo), _ptr(cand_hi), _ptr(status), _stream(stream)), "jca_bounds_from_segment_ids")
+
+
+def jca_build_work_queue(q_offsets, kv_lo, kv_hi, kv_count, q_rows: int, kv_rows: int, H: int,
+                         items: torch.Tensor, n_items: torch.Tensor, status, stream=None) -> int:
+    B = q_offsets.numel() - 1
+    return _check(lib().jca_build_work_queue(
+        _ptr(q_offsets), _ptr(kv_lo), _ptr(kv_hi), _ptr(kv_count), B, int(q_rows), int(kv_rows),
+        int(H), _idx_bits(q_offsets), _ptr(items), items.numel() // 4, _ptr(n_items), _ptr(status),
+        _stream(stream)), "jca_build_work_queue")
+
+
+def jca_max_work_items(B: int, rows: int, H: int) -> int:
+    return int(lib().jca_max_work_items(int(B), int(rows), int(H)))
+
+
+def jca_workspace_bytes(B: int, rows: int, H: int, d_head: int) -> int:
+    return int(lib().jca_workspace_bytes(int(B), int(rows), int(H), int(d_head)))
+
+
+def jagged_cand_attn_fwd(q, k, v, out, offsets, candidate_start=None, seg=None, scale: float = 0.0,
+                         workspace: Optional[torch.Tensor] = None,
+                         status: Optional[torch.Tensor] = None, stream=None) -> int:
+    T, H, d = q.shape
+    B = offsets.numel() - 1
+    if workspace is None:
+        workspace = torch.empty(jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=q.device)
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().jagged_cand_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), _ptr(candidate_start),
+        _ptr(seg), B, T, H, d, float(scale), _idx_bits(offsets), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream)), "jagged_cand_attn_fwd")
+
+
+def cand_only_attn_fwd(cand_q, own_k, own_v, cand_offsets, hist_k, hist_v, hist_offsets, out,
+                       hist_seg=None, scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                       status: Optional[torch.Tensor] = None, stream=None) -> int:
+    Nc, H, d = cand_q.shape
+    Th = hist_k.shape[0]
+    B = cand_offsets.numel() - 1
+    if workspace is None:
+        workspace = torch.empty(jca_workspace_bytes(B, Nc, H, d), dtype=torch.uint8,
+                                device=cand_q.device)
+    if status is None:
+        status = new_status(cand_q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().cand_only_attn_fwd(
+        _ptr(cand_q), _ptr(own_k), _ptr(own_v), _ptr(cand_offsets), _ptr(hist_k), _ptr(hist_v),
+        _ptr(hist_offsets), _ptr(hist_seg), _ptr(out), out_fp32, B, Nc, Th, H, d, float(scale),
+        _idx_bits(cand_offsets), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream)), "cand_only_attn_fwd")
+
+
+def jca_status_string(code: int) -> str:
+    return status_string(code)
+
+
+# ------------------------------------------------------------------------------------------------
+# Convenience: allocate outputs with torch, call, check the status word
+# ------------------------------------------------------------------------------------------------
+
+def attention(q, k, v, offsets, candidate_start=None, seg=None, out_fp32: bool = False,
+              scale: float = 0.0, check: bool = True) -> torch.Tensor:
+    out = torch.empty(q.shape, dtype=torch.float32 if out_fp32 else torch.bfloat16, device=q.device)
+    status = new_status(q.device)
+    jagged_cand_attn_fwd(q, k, v, out, offsets, candidate_start, seg, scale, status=status)
+    if check:
+        check_status(status, "jagged_cand_attn_fwd")
+    return out
+
+
+def cand_only(cand_q, own_k, own_v, cand_offsets, hist_k, hist_v, hist_offsets, hist_seg=None,
+              out_fp32: bool = False, scale: float = 0.0, check: bool = True) -> torch.Tensor:
+    out = torch.empty(cand_q.shape, dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                      device=cand_q.device)
+    status = new_status(cand_q.device)
+    cand_only_attn_fwd(cand_q, own_k, own_v, cand_offsets, hist_k, hist_v, hist_offsets, out,
+                       hist_seg, scale, status=status)
+    if check:
+        check_status(status, "cand_only_attn_fwd")
+    return out

@@ -1,0 +1,198 @@
+/*
+ * jca.h — C ABI of libjca.so: jagged, candidate-isolated softmax attention on NVIDIA B200 (sm_100a).
+ *
+ * A jagged batch holds B user rows laid out as [user prefix | history | candidates]
+ * (候选隔离注意力掩码, section 为什么需要它), packed back to back and described by offsets
+ * ('HSTU scale' tutorial, section 手算 padding 的浪费与 offset). Every token carries a segment ID:
+ * 1 = prefix/history, -1 = candidate, 0 = padding (候选隔离注意力掩码, section 段 ID：掩码的表达方式).
+ * Prefix and history attend to each other bidirectionally and never to candidates; each candidate
+ * attends to its user's prefix, history and itself; no position reads across a user boundary.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Memory.     Every pointer argument is DEVICE memory owned by the caller; the library never
+ *             allocates device memory and never frees what it is given. Scratch space, where an
+ *             entry point needs it, is the caller's `workspace` of at least
+ *             jca_workspace_bytes(...) bytes, 256-byte aligned.
+ * Layout.     Q/K/V/out are token-major [rows, H, d_head] (row stride H*d_head elements), bf16
+ *             unless stated; offsets/lengths/candidate starts/bounds are int32 or int64 as chosen
+ *             by `idx_bits` (32 or 64); segment IDs are int8; the padding mask is uint8 (1 = real).
+ * Streams.    Every call only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
+ *             stream) and returns without synchronising the host.
+ * Host errors.  Argument errors are detected before anything is enqueued and returned as a
+ *             negative JCA_ERR_* code; nothing is written then.
+ * Device errors. Data errors found on the device (bad offsets, bad candidate starts, a history
+ *             token after a candidate, a pipeline wait that timed out) are recorded as a positive
+ *             JCA_STATUS_* code in *status (int32, device memory). The first error wins. Every
+ *             kernel of the library reads *status when it starts and does nothing when it is
+ *             non-zero, so an error stops every later call that shares the status word. The caller
+ *             zeroes *status before the first call and reads it back when convenient.
+ * Limits.     rows < 2^31 per tensor; H >= 1; d_head in {16, 32, 64, 128}; pointers of Q/K/V/out
+ *             16-byte aligned.
+ * Numerics.   bf16 inputs, fp32 accumulation and fp32 online softmax; `scale` <= 0 selects
+ *             1/sqrt(d_head). Inputs are assumed finite.
+ * Device.     sm_100a (B200). On another device the attention entry points return JCA_ERR_DEVICE.
+ */
+#ifndef JCA_H_
+#define JCA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* jca_stream_t;
+
+enum jca_code {
+  JCA_OK = 0,
+  /* host-side argument errors (return values) */
+  JCA_ERR_NULL = -1,        /* a required pointer is NULL */
+  JCA_ERR_SHAPE = -2,       /* B < 0, rows < 0, H < 1, or a size beyond the limits */
+  JCA_ERR_HEAD_DIM = -3,    /* d_head not in {16, 32, 64, 128} */
+  JCA_ERR_ALIGN = -4,       /* a pointer is not 16-byte aligned (workspace: 256-byte) */
+  JCA_ERR_IDX_BITS = -5,    /* idx_bits not 32 or 64 */
+  JCA_ERR_WORKSPACE = -6,   /* workspace smaller than jca_workspace_bytes(...) */
+  JCA_ERR_CUDA = -7,        /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
+  JCA_ERR_DEVICE = -8,      /* current device is not sm_100 */
+  /* device-side data errors (written to *status) */
+  JCA_STATUS_BAD_LENGTH = 1,     /* a sequence length is negative, or offsets overflow int32 */
+  JCA_STATUS_BAD_OFFSETS = 2,    /* offsets[0] != 0, offsets decrease, or offsets[B] != rows */
+  JCA_STATUS_BAD_CAND_START = 3, /* candidate_start[b] outside [0, row length] */
+  JCA_STATUS_BAD_SEG_LAYOUT = 4, /* a segment-1 token follows a candidate inside a row */
+  JCA_STATUS_BAD_SEG_VALUE = 5,  /* a segment ID outside {-1, 0, 1} */
+  JCA_STATUS_QUEUE_OVERFLOW = 6, /* more work items than the workspace bound (internal) */
+  JCA_STATUS_TIMEOUT = 16        /* a pipeline wait in the attention kernel gave up */
+};
+
+/* Text of a JCA_ERR_* or JCA_STATUS_* code (static storage; never NULL). */
+const char* jca_status_string(int code);
+
+/*
+ * Offsets of a ragged batch: offsets[0] = 0 and offsets[b+1] = offsets[b] + lengths[b]
+ * ('HSTU scale' tutorial, section 手算 padding 的浪费与 offset: sequence b is
+ * values[offsets[b]:offsets[b+1]]).
+ *   lengths  [B] int32/int64 (idx_bits), read;   offsets [B+1] same type, written.
+ *   B >= 0 (B = 0 writes offsets[0] = 0).
+ * Device errors: a negative length, or (idx_bits = 32) a total beyond INT32_MAX ->
+ * JCA_STATUS_BAD_LENGTH; offsets are then unspecified.
+ */
+int jca_offsets_from_lengths(const void* lengths, void* offsets, int64_t B, int idx_bits,
+                             int32_t* status, jca_stream_t stream);
+
+/*
+ * Segment IDs of every packed token (候选隔离注意力掩码, section 段 ID：掩码的表达方式):
+ * for position idx of user row b (row-relative), is_candidate = idx >= candidate_start[b];
+ * valid = valid_mask[token] (or valid_mask[token] OR NOT is_candidate when
+ * attend_padded_history != 0); seg = valid ? (is_candidate ? -1 : 1) : 0.
+ *   offsets [B+1] and candidate_start [B] (row-relative) in the idx_bits type, read.
+ *   valid_mask [T] uint8 or NULL (NULL = every token is real), read.
+ *   seg [T] int8, written.
+ * Device errors: offsets not starting at 0, decreasing or not ending at T ->
+ * JCA_STATUS_BAD_OFFSETS; candidate_start[b] outside [0, offsets[b+1]-offsets[b]] ->
+ * JCA_STATUS_BAD_CAND_START.
+ */
+int jca_build_segment_ids(const void* offsets, const void* candidate_start,
+                          const uint8_t* valid_mask, int attend_padded_history,
+                          int64_t B, int64_t T, int idx_bits, int8_t* seg,
+                          int32_t* status, jca_stream_t stream);
+
+/*
+ * Per-user history and candidate intervals (候选隔离注意力掩码, section 段 ID：掩码的表达方式,
+ * bounds_from_segment_ids): [hist_lo, hist_hi) runs from the first to one past the last
+ * segment-1 token of the row, [cand_lo, cand_hi) from the first to one past the last
+ * segment -1 token; indices are absolute packed positions. An empty history gives
+ * hist_lo = hist_hi = offsets[b]; no candidate gives cand_lo = cand_hi = offsets[b+1]
+ * (a reading: the pages do not state the empty convention).
+ *   seg [T] int8 and offsets [B+1] (idx_bits type), read.
+ *   hist_lo, hist_hi, cand_lo, cand_hi [B] in the idx_bits type, written.
+ * Device errors: bad offsets -> JCA_STATUS_BAD_OFFSETS; a segment ID outside {-1,0,1} ->
+ * JCA_STATUS_BAD_SEG_VALUE; a segment-1 token after a candidate inside one row ->
+ * JCA_STATUS_BAD_SEG_LAYOUT.
+ */
+int jca_bounds_from_segment_ids(const int8_t* seg, const void* offsets, int64_t B, int64_t T,
+                                int idx_bits, void* hist_lo, void* hist_hi, void* cand_lo,
+                                void* cand_hi, int32_t* status, jca_stream_t stream);
+
+/*
+ * Work queue of the attention kernels: one item per (user b, head h, 128-row query tile t),
+ * ordered by cost (the number of 128-key tiles over the user's key interval), largest first,
+ * so that a persistent kernel taking items in order approximates longest-processing-time-first.
+ * Items of equal cost may come in any order.
+ *   q_offsets [B+1], kv_lo [B], kv_hi [B] in the idx_bits type, read (absolute rows; the key
+ *   interval of user b is [kv_lo[b], kv_hi[b])).
+ *   kv_count [B] int32 or NULL: number of valid keys inside the interval; when it differs from
+ *   kv_hi - kv_lo the user's key tiles are masked key by key.
+ *   items [max_items * 4] int32, written; item i = {first query row, h * 256 + rows in the
+ *   tile, kv_lo, (kv_hi - kv_lo) | (holes << 31)}.
+ *   n_items [1] int32, written.
+ *   q_rows / kv_rows: rows of the query and key tensors (q_offsets[B] must equal q_rows;
+ *   every key interval must lie inside [0, kv_rows)).
+ * Device errors: bad q_offsets or a key interval outside [0, kv_rows) -> JCA_STATUS_BAD_OFFSETS;
+ * more than max_items items -> JCA_STATUS_QUEUE_OVERFLOW. n_items is 0 after any error.
+ */
+int jca_build_work_queue(const void* q_offsets, const void* kv_lo, const void* kv_hi,
+                         const int32_t* kv_count, int64_t B, int64_t q_rows, int64_t kv_rows,
+                         int H, int idx_bits, int32_t* items, int64_t max_items,
+                         int32_t* n_items, int32_t* status, jca_stream_t stream);
+
+/* Upper bound on the work items of B users with `rows` query rows in total and H heads. */
+int64_t jca_max_work_items(int64_t B, int64_t rows, int H);
+
+/*
+ * Workspace bytes needed by jagged_cand_attn_fwd (rows = T) or cand_only_attn_fwd
+ * (rows = Nc) for B users, H heads and head size d_head. Returns 0 for invalid sizes.
+ */
+size_t jca_workspace_bytes(int64_t B, int64_t rows, int H, int d_head);
+
+/*
+ * Jagged candidate-isolated attention forward (候选隔离注意力掩码, sections 段 ID：掩码的表达方式
+ * and 掩码长什么样): for every user row and head, softmax(scale * Q K^T + mask) V with
+ *   mask[q, kv] = (kv is history AND (q is history OR q is a candidate))
+ *              OR (q and kv are the same candidate position),
+ * evaluated from segment intervals inside the kernel; no [L, L] mask is materialised
+ * (section 设计决策). Query rows of padding (segment 0) output 0.
+ *   q, k, v  [T, H, d_head] bf16, read.
+ *   out      [T, H, d_head] bf16 (out_fp32 = 0) or fp32 (out_fp32 != 0), written.
+ *   offsets  [B+1] (idx_bits type), read.
+ *   candidate_start [B] row-relative (idx_bits type), read when seg == NULL.
+ *   seg      [T] int8 or NULL. When given it replaces candidate_start (this is how padding
+ *            enters: build it with jca_build_segment_ids); when NULL no token is padding.
+ *   scale    softmax scale; <= 0 selects 1/sqrt(d_head).
+ *   workspace / workspace_bytes: >= jca_workspace_bytes(B, T, H, d_head).
+ * Runs on `stream`: segment IDs (when seg == NULL), bounds, work queue, attention kernel.
+ * Device errors: as the builders above, plus JCA_STATUS_TIMEOUT.
+ */
+int jagged_cand_attn_fwd(const void* q, const void* k, const void* v, void* out, int out_fp32,
+                         const void* offsets, const void* candidate_start, const int8_t* seg,
+                         int64_t B, int64_t T, int H, int d_head, float scale, int idx_bits,
+                         void* workspace, size_t workspace_bytes, int32_t* status,
+                         jca_stream_t stream);
+
+/*
+ * Candidate-only attention layer (候选隔离注意力掩码, section 只更新候选的末尾层; the arguments mirror
+ * the page's operator inputs candidate_q, history_k, history_v, own_k, own_v): each candidate of
+ * user b attends to the frozen history keys/values of user b and to its own key/value only.
+ * Its result equals the candidate rows of jagged_cand_attn_fwd on the same K/V.
+ *   cand_q, own_k, own_v [Nc, H, d_head] bf16, read; cand_offsets [B+1] (idx_bits type).
+ *   hist_k, hist_v [Th, H, d_head] bf16, read; hist_offsets [B+1] (idx_bits type).
+ *   hist_seg [Th] int8 or NULL: 1 = valid history row, 0 = padding (NULL = all valid).
+ *   out [Nc, H, d_head] bf16 or fp32 (out_fp32), written.
+ *   workspace / workspace_bytes: >= jca_workspace_bytes(B, Nc, H, d_head).
+ * Device errors: bad offsets -> JCA_STATUS_BAD_OFFSETS; hist_seg values other than 0/1 ->
+ * JCA_STATUS_BAD_SEG_VALUE; JCA_STATUS_TIMEOUT.
+ */
+int cand_only_attn_fwd(const void* cand_q, const void* own_k, const void* own_v,
+                       const void* cand_offsets, const void* hist_k, const void* hist_v,
+                       const void* hist_offsets, const int8_t* hist_seg, void* out, int out_fp32,
+                       int64_t B, int64_t Nc, int64_t Th, int H, int d_head, float scale,
+                       int idx_bits, void* workspace, size_t workspace_bytes, int32_t* status,
+                       jca_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JCA_H_ */

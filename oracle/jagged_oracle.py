@@ -235,22 +235,13 @@ def jagged_cand_attn_rows(q, k, v, offsets, seg, scale: float, rows) -> np.ndarr
     H, dv = q.shape[1], v.shape[2]
     out = np.zeros((rows.shape[0], H, dv), dtype=np.float64)
     users = np.searchsorted(offsets, rows, side="right") - 1
-    for i, (r, b) in enumerate(zip(rows, users)):
+    for b in np.unique(users):
         s, e = int(offsets[b]), int(offsets[b + 1])
-        mask_row = history_candidate_mask(seg[s:e])[int(r) - s:int(r) - s + 1]
-        out[i] = masked_softmax_attention(q[int(r):int(r) + 1], k[s:e], v[s:e], mask_row, scale)[0]
+        sel = np.nonzero(users == b)[0]
+        rel = rows[sel] - s
+        mask = history_candidate_mask(seg[s:e])[rel]
+        out[sel] = masked_softmax_attention(q[rows[sel]], k[s:e], v[s:e], mask, scale)
     return out
-
-
-def _concat_user(hk, hv, hseg, ck, cv, cq):
-    """Rows of the fallback evaluation for one user: [history rows | candidate rows]."""
-    n_h = hk.shape[0]
-    n_c = ck.shape[0]
-    q_cat = np.concatenate([np.zeros_like(hk), cq], axis=0)  # history queries are not evaluated
-    k_cat = np.concatenate([hk, ck], axis=0)
-    v_cat = np.concatenate([hv, cv], axis=0)
-    seg_cat = np.concatenate([hseg.astype(np.int8), np.full(n_c, SEG_CANDIDATE, np.int8)])
-    return q_cat, k_cat, v_cat, seg_cat, n_h
 
 
 def cand_only_attn(cq, ck, cv, cand_offsets, hk, hv, hist_offsets, hist_seg, scale: float,
@@ -258,13 +249,15 @@ def cand_only_attn(cq, ck, cv, cand_offsets, hk, hv, hist_offsets, hist_seg, sca
     """Candidate-only layer: candidate queries over frozen history K/V plus their own K/V.
 
     Evaluated through the full-layer fallback (候选隔离注意力掩码, section 只更新候选的末尾层):
-    each user's row is [history | candidates] with history segments taken from ``hist_seg``
-    (1 = valid, 0 = padding; None = all valid) and candidates marked -1; the full mask runs over the
-    row and only the candidate rows are kept. ``cand_rows`` (absolute candidate indices) restricts
-    the output to those rows, returned in that order.
+    each user's row is [history | candidates], with history segments taken from ``hist_seg``
+    (1 = valid, 0 = padding; None = all valid) and candidates marked -1; the full mask runs over
+    the row and only the candidate rows are kept.
+
+    ``cand_rows`` (absolute candidate indices) returns only those rows, in that order; the row of
+    user b is then [history | the requested candidates of b]. This relies on candidate isolation
+    (a candidate's output does not depend on the other candidates), which the oracle's own pins
+    check by adding and removing candidates.
     """
-    cq, ck, cv = _as_f64(cq), _as_f64(ck), _as_f64(cv)
-    hk, hv = _as_f64(hk), _as_f64(hv)
     coff = np.asarray(cand_offsets, dtype=np.int64)
     hoff = np.asarray(hist_offsets, dtype=np.int64)
     B = coff.shape[0] - 1
@@ -274,27 +267,31 @@ def cand_only_attn(cq, ck, cv, cand_offsets, hk, hv, hist_offsets, hist_seg, sca
     H, dv = cq.shape[1], cv.shape[2]
     if cand_rows is not None:
         cand_rows = np.asarray(cand_rows, dtype=np.int64)
-        out = np.zeros((cand_rows.shape[0], H, dv), dtype=np.float64)
+        groups = {}
         users_of = np.searchsorted(coff, cand_rows, side="right") - 1
-        for i, (r, b) in enumerate(zip(cand_rows, users_of)):
-            hs, he = int(hoff[b]), int(hoff[b + 1])
-            r = int(r)
-            q_cat, k_cat, v_cat, seg_cat, n_h = _concat_user(
-                hk[hs:he], hv[hs:he], hseg[hs:he], ck[r:r + 1], cv[r:r + 1], cq[r:r + 1])
-            mask = mask_fn(seg_cat)
-            out[i] = masked_softmax_attention(q_cat, k_cat, v_cat, mask, scale)[n_h]
-        return out
-    Nc = int(coff[-1])
-    out = np.zeros((Nc, H, dv), dtype=np.float64)
-    for b in (range(B) if users is None else users):
-        cs, ce = int(coff[b]), int(coff[b + 1])
+        for i, b in enumerate(users_of):
+            groups.setdefault(int(b), []).append(i)
+        out = np.zeros((cand_rows.shape[0], H, dv), dtype=np.float64)
+    else:
+        groups = {b: None for b in (range(B) if users is None else users)}
+        out = np.zeros((int(coff[-1]), H, dv), dtype=np.float64)
+    for b, sel in groups.items():
         hs, he = int(hoff[b]), int(hoff[b + 1])
-        if ce == cs:
+        if sel is None:
+            rows = np.arange(int(coff[b]), int(coff[b + 1]))
+            dst = rows
+        else:
+            rows = cand_rows[sel]
+            dst = np.asarray(sel)
+        if rows.size == 0:
             continue
-        q_cat, k_cat, v_cat, seg_cat, n_h = _concat_user(
-            hk[hs:he], hv[hs:he], hseg[hs:he], ck[cs:ce], cv[cs:ce], cq[cs:ce])
+        n_h = he - hs
+        k_cat = np.concatenate([_as_f64(hk[hs:he]), _as_f64(ck[rows])], axis=0)
+        v_cat = np.concatenate([_as_f64(hv[hs:he]), _as_f64(cv[rows])], axis=0)
+        seg_cat = np.concatenate([hseg[hs:he], np.full(rows.size, SEG_CANDIDATE, np.int8)])
         mask = mask_fn(seg_cat)
-        out[cs:ce] = masked_softmax_attention(q_cat, k_cat, v_cat, mask, scale)[n_h:]
+        q_rows = _as_f64(cq[rows])
+        out[dst] = masked_softmax_attention(q_rows, k_cat, v_cat, mask[n_h:], scale)
     return out
 
 
