@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark of the jagged candidate-isolated attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the hot path over one batch of the 256-user workload (256 users,
+lognormal histories with median 280 clipped to [0, 4096], 4 prefix tokens and 64 candidates per
+user, H = 8, d_head = 128, bf16, seed 0): offsets from lengths, then the plan (segment IDs, bounds,
+cost-sorted work queue) and the attention kernel, all through the C ABI of libjca.so. Inputs are
+resident in HBM when the timed region starts; Q/K/V (837 MB) exceed the 126 MB L2, so no flush is
+needed between steps. The metric is effective attention TFLOP/s: 4 * d_head * H FLOPs per
+(query, key) pair the candidate-isolation mask allows (padding and masked pairs not counted).
+
+With torchrun (N > 1) every rank runs its own batch (weak scaling, no data-path collective); the
+time is the max over ranks and the value counts the work of all ranks. ``--impl reference`` times
+the CPU oracle (the reference arm of this build) on a bounded sample of the same workload.
+Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "effective attention TFLOP/s (unpadded) and tokens/s, % of B200 bf16 peak"
+WORKLOAD = ("users256: 256 users, history lengths floor(lognormal(ln 280, 1)) clipped to [0, 4096] "
+            "(users 0, 64, 128, 192 empty, user 1 = 4096), 4 prefix + 64 candidates per user, "
+            "H=8, d_head=128, bf16 N(0,1), seed 0")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "candidate_isolated_jagged_b200", "csrc")
+    for name in ("attention.cu", "jca_device.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name: str):
+    """DRAM bytes per launch recorded in profiles/<name>.md by an ncu capture, or None when the
+    summary is missing or the kernel source changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", name + ".md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != kernel_source_sha():
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """Samples SM clocks and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:  # noqa: BLE001 - NVML missing: report no clocks
+            self.ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "note": "NVML unavailable" if not self.ok else "no samples"}
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p["num_threads"] for p in threadpool_info() if p.get("user_api") == "blas"]
+        return int(max(n)) if n else 1
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle arm
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample_users(batch, stride: int, phase: int):
+    return [u for u in range(batch.B) if u % stride == phase]
+
+
+def time_oracle(batch, users, repeats: int = 1):
+    """Effective TFLOP/s of the fp64 oracle on the given users of the batch (host cores)."""
+    import oracle
+    from candidate_isolated_jagged_b200 import metrics
+    off = oracle.offsets_from_lengths(batch.row_lengths)
+    seg = oracle.segment_ids(off, batch.cand_start, batch.valid)
+    n1 = (batch.prefix + batch.hist_real)[users]
+    pairs = metrics.allowed_pairs_from_counts(n1, batch.n_cand[users])
+    flops = metrics.effective_flops(pairs, batch.H, batch.d)
+    tokens = int(np.sum(batch.row_lengths[users]))
+    times = []
+    for _ in range(repeats):
+        t0 = time.perf_counter()
+        oracle.jagged_cand_attn(batch.q, batch.k, batch.v, off, seg, batch.scale, users=users)
+        times.append(time.perf_counter() - t0)
+    return flops, tokens, times
+
+
+def run_reference(args, rank: int):
+    if rank != 0:
+        return 0
+    import synth
+    batch = synth.users256()
+    # Each step: the oracle over 8 representative users (index = 5 mod 32) of the same batch.
+    users = oracle_sample_users(batch, 32, 5)
+    flops, tokens, _ = time_oracle(batch, users, repeats=max(1, args.warmup))
+    _, _, times = time_oracle(batch, users, repeats=args.steps)
+    total = float(np.sum(times))
+    value = flops * args.steps / total / 1e12
+    cores = blas_threads()
+    sample = (f"users with index = 5 mod 32 ({len(users)} of 256, {tokens} rows, "
+              f"{flops / 1e9:.2f} effective GFLOP) per step, fp64 numpy")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "tokens_per_s": tokens * args.steps / total,
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import torch
+    import synth
+    from candidate_isolated_jagged_b200 import jca, metrics
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist  # noqa: F811
+
+    peaks = load_peaks()
+    batch = synth.users256()
+    B, T, H, d = batch.B, batch.T, batch.H, batch.d
+    n1 = batch.prefix + batch.hist_real
+    pairs = metrics.allowed_pairs_from_counts(n1, batch.n_cand)
+    flops = metrics.effective_flops(pairs, H, d)
+    valid_tokens = int(batch.row_lengths.sum()) if batch.valid is None else int(batch.valid.sum())
+
+    stream = torch.cuda.current_stream(dev)
+    q, k, v = (t.to(dev) for t in (batch.q, batch.k, batch.v))
+    lengths = torch.tensor(batch.row_lengths, dtype=torch.int64, device=dev)
+    cand_start = torch.tensor(batch.cand_start, dtype=torch.int64, device=dev)
+    offsets = torch.empty(B + 1, dtype=torch.int64, device=dev)
+    out = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(jca.jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=dev)
+    status = jca.new_status(dev)
+    launches_per_step = 5  # offsets, segment IDs, bounds, work queue, attention
+
+    def step(ev=None):
+        jca.jca_offsets_from_lengths(lengths, offsets, status, stream)
+        jca.jagged_cand_attn_plan(offsets, cand_start, None, T, H, d, ws, status, stream)
+        if ev is not None:
+            ev[0].record(stream)
+        jca.jagged_cand_attn_run(q, k, v, out, None, B, ws, status, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    jca.check_status(status, "warm-up")
+    assert bool(torch.isfinite(out.float()).all()), "non-finite attention output"
+
+    kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    with sampler:
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(kev[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+    jca.check_status(status, "timed region")
+    elapsed_ms = t_start.elapsed_time(t_end)
+    kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
+    if dist:
+        t = torch.tensor([elapsed_ms, kernel_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, kernel_ms = float(t[0]), float(t[1])
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops * args.steps / (elapsed_ms / 1e3) / 1e12
+
+    # ---- end to end through the public API: host inputs in, host output back ----
+    e2e_steps = max(1, min(args.steps, args.e2e_steps))
+    pin = lambda t: t.pin_memory()  # noqa: E731
+    q_h, k_h, v_h = pin(batch.q), pin(batch.k), pin(batch.v)
+    len_h = pin(torch.tensor(batch.row_lengths, dtype=torch.int64))
+    cs_h = pin(torch.tensor(batch.cand_start, dtype=torch.int64))
+    out_h = torch.empty(T, H, d, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, len_h, cs_h))
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        lengths.copy_(len_h, non_blocking=True)
+        cand_start.copy_(cs_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t[0])
+    jca.check_status(status, "end-to-end")
+    e2e_value = world * flops * e2e_steps / (e2e_ms / 1e3) / 1e12
+
+    achieved = flops / (kernel_ms / 1e3) / 1e12
+    roofline = {
+        "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+        "frac": achieved / peaks["bf16_tflops"],
+        "traffic": profiled_traffic("attn_users256_d128"),
+        "kernel": "jagged_attn_kernel<128>", "kernel_ms": kernel_ms,
+        "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+        "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
+        "algorithmic_flops_per_launch": flops,
+        "algorithmic_bytes_per_launch": metrics.full_attention_bytes(T, H, d),
+    }
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "rows": T, "valid_tokens": valid_tokens,
+                   "allowed_pairs": pairs, "effective_flops_per_step": flops,
+                   "l2": "inputs (Q/K/V 837 MB) larger than L2 (126 MB); no flush",
+                   "parallelism": f"dp{world}: users sharded by batch, no collective"},
+        "tokens_per_s": world * valid_tokens * args.steps / (elapsed_ms / 1e3),
+        "pct_of_bf16_peak": 100.0 * value / (world * peaks["bf16_tflops"]),
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": e2e_ms / e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+    }
+    del q_h, k_h, v_h, out_h
+
+    if rank == 0 and world == 1 and not args.no_extras:
+        line["cand_only"] = run_cand_only_extras(args, dev, stream, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        users = oracle_sample_users(batch, args.cpu_sample_stride, 3)
+        fl, tok, times = time_oracle(batch, users, repeats=1)
+        line["cpu_baseline"] = {
+            "value": fl / times[0] / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle", "seconds": times[0],
+            "sample": (f"users with index = 3 mod {args.cpu_sample_stride} ({len(users)} of 256,"
+                       f" {tok} rows, {fl / 1e9:.1f} effective GFLOP), fp64 numpy, one pass")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_cand_only_extras(args, dev, stream, peaks):
+    """The candidate-only entry point on its two workloads: attention kernel time (CUDA events,
+    mean over timed launches after one plan), effective TFLOP/s and algorithmic HBM GB/s."""
+    import torch
+    import oracle
+    import synth
+    from candidate_isolated_jagged_b200 import jca, metrics
+    res = {}
+    for name, make in (("cand_only256", synth.cand_only256), ("retrieval", synth.retrieval)):
+        cb = make()
+        coff = torch.tensor(oracle.offsets_from_lengths(cb.cand_counts), device=dev)
+        hoff = torch.tensor(oracle.offsets_from_lengths(cb.hist_lengths), device=dev)
+        cq, ck, cv, hk, hv = (t.to(dev) for t in (cb.cq, cb.ck, cb.cv, cb.hk, cb.hv))
+        out = torch.empty(cq.shape, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(jca.jca_workspace_bytes(cb.B, cb.Nc, cb.H, cb.d), dtype=torch.uint8,
+                         device=dev)
+        st = jca.new_status(dev)
+        jca.cand_only_attn_plan(coff, hoff, None, cb.Nc, cb.Th, cb.H, cb.d, ws, st, stream)
+        for _ in range(max(3, args.warmup)):
+            jca.cand_only_attn_run(cq, ck, cv, hk, hv, None, out, cb.B, ws, st, stream=stream)
+        n = max(10, min(args.steps, 100))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n):
+            jca.cand_only_attn_run(cq, ck, cv, hk, hv, None, out, cb.B, ws, st, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        jca.check_status(st, name)
+        ms = e0.elapsed_time(e1) / n
+        pairs = int(np.sum(cb.cand_counts * (cb.hist_lengths + 1)))
+        fl = metrics.effective_flops(pairs, cb.H, cb.d)
+        byts = metrics.cand_only_bytes(cb.Nc, cb.Th, cb.H, cb.d)
+        res[name] = {
+            "kernel_ms": ms, "effective_tflops": fl / ms / 1e9,
+            "pct_of_bf16_peak": 100 * fl / ms / 1e9 / peaks["bf16_tflops"],
+            "candidates_per_s": cb.Nc / ms * 1e3,
+            "roofline": {"bound": "hbm", "achieved": byts / ms / 1e6, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": byts / ms / 1e6 / peaks["hbm_gbs"],
+                         "algorithmic_bytes_per_launch": byts},
+            "launches_timed": n,
+        }
+        del cq, ck, cv, hk, hv, out, ws
+        torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-extras", action="store_true", help="skip the candidate-only workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-stride", type=int, default=4)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

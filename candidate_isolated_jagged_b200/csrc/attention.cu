@@ -63,27 +63,26 @@ struct Cfg {
   static constexpr int KSTEPS_QK = D / 16;
   static constexpr int KSTEPS_PER_BLK = SW / 32;
   static constexpr int KSTEPS_PV = BN / 16;
-  static constexpr int P_BLK_BYTES = BM * 128;                     // P: two 64-key blocks
-  static constexpr int P_BYTES = 2 * P_BLK_BYTES;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
-  static constexpr int OFF_P = OFF_V + 2 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int NUM_BARS = 20;
+  static constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
+  static constexpr int NUM_BARS = 24;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 16;
   static constexpr int SMEM_RAW = SMEM_USED + 1024;                // slack for 1 KB alignment
   // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
   static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
-  static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256, TMEM_COLS = 512;
+  // TMEM columns: S0 | S1 (fp32 scores) | O (fp32 accumulator) | P0 | P1 (bf16 pairs).
+  static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256, TMEM_P0 = 384,
+                            TMEM_COLS = 512;
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
 };
 
 // Barrier slots.
 enum : int {
   kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = 6, kVFull = 8, kVEmpty = 10,
-  kSFull = 12, kSEmpty = 14, kPFull = 16, kPVDone = 17, kDrain = 18
+  kSFull = 12, kSEmpty = 14, kPFull = 16, kPVDone = 18, kDrain = 20
 };
 
 constexpr int kThreads = 192;
@@ -162,30 +161,33 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
 // ------------------------------------------------------------------------------------------
 // MMA issuer
 // ------------------------------------------------------------------------------------------
+// O += P V for key tile gg (P from TMEM buffer gg % 2), whose first `valid` keys are real: only
+// ceil(valid / 16) k-steps are issued.
 template <int D>
-__device__ __forceinline__ bool issue_pv(uint32_t gg, bool first, uint32_t sbase, uint32_t bars,
-                                         uint32_t tmem, const AttnArgs& a,
+__device__ __forceinline__ bool issue_pv(uint32_t gg, int valid, bool first, uint32_t sbase,
+                                         uint32_t bars, uint32_t tmem, const AttnArgs& a,
                                          volatile int* abort_flag) {
   using C = Cfg<D>;
   constexpr uint32_t kIdescPV = idesc_bf16_f32(C::BM, D, false, true);
   const int s = gg & 1;
   const uint32_t ph = (gg >> 1) & 1;
   if (!mbar_wait(bars + 8 * (kVFull + s), ph, abort_flag, a.status)) return false;
-  if (!mbar_wait(bars + 8 * kPFull, gg & 1, abort_flag, a.status)) return false;
+  if (!mbar_wait(bars + 8 * (kPFull + s), ph, abort_flag, a.status)) return false;
   tc_fence_after();
-  const uint32_t p_base = sbase + C::OFF_P;
+  const uint32_t p_tmem = tmem + C::TMEM_P0 + (uint32_t)s * 64u;
   const uint32_t v_base = sbase + C::OFF_V + s * C::TILE_BYTES;
+  const int ksteps = (valid + 15) >> 4;
 #pragma unroll
   for (int kk = 0; kk < C::KSTEPS_PV; ++kk) {
-    // P: K-major, 128-byte swizzle, two 64-key blocks; V: MN-major (head dim contiguous).
-    const uint64_t adesc =
-        smem_desc(p_base + (kk / 4) * C::P_BLK_BYTES + (kk % 4) * 32, 16, 1024, 2u);
+    if (kk >= ksteps) break;
+    // P: 16 keys = 8 TMEM columns per k-step; V: MN-major (head dim contiguous), 16 key rows.
     const uint64_t bdesc =
         smem_desc(v_base + kk * 16 * C::SW, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
-    tc_mma(tmem + C::TMEM_O, adesc, bdesc, kIdescPV, (first && kk == 0) ? 0u : 1u);
+    tc_mma_ts(tmem + C::TMEM_O, p_tmem + (uint32_t)kk * 8u, bdesc, kIdescPV,
+              (first && kk == 0) ? 0u : 1u);
   }
   tc_commit(bars + 8 * (kVEmpty + s));
-  tc_commit(bars + 8 * kPVDone);
+  tc_commit(bars + 8 * (kPVDone + s));
   return true;
 }
 
@@ -193,7 +195,8 @@ template <int D>
 __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          int n_items, volatile int* abort_flag) {
   using C = Cfg<D>;
-  constexpr uint32_t kIdescQK = idesc_bf16_f32(C::BM, C::BN, false, false);
+  // QK^T with N = keys of the tile rounded up to 16 (the last key tile of a user is trimmed).
+  constexpr uint32_t kIdescQK0 = idesc_bf16_f32(C::BM, 16, false, false) & ~(0x3Fu << 17);
   uint32_t g = 0, qi = 0;
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
@@ -204,9 +207,12 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     if (!ok) break;
     tc_fence_after();
     const uint32_t q_base = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+    int prev_valid = 0;
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = g & 1;
       const uint32_t ph = (g >> 1) & 1;
+      const int valid = min(C::BN, w.kv_len - j * C::BN);
+      const uint32_t idesc_qk = kIdescQK0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17);
       ok = mbar_wait(bars + 8 * (kKFull + s), ph, abort_flag, a.status) &&
            mbar_wait(bars + 8 * (kSEmpty + s), ph ^ 1, abort_flag, a.status);
       if (!ok) break;
@@ -218,19 +224,20 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
         const uint32_t off =
             (kk / C::KSTEPS_PER_BLK) * C::BLK_BYTES + (kk % C::KSTEPS_PER_BLK) * 32;
         tc_mma(d_tmem, smem_desc(q_base + off, 16, 8 * C::SW, C::LAYOUT),
-               smem_desc(k_base + off, 16, 8 * C::SW, C::LAYOUT), kIdescQK, kk > 0 ? 1u : 0u);
+               smem_desc(k_base + off, 16, 8 * C::SW, C::LAYOUT), idesc_qk, kk > 0 ? 1u : 0u);
       }
       tc_commit(bars + 8 * (kKEmpty + s));
       tc_commit(bars + 8 * (kSFull + s));
       // PV of the previous key tile goes behind this QK, so the tensor core computes the next
       // S while the softmax warps work on the previous one.
       if (j > 0) {
-        ok = issue_pv<D>(g - 1, j == 1, sbase, bars, tmem, a, abort_flag);
+        ok = issue_pv<D>(g - 1, prev_valid, j == 1, sbase, bars, tmem, a, abort_flag);
         if (!ok) break;
       }
+      prev_valid = valid;
     }
     if (!ok) break;
-    ok = issue_pv<D>(g - 1, w.n_kv == 1, sbase, bars, tmem, a, abort_flag);
+    ok = issue_pv<D>(g - 1, prev_valid, w.n_kv == 1, sbase, bars, tmem, a, abort_flag);
     if (!ok) break;
     tc_commit(bars + 8 * (kQEmpty + qs));
     ++qi;
@@ -245,29 +252,6 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
 // ------------------------------------------------------------------------------------------
 // Softmax + epilogue
 // ------------------------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ void load_o_row(uint32_t t_o, float* o) {
-  if constexpr (D == 16) {
-    uint32_t r[16];
-    tmem_ld_x16(t_o, r);
-    tmem_wait_ld();
-    reg_fence16(r);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[i] = __uint_as_float(r[i]);
-  } else {
-#pragma unroll
-    for (int c = 0; c < D; c += 32) {
-      uint32_t r[32];
-      tmem_ld_x32(t_o + c, r);
-      tmem_wait_ld();
-      reg_fence16(r);
-      reg_fence16(r + 16);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[c + i] = __uint_as_float(r[i]);
-    }
-  }
-}
-
 template <int D>
 __device__ __forceinline__ void rescale_o_row(uint32_t t_o, float alpha) {
   if constexpr (D == 16) {
@@ -294,39 +278,65 @@ __device__ __forceinline__ void rescale_o_row(uint32_t t_o, float alpha) {
   tmem_wait_st();
 }
 
-// Diagonal merge (the candidate's own key/value), normalisation and store of one output row.
+// Epilogue of one query row: diagonal merge (a candidate's own key/value), normalisation and
+// store. Every lane of the warp calls this (the TMEM loads are warp-collective); rows outside the
+// tile only skip their memory accesses.
 template <int D>
-__device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int r, float m,
-                                           float l, float* o) {
-  if (r >= w.nrows) return;
-  const int row = w.q_row0 + r;
+__device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int r, uint32_t t_o,
+                                           bool has_o, float m, float l) {
+  const bool row_ok = r < w.nrows;
+  const int row = w.q_row0 + (row_ok ? r : 0);
   const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
-  const int seg = a.q_seg ? (int)a.q_seg[row] : -1;
-  float inv;
-  if (seg == 0) {
-    inv = 0.f;  // padding query: no visible key
-  } else {
-    if (seg == -1) {
-      const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
-      const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const int seg = row_ok ? (a.q_seg ? (int)a.q_seg[row] : -1) : 0;
+  float alpha = 1.f, beta = 0.f;
+  if (seg == -1) {
+    const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
+    const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
-        const uint4 qa = ld_global_nc_v4(qp + c);
-        const uint4 ka = ld_global_nc_v4(kp + c);
-        acc[0] = fmaf(bf16_lo(qa.x), bf16_lo(ka.x), fmaf(bf16_hi(qa.x), bf16_hi(ka.x), acc[0]));
-        acc[1] = fmaf(bf16_lo(qa.y), bf16_lo(ka.y), fmaf(bf16_hi(qa.y), bf16_hi(ka.y), acc[1]));
-        acc[2] = fmaf(bf16_lo(qa.z), bf16_lo(ka.z), fmaf(bf16_hi(qa.z), bf16_hi(ka.z), acc[2]));
-        acc[3] = fmaf(bf16_lo(qa.w), bf16_lo(ka.w), fmaf(bf16_hi(qa.w), bf16_hi(ka.w), acc[3]));
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 qa = ld_global_nc_v4(qp + c);
+      const uint4 ka = ld_global_nc_v4(kp + c);
+      acc[0] = fmaf(bf16_lo(qa.x), bf16_lo(ka.x), fmaf(bf16_hi(qa.x), bf16_hi(ka.x), acc[0]));
+      acc[1] = fmaf(bf16_lo(qa.y), bf16_lo(ka.y), fmaf(bf16_hi(qa.y), bf16_hi(ka.y), acc[1]));
+      acc[2] = fmaf(bf16_lo(qa.z), bf16_lo(ka.z), fmaf(bf16_hi(qa.z), bf16_hi(ka.z), acc[2]));
+      acc[3] = fmaf(bf16_lo(qa.w), bf16_lo(ka.w), fmaf(bf16_hi(qa.w), bf16_hi(ka.w), acc[3]));
+    }
+    const float sd = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * a.scale_log2;
+    const float m_new = fmaxf(m, sd);
+    alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+    beta = fast_exp2(sd - m_new);
+    l = l * alpha + beta;
+  }
+  // Padding queries (segment 0) see no key and output 0.
+  const float inv = (seg != 0 && l > 0.f) ? 1.f / l : 0.f;
+  constexpr int CW = D < 32 ? D : 32;   // columns per TMEM load
+#pragma unroll
+  for (int c0 = 0; c0 < D; c0 += CW) {
+    float o[CW];
+    if (has_o) {
+      uint32_t u[CW];
+      if constexpr (CW == 32) {
+        tmem_ld_x32(t_o + c0, u);
+        tmem_wait_ld();
+        reg_fence16(u);
+        reg_fence16(u + 16);
+      } else {
+        tmem_ld_x16(t_o + c0, u);
+        tmem_wait_ld();
+        reg_fence16(u);
       }
-      const float sd = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * a.scale_log2;
-      const float m_new = fmaxf(m, sd);
-      const float alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
-      const float beta = fast_exp2(sd - m_new);
-      l = l * alpha + beta;
-      const uint4* vp = reinterpret_cast<const uint4*>(a.dv + base);
 #pragma unroll
-      for (int c = 0; c < D / 8; ++c) {
+      for (int i = 0; i < CW; ++i) o[i] = __uint_as_float(u[i]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < CW; ++i) o[i] = 0.f;
+    }
+    if (!row_ok) continue;
+    if (seg == -1) {
+      const uint4* vp = reinterpret_cast<const uint4*>(a.dv + base + c0);
+#pragma unroll
+      for (int c = 0; c < CW / 8; ++c) {
         const uint4 va = ld_global_nc_v4(vp + c);
         const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
 #pragma unroll
@@ -336,23 +346,33 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int
         }
       }
     }
-    inv = l > 0.f ? 1.f / l : 0.f;
-  }
-  if (a.out_fp32) {
-    float4* op = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base);
+    if (seg == 0) {
 #pragma unroll
-    for (int c = 0; c < D / 4; ++c)
-      op[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
-                          o[4 * c + 3] * inv);
-  } else {
-    uint4* op = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base);
+      for (int i = 0; i < CW; ++i) o[i] = 0.f;
+    }
+    if (a.out_fp32) {
+      float4* op = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base + c0);
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c)
-      op[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
-                         pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
-                         pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
-                         pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+      for (int c = 0; c < CW / 4; ++c)
+        op[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
+                            o[4 * c + 3] * inv);
+    } else {
+      uint4* op =
+          reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base + c0);
+#pragma unroll
+      for (int c = 0; c < CW / 8; ++c)
+        op[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
+                           pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
+                           pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
+                           pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+    }
   }
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 template <int D>
@@ -362,21 +382,29 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, u
   const int quarter = warp & 3;               // TMEM lane quarter this warp may access
   const int r = quarter * 32 + lane;          // query row of this thread inside the tile
   const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-  const uint32_t p_row = sbase + C::OFF_P + (uint32_t)r * 128u;
-  const uint32_t sw = (uint32_t)(r & 7);
+  const float sl2 = a.scale_log2;
   uint32_t g = 0;
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = g & 1;
       const uint32_t ph = (g >> 1) & 1;
+      const int valid = min(C::BN, w.kv_len - j * C::BN);
+      // Edge tiles (the trimmed last tile, or any tile of a user with padding holes) are masked
+      // column by column; interior tiles take the unmasked path.
+      const bool edge = valid < C::BN || w.holes;
+      const int8_t* kseg = w.holes ? a.kv_seg + (w.kv_lo + j * C::BN) : nullptr;
+      const int nchunks = (valid + 31) >> 5;
       ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (kSFull + s), ph, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      uint32_t x[128];
       const uint32_t t_s = t_lane + (s ? C::TMEM_S1 : C::TMEM_S0);
+
+      // Pass 1: the whole S row in registers (four 32-column TMEM loads, one wait), then the
+      // max of the raw scores (the scale is positive, so it commutes with max).
+      uint32_t x[128];
       tmem_ld_x32(t_s + 0, x);
       tmem_ld_x32(t_s + 32, x + 32);
       tmem_ld_x32(t_s + 64, x + 64);
@@ -384,82 +412,95 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, u
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 128; c += 16) reg_fence16(x + c);
+      // S is in registers: the MMA warp may overwrite this buffer.
       tc_fence_before();
       mbar_arrive(bars + 8 * (kSEmpty + s));
-
-      // Masked scores in the log2 domain.
-      const int valid_cols = min(C::BN, w.kv_len - j * C::BN);
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (!w.holes) {
+      if (edge) {
+        // Every row of the tile sees the same key columns: the warp builds the tile's 128-bit
+        // column mask with one ballot per 32 columns (lane i tests column 32k + i).
+        uint32_t bits[4];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float v = __uint_as_float(x[c]) * a.scale_log2;
-          v = c < valid_cols ? v : -INFINITY;
-          x[c] = __float_as_uint(v);
-          mx[c & 3] = fmaxf(mx[c & 3], v);
+        for (int k = 0; k < 4; ++k) {
+          const int c = 32 * k + lane;
+          bool keep = c < valid;
+          if (keep && kseg != nullptr) keep = kseg[c] == 1;
+          bits[k] = __ballot_sync(0xffffffffu, keep);
         }
-      } else {
-        const int8_t* kseg = a.kv_seg + (w.kv_lo + j * C::BN);
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          float v = __uint_as_float(x[c]) * a.scale_log2;
-          const bool keep = c < valid_cols && kseg[c] == 1;
-          v = keep ? v : -INFINITY;
-          x[c] = __float_as_uint(v);
-          mx[c & 3] = fmaxf(mx[c & 3], v);
-        }
+        for (int c = 0; c < 128; ++c)
+          x[c] = ((bits[c >> 5] >> (c & 31)) & 1u) ? x[c] : 0xff800000u;   // -inf
       }
-      const float m_tile = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        mx0 = fmax3(mx0, __uint_as_float(x[c]), __uint_as_float(x[c + 1]));
+        mx1 = fmax3(mx1, __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+        mx2 = fmax3(mx2, __uint_as_float(x[c + 4]), __uint_as_float(x[c + 5]));
+        mx3 = fmax3(mx3, __uint_as_float(x[c + 6]), __uint_as_float(x[c + 7]));
+      }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
       const float m_new = fmaxf(m, m_tile);
       // Lazy rescaling: keep the stale reference unless the max grew by more than 2^8.
       const bool rescale = m_new > m + 8.0f;
       const float m_use = rescale ? m_new : m;
-      const float m_sub = (m_use == -INFINITY) ? 0.f : m_use;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < 128; c += 2) {
-        const float p0 = fast_exp2(__uint_as_float(x[c]) - m_sub);
-        const float p1 = fast_exp2(__uint_as_float(x[c + 1]) - m_sub);
-        sum[(c >> 1) & 3] += p0 + p1;
-        x[c >> 1] = pack_bf16x2(p0, p1);  // packed P overwrites consumed scores in place
-      }
-      // The previous PV must be complete before P is overwritten and before O is rescaled.
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * kPVDone, (g - 1) & 1, abort_flag,
-                                                 a.status));
-        if (!ok) break;
-        tc_fence_after();
-      }
-      const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
-      if (rescale && j > 0) rescale_o_row<D>(t_lane + C::TMEM_O, alpha);
-      l = (rescale ? l * alpha : l) + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
-      m = m_use;
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int k = cb * 32 + ch * 4;
-          st_shared_v4(p_row + cb * C::P_BLK_BYTES + (((uint32_t)ch ^ sw) << 4), x[k], x[k + 1],
-                       x[k + 2], x[k + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bars + 8 * kPFull);
-    }
-    if (!ok) break;
-    float o[D];
-    if (w.n_kv > 0) {
+      const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
+
+      // P buffer s was last read by the PV of tile g - 2: it must have completed.
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bars + 8 * kPVDone, (g - 1) & 1, abort_flag, a.status));
+                      mbar_wait(bars + 8 * (kPVDone + s), ph ^ 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      load_o_row<D>(t_lane + C::TMEM_O, o);
-    } else {
+
+      // Pass 2: p = 2^(scale_log2 * s - m), streamed to TMEM 32 keys at a time as bf16 pairs
+      // (column k of the P buffer holds keys 2k, 2k+1). Chunks past the last real key are
+      // never read by the trimmed PV and are skipped.
+      const uint32_t t_p = t_lane + C::TMEM_P0 + (uint32_t)s * 64u;
+      float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
 #pragma unroll
-      for (int i = 0; i < D; ++i) o[i] = 0.f;
+      for (int c = 0; c < 4; ++c) {
+        if (c >= nchunks) break;
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i]), sl2, neg_m));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i + 1]), sl2, neg_m));
+          const float p2 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i + 2]), sl2, neg_m));
+          const float p3 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i + 3]), sl2, neg_m));
+          sum0 += p0;
+          sum1 += p1;
+          sum2 += p2;
+          sum3 += p3;
+          pk[i / 2] = pack_bf16x2(p0, p1);
+          pk[i / 2 + 1] = pack_bf16x2(p2, p3);
+        }
+        tmem_st_x16(t_p + 16 * c, pk);
+      }
+      const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
+      // TMEM loads/stores are warp-collective: the warp rescales when any of its rows must.
+      // O must be stable, i.e. the PV of tile g - 1 complete.
+      if (__any_sync(0xffffffffu, rescale && j > 0)) {
+        const uint32_t gp = g - 1;
+        ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (kPVDone + (gp & 1)), (gp >> 1) & 1,
+                                               abort_flag, a.status));
+        if (!ok) break;
+        tc_fence_after();
+        rescale_o_row<D>(t_lane + C::TMEM_O, alpha);
+      }
+      l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
+      m = m_use;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bars + 8 * (kPFull + s));
     }
-    finish_row<D>(a, w, r, m, l, o);
+    if (!ok) break;
+    if (w.n_kv > 0) {
+      const uint32_t gl = g - 1;   // last key tile of this item
+      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (kPVDone + (gl & 1)), (gl >> 1) & 1,
+                                             abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+    }
+    finish_row<D>(a, w, r, t_lane + C::TMEM_O, w.n_kv > 0, m, l);
   }
 }
 
@@ -492,9 +533,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (kVEmpty + i), 1);
       mbar_init(bars + 8 * (kSFull + i), 1);
       mbar_init(bars + 8 * (kSEmpty + i), kSoftmaxThreads);
+      mbar_init(bars + 8 * (kPFull + i), kSoftmaxThreads);
+      mbar_init(bars + 8 * (kPVDone + i), 1);
     }
-    mbar_init(bars + 8 * kPFull, kSoftmaxThreads);
-    mbar_init(bars + 8 * kPVDone, 1);
     mbar_init(bars + 8 * kDrain, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -633,9 +674,96 @@ bool idx_ok(int idx_bits) { return idx_bits == 32 || idx_bits == 64; }
 
 using namespace jca;
 
+namespace jca {
+namespace {
+
+// Checks shared by the plan/run entry points; returns JCA_OK or a negative code.
+int check_sizes(int idx_bits, int d_head, int64_t B, int64_t rows, int64_t kv_rows, int H) {
+  if (!idx_ok(idx_bits)) return JCA_ERR_IDX_BITS;
+  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
+  if (B < 0 || rows < 0 || kv_rows < 0 || H < 1 || H >= 65536 || rows >= (int64_t)INT_MAX ||
+      kv_rows >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX)
+    return JCA_ERR_SHAPE;
+  if (B == 0 && (rows != 0 || kv_rows != 0)) return JCA_ERR_SHAPE;
+  if (workspace_layout(B, rows, H).max_items >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  return JCA_OK;
+}
+
+int check_workspace(const void* workspace, size_t workspace_bytes, int64_t B, int64_t rows, int H) {
+  if (!workspace) return JCA_ERR_NULL;
+  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+  if (workspace_bytes < workspace_layout(B, rows, H).total) return JCA_ERR_WORKSPACE;
+  return JCA_OK;
+}
+
+}  // namespace
+}  // namespace jca
+
 extern "C" size_t jca_workspace_bytes(int64_t B, int64_t rows, int H, int d_head) {
   if (B < 0 || rows < 0 || H < 1 || !head_dim_ok(d_head)) return 0;
   return workspace_layout(B, rows, H).total;
+}
+
+extern "C" int jagged_cand_attn_plan(const void* offsets, const void* candidate_start,
+                                     const int8_t* seg, int64_t B, int64_t T, int H, int d_head,
+                                     int idx_bits, void* workspace, size_t workspace_bytes,
+                                     int32_t* status, jca_stream_t stream) {
+  int rc = check_sizes(idx_bits, d_head, B, T, T, H);
+  if (rc) return rc;
+  if (!status || !offsets) return JCA_ERR_NULL;
+  if (B > 0 && !seg && !candidate_start) return JCA_ERR_NULL;
+  rc = check_workspace(workspace, workspace_bytes, B, T, H);
+  if (rc) return rc;
+  const WorkspaceLayout L = workspace_layout(B, T, H);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  int8_t* segp = seg ? const_cast<int8_t*>(seg) : reinterpret_cast<int8_t*>(ws + L.seg);
+  int32_t* kv_count = reinterpret_cast<int32_t*>(ws + L.kv_count);
+  if (!seg && launch_segment_ids(offsets, candidate_start, nullptr, 0, B, T, idx_bits, segp,
+                                 status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  if (launch_bounds(segp, offsets, B, T, idx_bits, ws + L.hist_lo, ws + L.hist_hi, ws + L.cand_lo,
+                    ws + L.cand_hi, kv_count, 0, status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  if (launch_work_queue(offsets, ws + L.hist_lo, ws + L.hist_hi, kv_count, B, T, T, H, idx_bits,
+                        reinterpret_cast<int32_t*>(ws + L.items), L.max_items,
+                        reinterpret_cast<int32_t*>(ws + L.n_items), status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  return JCA_OK;
+}
+
+extern "C" int jagged_cand_attn_run(const void* q, const void* k, const void* v, void* out,
+                                    int out_fp32, const int8_t* seg, int64_t B, int64_t T, int H,
+                                    int d_head, float scale, void* workspace,
+                                    size_t workspace_bytes, int32_t* status,
+                                    jca_stream_t stream) {
+  int rc = check_sizes(32, d_head, B, T, T, H);
+  if (rc) return rc;
+  if (!status) return JCA_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !out)) return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)))
+    return JCA_ERR_ALIGN;
+  rc = check_workspace(workspace, workspace_bytes, B, T, H);
+  if (rc) return rc;
+  if (T == 0) return JCA_OK;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
+  const WorkspaceLayout L = workspace_layout(B, T, H);
+  char* ws = static_cast<char*>(workspace);
+  const int8_t* segp = seg ? seg : reinterpret_cast<const int8_t*>(ws + L.seg);
+  AttnArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.dk = static_cast<const __nv_bfloat16*>(k);
+  a.dv = static_cast<const __nv_bfloat16*>(v);
+  a.q_seg = segp;
+  a.kv_seg = segp;
+  a.out = out;
+  a.items = reinterpret_cast<const int4*>(ws + L.items);
+  a.n_items = reinterpret_cast<const int32_t*>(ws + L.n_items);
+  a.status = status;
+  a.H = H;
+  a.out_fp32 = out_fp32 ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  return launch_attention(d_head, a, q, T, k, v, T, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int jagged_cand_attn_fwd(const void* q, const void* k, const void* v, void* out,
@@ -644,82 +772,33 @@ extern "C" int jagged_cand_attn_fwd(const void* q, const void* k, const void* v,
                                     int64_t T, int H, int d_head, float scale, int idx_bits,
                                     void* workspace, size_t workspace_bytes, int32_t* status,
                                     jca_stream_t stream) {
-  if (!idx_ok(idx_bits)) return JCA_ERR_IDX_BITS;
-  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
-  if (B < 0 || T < 0 || H < 1 || H >= 65536 || T >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX)
-    return JCA_ERR_SHAPE;
-  if (B == 0 && T != 0) return JCA_ERR_SHAPE;
-  if (!status || !offsets || !workspace) return JCA_ERR_NULL;
+  int rc = check_sizes(idx_bits, d_head, B, T, T, H);
+  if (rc) return rc;
+  if (!status || !offsets) return JCA_ERR_NULL;
   if (T > 0 && (!q || !k || !v || !out)) return JCA_ERR_NULL;
   if (B > 0 && !seg && !candidate_start) return JCA_ERR_NULL;
   if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)))
     return JCA_ERR_ALIGN;
-  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
-  const WorkspaceLayout L = workspace_layout(B, T, H);
-  if (L.max_items >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
-  if (workspace_bytes < L.total) return JCA_ERR_WORKSPACE;
-  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  char* ws = static_cast<char*>(workspace);
-  int8_t* segp = seg ? const_cast<int8_t*>(seg) : reinterpret_cast<int8_t*>(ws + L.seg);
-  int32_t* kv_count = reinterpret_cast<int32_t*>(ws + L.kv_count);
-  int32_t* items = reinterpret_cast<int32_t*>(ws + L.items);
-  int32_t* n_items = reinterpret_cast<int32_t*>(ws + L.n_items);
-  if (!seg && launch_segment_ids(offsets, candidate_start, nullptr, 0, B, T, idx_bits, segp,
-                                 status, st) != cudaSuccess)
-    return JCA_ERR_CUDA;
-  if (launch_bounds(segp, offsets, B, T, idx_bits, ws + L.hist_lo, ws + L.hist_hi, ws + L.cand_lo,
-                    ws + L.cand_hi, kv_count, 0, status, st) != cudaSuccess)
-    return JCA_ERR_CUDA;
-  if (launch_work_queue(offsets, ws + L.hist_lo, ws + L.hist_hi, kv_count, B, T, T, H, idx_bits,
-                        items, L.max_items, n_items, status, st) != cudaSuccess)
-    return JCA_ERR_CUDA;
-  if (T == 0) return JCA_OK;
-  AttnArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.dk = static_cast<const __nv_bfloat16*>(k);
-  a.dv = static_cast<const __nv_bfloat16*>(v);
-  a.q_seg = segp;
-  a.kv_seg = segp;
-  a.out = out;
-  a.items = reinterpret_cast<const int4*>(items);
-  a.n_items = n_items;
-  a.status = status;
-  a.H = H;
-  a.out_fp32 = out_fp32 ? 1 : 0;
-  a.scale_log2 = scale * 1.4426950408889634f;
-  return launch_attention(d_head, a, q, T, k, v, T, st);
+  rc = jagged_cand_attn_plan(offsets, candidate_start, seg, B, T, H, d_head, idx_bits, workspace,
+                             workspace_bytes, status, stream);
+  if (rc) return rc;
+  return jagged_cand_attn_run(q, k, v, out, out_fp32, seg, B, T, H, d_head, scale, workspace,
+                              workspace_bytes, status, stream);
 }
 
-extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const void* own_v,
-                                  const void* cand_offsets, const void* hist_k,
-                                  const void* hist_v, const void* hist_offsets,
-                                  const int8_t* hist_seg, void* out, int out_fp32, int64_t B,
-                                  int64_t Nc, int64_t Th, int H, int d_head, float scale,
-                                  int idx_bits, void* workspace, size_t workspace_bytes,
-                                  int32_t* status, jca_stream_t stream) {
-  if (!idx_ok(idx_bits)) return JCA_ERR_IDX_BITS;
-  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
-  if (B < 0 || Nc < 0 || Th < 0 || H < 1 || H >= 65536 || Nc >= (int64_t)INT_MAX ||
-      Th >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX)
-    return JCA_ERR_SHAPE;
-  if (B == 0 && (Nc != 0 || Th != 0)) return JCA_ERR_SHAPE;
-  if (!status || !cand_offsets || !hist_offsets || !workspace) return JCA_ERR_NULL;
-  if (Nc > 0 && (!cand_q || !own_k || !own_v || !out)) return JCA_ERR_NULL;
-  if (Th > 0 && (!hist_k || !hist_v)) return JCA_ERR_NULL;
-  if (Nc > 0 && (!aligned(cand_q, 16) || !aligned(own_k, 16) || !aligned(own_v, 16) ||
-                 !aligned(out, 16)))
-    return JCA_ERR_ALIGN;
-  if (Th > 0 && (!aligned(hist_k, 16) || !aligned(hist_v, 16))) return JCA_ERR_ALIGN;
-  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+extern "C" int cand_only_attn_plan(const void* cand_offsets, const void* hist_offsets,
+                                   const int8_t* hist_seg, int64_t B, int64_t Nc, int64_t Th,
+                                   int H, int d_head, int idx_bits, void* workspace,
+                                   size_t workspace_bytes, int32_t* status,
+                                   jca_stream_t stream) {
+  int rc = check_sizes(idx_bits, d_head, B, Nc, Th, H);
+  if (rc) return rc;
+  if (!status || !cand_offsets || !hist_offsets) return JCA_ERR_NULL;
+  rc = check_workspace(workspace, workspace_bytes, B, Nc, H);
+  if (rc) return rc;
   const WorkspaceLayout L = workspace_layout(B, Nc, H);
-  if (L.max_items >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
-  if (workspace_bytes < L.total) return JCA_ERR_WORKSPACE;
-  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(workspace);
-  int32_t* items = reinterpret_cast<int32_t*>(ws + L.items);
-  int32_t* n_items = reinterpret_cast<int32_t*>(ws + L.n_items);
   const void* kv_lo;
   const void* kv_hi;
   const int32_t* kv_count = nullptr;
@@ -736,10 +815,34 @@ extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const v
     kv_lo = hist_offsets;
     kv_hi = static_cast<const char*>(hist_offsets) + idx_bits / 8;
   }
-  if (launch_work_queue(cand_offsets, kv_lo, kv_hi, kv_count, B, Nc, Th, H, idx_bits, items,
-                        L.max_items, n_items, status, st) != cudaSuccess)
+  if (launch_work_queue(cand_offsets, kv_lo, kv_hi, kv_count, B, Nc, Th, H, idx_bits,
+                        reinterpret_cast<int32_t*>(ws + L.items), L.max_items,
+                        reinterpret_cast<int32_t*>(ws + L.n_items), status, st) != cudaSuccess)
     return JCA_ERR_CUDA;
+  return JCA_OK;
+}
+
+extern "C" int cand_only_attn_run(const void* cand_q, const void* own_k, const void* own_v,
+                                  const void* hist_k, const void* hist_v, const int8_t* hist_seg,
+                                  void* out, int out_fp32, int64_t B, int64_t Nc, int64_t Th,
+                                  int H, int d_head, float scale, void* workspace,
+                                  size_t workspace_bytes, int32_t* status,
+                                  jca_stream_t stream) {
+  int rc = check_sizes(32, d_head, B, Nc, Th, H);
+  if (rc) return rc;
+  if (!status) return JCA_ERR_NULL;
+  if (Nc > 0 && (!cand_q || !own_k || !own_v || !out)) return JCA_ERR_NULL;
+  if (Th > 0 && (!hist_k || !hist_v)) return JCA_ERR_NULL;
+  if (Nc > 0 && (!aligned(cand_q, 16) || !aligned(own_k, 16) || !aligned(own_v, 16) ||
+                 !aligned(out, 16)))
+    return JCA_ERR_ALIGN;
+  if (Th > 0 && (!aligned(hist_k, 16) || !aligned(hist_v, 16))) return JCA_ERR_ALIGN;
+  rc = check_workspace(workspace, workspace_bytes, B, Nc, H);
+  if (rc) return rc;
   if (Nc == 0) return JCA_OK;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
+  const WorkspaceLayout L = workspace_layout(B, Nc, H);
+  char* ws = static_cast<char*>(workspace);
   AttnArgs a;
   a.q = static_cast<const __nv_bfloat16*>(cand_q);
   a.dk = static_cast<const __nv_bfloat16*>(own_k);
@@ -747,8 +850,8 @@ extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const v
   a.q_seg = nullptr;
   a.kv_seg = hist_seg;
   a.out = out;
-  a.items = reinterpret_cast<const int4*>(items);
-  a.n_items = n_items;
+  a.items = reinterpret_cast<const int4*>(ws + L.items);
+  a.n_items = reinterpret_cast<const int32_t*>(ws + L.n_items);
   a.status = status;
   a.H = H;
   a.out_fp32 = out_fp32 ? 1 : 0;
@@ -756,7 +859,31 @@ extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const v
   // With no history rows at all, the key maps are never read; they point at the candidates.
   const void* kp = Th > 0 ? hist_k : own_k;
   const void* vp = Th > 0 ? hist_v : own_v;
-  return launch_attention(d_head, a, cand_q, Nc, kp, vp, Th > 0 ? Th : Nc, st);
+  return launch_attention(d_head, a, cand_q, Nc, kp, vp, Th > 0 ? Th : Nc,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const void* own_v,
+                                  const void* cand_offsets, const void* hist_k,
+                                  const void* hist_v, const void* hist_offsets,
+                                  const int8_t* hist_seg, void* out, int out_fp32, int64_t B,
+                                  int64_t Nc, int64_t Th, int H, int d_head, float scale,
+                                  int idx_bits, void* workspace, size_t workspace_bytes,
+                                  int32_t* status, jca_stream_t stream) {
+  int rc = check_sizes(idx_bits, d_head, B, Nc, Th, H);
+  if (rc) return rc;
+  if (!status || !cand_offsets || !hist_offsets) return JCA_ERR_NULL;
+  if (Nc > 0 && (!cand_q || !own_k || !own_v || !out)) return JCA_ERR_NULL;
+  if (Th > 0 && (!hist_k || !hist_v)) return JCA_ERR_NULL;
+  if (Nc > 0 && (!aligned(cand_q, 16) || !aligned(own_k, 16) || !aligned(own_v, 16) ||
+                 !aligned(out, 16)))
+    return JCA_ERR_ALIGN;
+  if (Th > 0 && (!aligned(hist_k, 16) || !aligned(hist_v, 16))) return JCA_ERR_ALIGN;
+  rc = cand_only_attn_plan(cand_offsets, hist_offsets, hist_seg, B, Nc, Th, H, d_head, idx_bits,
+                           workspace, workspace_bytes, status, stream);
+  if (rc) return rc;
+  return cand_only_attn_run(cand_q, own_k, own_v, hist_k, hist_v, hist_seg, out, out_fp32, B, Nc,
+                            Th, H, d_head, scale, workspace, workspace_bytes, status, stream);
 }
 
 extern "C" const char* jca_status_string(int code) {

@@ -40,6 +40,14 @@ _SIGNATURES = {
     "cand_only_attn_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32,
                                    c_i64, c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp, c_sz,
                                    c_vp, c_vp]),
+    "jagged_cand_attn_plan": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_i32, c_vp,
+                                      c_sz, c_vp, c_vp]),
+    "jagged_cand_attn_run": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i64, c_i64, c_i32,
+                                     c_i32, c_f32, c_vp, c_sz, c_vp, c_vp]),
+    "cand_only_attn_plan": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i64, c_i64, c_i32, c_i32, c_i32,
+                                    c_vp, c_sz, c_vp, c_vp]),
+    "cand_only_attn_run": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64,
+                                   c_i64, c_i32, c_i32, c_f32, c_vp, c_sz, c_vp, c_vp]),
 }
 
 
@@ -201,6 +209,45 @@ def cand_only_attn_fwd(cand_q, own_k, own_v, cand_offsets, hist_k, hist_v, hist_
         _ptr(hist_offsets), _ptr(hist_seg), _ptr(out), out_fp32, B, Nc, Th, H, d, float(scale),
         _idx_bits(cand_offsets), _ptr(workspace), workspace.numel(), _ptr(status),
         _stream(stream)), "cand_only_attn_fwd")
+
+
+def jagged_cand_attn_plan(offsets, candidate_start, seg, T: int, H: int, d_head: int,
+                          workspace: torch.Tensor, status: torch.Tensor, stream=None) -> int:
+    B = offsets.numel() - 1
+    return _check(lib().jagged_cand_attn_plan(
+        _ptr(offsets), _ptr(candidate_start), _ptr(seg), B, int(T), int(H), int(d_head),
+        _idx_bits(offsets), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
+        "jagged_cand_attn_plan")
+
+
+def jagged_cand_attn_run(q, k, v, out, seg, B: int, workspace: torch.Tensor, status: torch.Tensor,
+                         scale: float = 0.0, stream=None) -> int:
+    T, H, d = q.shape
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().jagged_cand_attn_run(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(seg), int(B), T, H, d, float(scale),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)), "jagged_cand_attn_run")
+
+
+def cand_only_attn_plan(cand_offsets, hist_offsets, hist_seg, Nc: int, Th: int, H: int, d_head: int,
+                        workspace: torch.Tensor, status: torch.Tensor, stream=None) -> int:
+    B = cand_offsets.numel() - 1
+    return _check(lib().cand_only_attn_plan(
+        _ptr(cand_offsets), _ptr(hist_offsets), _ptr(hist_seg), B, int(Nc), int(Th), int(H),
+        int(d_head), _idx_bits(cand_offsets), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream)), "cand_only_attn_plan")
+
+
+def cand_only_attn_run(cand_q, own_k, own_v, hist_k, hist_v, hist_seg, out, B: int,
+                       workspace: torch.Tensor, status: torch.Tensor, scale: float = 0.0,
+                       stream=None) -> int:
+    Nc, H, d = cand_q.shape
+    Th = hist_k.shape[0]
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().cand_only_attn_run(
+        _ptr(cand_q), _ptr(own_k), _ptr(own_v), _ptr(hist_k), _ptr(hist_v), _ptr(hist_seg),
+        _ptr(out), out_fp32, int(B), Nc, Th, H, d, float(scale), _ptr(workspace),
+        workspace.numel(), _ptr(status), _stream(stream)), "cand_only_attn_run")
 
 
 def jca_status_string(code: int) -> str:

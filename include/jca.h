@@ -172,6 +172,25 @@ int jagged_cand_attn_fwd(const void* q, const void* k, const void* v, void* out,
                          jca_stream_t stream);
 
 /*
+ * The two halves of jagged_cand_attn_fwd, for callers that run several attention layers over one
+ * batch layout (the ranker's full layers all share it):
+ *   jagged_cand_attn_plan  derives everything that depends only on the layout — segment IDs
+ *                          (when seg == NULL), bounds and the work queue — into `workspace`;
+ *   jagged_cand_attn_run   launches only the attention kernel, reading that plan. It may be called
+ *                          any number of times after one plan, as long as `workspace` and the
+ *                          layout arguments (seg, B, T, H, d_head) are the same as at plan time.
+ * Arguments, errors and workspace size are as for jagged_cand_attn_fwd.
+ */
+int jagged_cand_attn_plan(const void* offsets, const void* candidate_start, const int8_t* seg,
+                          int64_t B, int64_t T, int H, int d_head, int idx_bits, void* workspace,
+                          size_t workspace_bytes, int32_t* status, jca_stream_t stream);
+
+int jagged_cand_attn_run(const void* q, const void* k, const void* v, void* out, int out_fp32,
+                         const int8_t* seg, int64_t B, int64_t T, int H, int d_head, float scale,
+                         void* workspace, size_t workspace_bytes, int32_t* status,
+                         jca_stream_t stream);
+
+/*
  * Candidate-only attention layer (候选隔离注意力掩码, section 只更新候选的末尾层; the arguments mirror
  * the page's operator inputs candidate_q, history_k, history_v, own_k, own_v): each candidate of
  * user b attends to the frozen history keys/values of user b and to its own key/value only.
@@ -189,6 +208,22 @@ int cand_only_attn_fwd(const void* cand_q, const void* own_k, const void* own_v,
                        const void* hist_offsets, const int8_t* hist_seg, void* out, int out_fp32,
                        int64_t B, int64_t Nc, int64_t Th, int H, int d_head, float scale,
                        int idx_bits, void* workspace, size_t workspace_bytes, int32_t* status,
+                       jca_stream_t stream);
+
+/*
+ * The two halves of cand_only_attn_fwd (see jagged_cand_attn_plan/run): the plan holds the key
+ * intervals and the work queue of the candidate/history layout; `hist_seg` given to run must be the
+ * one given to plan.
+ */
+int cand_only_attn_plan(const void* cand_offsets, const void* hist_offsets, const int8_t* hist_seg,
+                        int64_t B, int64_t Nc, int64_t Th, int H, int d_head, int idx_bits,
+                        void* workspace, size_t workspace_bytes, int32_t* status,
+                        jca_stream_t stream);
+
+int cand_only_attn_run(const void* cand_q, const void* own_k, const void* own_v,
+                       const void* hist_k, const void* hist_v, const int8_t* hist_seg, void* out,
+                       int out_fp32, int64_t B, int64_t Nc, int64_t Th, int H, int d_head,
+                       float scale, void* workspace, size_t workspace_bytes, int32_t* status,
                        jca_stream_t stream);
 
 #ifdef __cplusplus

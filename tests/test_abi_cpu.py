@@ -24,7 +24,9 @@ def test_header_declares_the_entry_points():
     names = jca.header_functions()
     for n in ["jca_offsets_from_lengths", "jca_build_segment_ids", "jca_bounds_from_segment_ids",
               "jca_build_work_queue", "jca_max_work_items", "jca_workspace_bytes",
-              "jagged_cand_attn_fwd", "cand_only_attn_fwd", "jca_status_string"]:
+              "jagged_cand_attn_fwd", "cand_only_attn_fwd", "jca_status_string",
+              "jagged_cand_attn_plan", "jagged_cand_attn_run", "cand_only_attn_plan",
+              "cand_only_attn_run"]:
         assert n in names
 
 
