@@ -897,6 +897,8 @@ extern "C" const char* jca_status_string(int code) {
     case JCA_ERR_WORKSPACE: return "workspace smaller than jca_workspace_bytes()";
     case JCA_ERR_CUDA: return "a CUDA call failed";
     case JCA_ERR_DEVICE: return "the current device is not sm_100 (B200)";
+    case JCA_ERR_SCRATCH_LIMIT:
+      return "problem needs more scratch than the library's static array holds";
     case JCA_STATUS_BAD_LENGTH: return "negative length or offsets overflow the index type";
     case JCA_STATUS_BAD_OFFSETS: return "offsets do not start at 0, decrease, or do not end at rows";
     case JCA_STATUS_BAD_CAND_START: return "candidate_start outside [0, row length]";

@@ -48,6 +48,10 @@ _SIGNATURES = {
                                     c_vp, c_sz, c_vp, c_vp]),
     "cand_only_attn_run": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64,
                                    c_i64, c_i32, c_i32, c_f32, c_vp, c_sz, c_vp, c_vp]),
+    "jca_noalloc_scratch_bytes": (c_sz, []),
+    "jagged_cand_attn_fwd_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp,
+                                             c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp,
+                                             c_vp]),
 }
 
 
@@ -248,6 +252,27 @@ def cand_only_attn_run(cand_q, own_k, own_v, hist_k, hist_v, hist_seg, out, B: i
         _ptr(cand_q), _ptr(own_k), _ptr(own_v), _ptr(hist_k), _ptr(hist_v), _ptr(hist_seg),
         _ptr(out), out_fp32, int(B), Nc, Th, H, d, float(scale), _ptr(workspace),
         workspace.numel(), _ptr(status), _stream(stream)), "cand_only_attn_run")
+
+
+def jagged_cand_attn_fwd_noalloc(q, k, v, out, offsets, candidate_start=None, seg=None,
+                                 scale: float = 0.0, status: Optional[torch.Tensor] = None,
+                                 stream=None) -> int:
+    """jagged_cand_attn_fwd for callers that cannot allocate device memory at call time: the
+    library uses its own fixed 8 MiB static scratch array instead of a caller workspace (see
+    include/jca.h for the size limit and the sharing rules)."""
+    T, H, d = q.shape
+    B = offsets.numel() - 1
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().jagged_cand_attn_fwd_noalloc(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), _ptr(candidate_start),
+        _ptr(seg), B, T, H, d, float(scale), _idx_bits(offsets), _ptr(status), _stream(stream)),
+        "jagged_cand_attn_fwd_noalloc")
+
+
+def jca_noalloc_scratch_bytes() -> int:
+    return int(lib().jca_noalloc_scratch_bytes())
 
 
 def jca_status_string(code: int) -> str:

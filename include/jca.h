@@ -57,6 +57,8 @@ enum jca_code {
   JCA_ERR_WORKSPACE = -6,   /* workspace smaller than jca_workspace_bytes(...) */
   JCA_ERR_CUDA = -7,        /* a CUDA runtime/driver call failed (launch, tensor map, ...) */
   JCA_ERR_DEVICE = -8,      /* current device is not sm_100 */
+  JCA_ERR_SCRATCH_LIMIT = -9, /* jagged_cand_attn_fwd_noalloc: problem needs more scratch than
+                                 the library's static array (jca_noalloc_scratch_bytes()) */
   /* device-side data errors (written to *status) */
   JCA_STATUS_BAD_LENGTH = 1,     /* a sequence length is negative, or offsets overflow int32 */
   JCA_STATUS_BAD_OFFSETS = 2,    /* offsets[0] != 0, offsets decrease, or offsets[B] != rows */
@@ -225,6 +227,35 @@ int cand_only_attn_run(const void* cand_q, const void* own_k, const void* own_v,
                        int out_fp32, int64_t B, int64_t Nc, int64_t Th, int H, int d_head,
                        float scale, void* workspace, size_t workspace_bytes, int32_t* status,
                        jca_stream_t stream);
+
+/*
+ * jagged_cand_attn_fwd without a workspace argument. (No counterpart on the source pages: this is
+ * an interface for callers, not part of the method.)
+ *
+ * For callers that cannot allocate device memory when they call: a serving loop whose memory is
+ * fixed up front, a plugin that is handed only its input and output tensors, or code that must not
+ * pay cudaMalloc's implicit device synchronisation on the request path. The scratch this call
+ * needs (segment IDs, per-user bounds, the work queue) lives in one static device array inside the
+ * library, jca_noalloc_scratch_bytes() = 8 MiB, which every GPU that loads the library holds until
+ * the process exits. The call allocates and frees nothing.
+ *
+ *   Arguments, results and device-side errors: as jagged_cand_attn_fwd.
+ *   Size limit: when jca_workspace_bytes(B, T, H, d_head) exceeds jca_noalloc_scratch_bytes(),
+ *   the call returns JCA_ERR_SCRATCH_LIMIT before enqueuing anything (use jagged_cand_attn_fwd
+ *   with a workspace then). Roughly: T + 44 B + 16 H (T/128 + B + 1) bytes must fit in 8 MiB.
+ *   First call per device: it looks up the array's device address (cudaGetSymbolAddress, with
+ *   that device current) and caches it; make that first call before any stream capture.
+ *   Sharing: all calls on a device use the same array, which keeps the last call's contents (no
+ *   part of it needs to start at zero). Calls whose execution overlaps on the GPU — on different
+ *   streams without ordering between them, or from several host threads — race on it; order them
+ *   on one stream or with events.
+ */
+size_t jca_noalloc_scratch_bytes(void);
+
+int jagged_cand_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                 int out_fp32, const void* offsets, const void* candidate_start,
+                                 const int8_t* seg, int64_t B, int64_t T, int H, int d_head,
+                                 float scale, int idx_bits, int32_t* status, jca_stream_t stream);
 
 #ifdef __cplusplus
 }
