@@ -9,14 +9,20 @@
 // (history x candidate and candidate x other-candidate pairs are skipped wholesale), and the
 // candidate's self term is merged into the online softmax as a diagonal epilogue on CUDA cores.
 //
-// Kernel structure (one persistent CTA per SM, 6 warps):
-//   warp 0      TMA producer: Q tile (2 buffers), K and V tiles (2-stage rings each).
-//   warp 1      TMEM allocator and single-thread MMA issuer: S = Q K^T into one of two TMEM
-//               S buffers, O += P V into the TMEM O accumulator; completion via tcgen05.commit.
-//   warps 2..5  softmax + epilogue, one query row per thread (TMEM lane = row): masked online
-//               softmax in the log2 domain with fp32 m, l in registers, P written as bf16 to a
-//               128-byte-swizzled shared tile, lazy O rescaling (only when the running max grows
-//               by more than 2^8), then the diagonal merge, 1/l and the store.
+// Kernel structure (one persistent CTA per SM, 10 warps):
+//   warp 0      two TMA producer threads: lane 0 loads the Q tile (2 buffers) and K tiles, lane 1
+//               loads V tiles (2-stage rings each).
+//   warp 1      TMEM allocator and single-thread MMA issuer.
+//   warps 2..9  two softmax warpgroups, one query row per thread (TMEM lane = row). Group 0 takes
+//               the even key tiles of an item and group 1 the odd ones, each with its own S buffer
+//               in TMEM (P is written back over S as bf16 pairs and read from there by the PV MMA)
+//               and its own fp32 O accumulator and running max / sum. The two partial results are
+//               merged once per item in the epilogue, together with the diagonal term.
+// TMEM columns: S0 | S1 | O0 | O1 (128 each). MMA order per item: QK_0, QK_1, PV_0, QK_2, PV_1, ...
+// so the tensor core computes the next tile's S while a softmax group works on the previous one.
+// An MMA that overwrites S_w is issued after the PV that reads the P stored there, and MMAs from
+// one thread execute in issue order; a commit fires only when every earlier MMA has completed, so
+// once a group sees S_w full its previous PV into O_w is done and O_w may be rescaled in place.
 // Work items (user, head, 128-row query tile) come from the cost-sorted queue; CTA c takes items
 // c, c + grid, c + 2 grid, ... so the longest items start first.
 #include <climits>
@@ -69,12 +75,16 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
   static constexpr int NUM_BARS = 24;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_USED = OFF_MISC + 16;
+  // Epilogue exchange between the two groups' threads of a row: (max, sum, partial diagonal dot)
+  // as [2 parity][2 group][128 rows][4] fp32.
+  static constexpr int OFF_XCH = OFF_MISC + 16;
+  static constexpr int XCH_FLOATS = 2 * 2 * 128 * 4;
+  static constexpr int SMEM_USED = OFF_XCH + XCH_FLOATS * 4;
   static constexpr int SMEM_RAW = SMEM_USED + 1024;                // slack for 1 KB alignment
   // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
   static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
-  // TMEM columns: S0 | S1 (fp32 scores) | O (fp32 accumulator) | P0 | P1 (bf16 pairs).
-  static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256, TMEM_P0 = 384,
+  // TMEM columns: S0 | S1 (fp32 scores, then bf16 P over their first 64 columns) | O0 | O1.
+  static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 384,
                             TMEM_COLS = 512;
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
 };
@@ -82,11 +92,18 @@ struct Cfg {
 // Barrier slots.
 enum : int {
   kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = 6, kVFull = 8, kVEmpty = 10,
-  kSFull = 12, kSEmpty = 14, kPFull = 16, kPVDone = 18, kDrain = 20
+  kSFull = 12,   // per softmax group: S_w written by a QK
+  kPFull = 14,   // per softmax group: P_w written (and S_w read) by the group
+  kOReady = 16,  // every MMA of an item complete: O0 / O1 final
+  kOFree = 17,   // both groups have read O0 / O1 of an item
+  kXEpi = 18,    // epilogue exchange, 2 parities
+  kDrain = 20
 };
 
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
+// Warps: 0 TMA producers, 1 TMEM allocator + MMA issuer, 2..9 softmax/epilogue. Softmax warp w
+// belongs to group (w - 2) / 4 and owns TMEM lane quarter w % 4 (query rows 32 (w % 4) .. +31).
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
 
 struct Item {
   int q_row0, h, nrows, kv_lo, kv_len, holes, n_kv;
@@ -107,87 +124,125 @@ __device__ __forceinline__ Item decode_item(int4 v) {
 // ------------------------------------------------------------------------------------------
 // Producer
 // ------------------------------------------------------------------------------------------
+// Two producer threads in warp 0 walk the same item sequence: lane 0 loads Q and K tiles (slots
+// freed by QK completions), lane 1 loads V tiles (slots freed by PV completions), so a slow PV
+// never holds back the next K.
 template <int D>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV, const AttnArgs& a, uint32_t sbase,
-                              uint32_t bars, int n_items, volatile int* abort_flag) {
+                              uint32_t bars, int n_items, volatile int* abort_flag, bool loads_v) {
   using C = Cfg<D>;
-  uint32_t armed[6] = {0, 0, 0, 0, 0, 0};  // q0 q1 k0 k1 v0 v1
+  uint32_t armed[4] = {0, 0, 0, 0};  // Q or V stage 0, 1 | K stage 0, 1
   uint32_t g = 0, qi = 0;
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
     if (w.n_kv == 0) continue;
-    const int qs = qi & 1;
-    ok = mbar_wait(bars + 8 * (kQEmpty + qs), ((qi >> 1) & 1) ^ 1, abort_flag, a.status);
-    if (!ok) break;
-    mbar_arrive_expect_tx(bars + 8 * (kQFull + qs), C::TILE_BYTES);
-    ++armed[qs];
+    if (!loads_v) {
+      const int qs = qi & 1;
+      ok = mbar_wait(bars + 8 * (kQEmpty + qs), ((qi >> 1) & 1) ^ 1, abort_flag, a.status);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bars + 8 * (kQFull + qs), C::TILE_BYTES);
+      ++armed[qs];
 #pragma unroll
-    for (int c = 0; c < C::NBLK; ++c)
-      tma_load_3d(sbase + C::OFF_Q + qs * C::TILE_BYTES + c * C::BLK_BYTES, tmQ,
-                  bars + 8 * (kQFull + qs), c * C::BOX_X, w.h, w.q_row0);
-    ++qi;
+      for (int c = 0; c < C::NBLK; ++c)
+        tma_load_3d(sbase + C::OFF_Q + qs * C::TILE_BYTES + c * C::BLK_BYTES, tmQ,
+                    bars + 8 * (kQFull + qs), c * C::BOX_X, w.h, w.q_row0);
+      ++qi;
+    }
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = g & 1;
       const uint32_t ph = (g >> 1) & 1;
       const int row = w.kv_lo + j * C::BN;
-      ok = mbar_wait(bars + 8 * (kKEmpty + s), ph ^ 1, abort_flag, a.status);
+      const int empty = loads_v ? kVEmpty : kKEmpty;
+      const int full = loads_v ? kVFull : kKFull;
+      const CUtensorMap* map = loads_v ? tmV : tmK;
+      const int off = loads_v ? C::OFF_V : C::OFF_K;
+      ok = mbar_wait(bars + 8 * (empty + s), ph ^ 1, abort_flag, a.status);
       if (!ok) break;
-      mbar_arrive_expect_tx(bars + 8 * (kKFull + s), C::TILE_BYTES);
-      ++armed[2 + s];
+      mbar_arrive_expect_tx(bars + 8 * (full + s), C::TILE_BYTES);
+      ++armed[loads_v ? s : 2 + s];
 #pragma unroll
       for (int c = 0; c < C::NBLK; ++c)
-        tma_load_3d(sbase + C::OFF_K + s * C::TILE_BYTES + c * C::BLK_BYTES, tmK,
-                    bars + 8 * (kKFull + s), c * C::BOX_X, w.h, row);
-      ok = mbar_wait(bars + 8 * (kVEmpty + s), ph ^ 1, abort_flag, a.status);
-      if (!ok) break;
-      mbar_arrive_expect_tx(bars + 8 * (kVFull + s), C::TILE_BYTES);
-      ++armed[4 + s];
-#pragma unroll
-      for (int c = 0; c < C::NBLK; ++c)
-        tma_load_3d(sbase + C::OFF_V + s * C::TILE_BYTES + c * C::BLK_BYTES, tmV,
-                    bars + 8 * (kVFull + s), c * C::BOX_X, w.h, row);
+        tma_load_3d(sbase + off + s * C::TILE_BYTES + c * C::BLK_BYTES, map,
+                    bars + 8 * (full + s), c * C::BOX_X, w.h, row);
     }
   }
   if (!ok) {
     // Aborting: let every copy this thread started land before the CTA exits.
-    const int full_slot[6] = {kQFull, kQFull + 1, kKFull, kKFull + 1, kVFull, kVFull + 1};
-    for (int i = 0; i < 6; ++i)
-      if (armed[i]) mbar_wait_drain(bars + 8 * full_slot[i], (armed[i] - 1) & 1);
+    const int slot[4] = {loads_v ? kVFull : kQFull, loads_v ? kVFull + 1 : kQFull + 1, kKFull,
+                         kKFull + 1};
+    for (int i = 0; i < 4; ++i)
+      if (armed[i]) mbar_wait_drain(bars + 8 * slot[i], (armed[i] - 1) & 1);
   }
 }
 
 // ------------------------------------------------------------------------------------------
 // MMA issuer
 // ------------------------------------------------------------------------------------------
-// O += P V for key tile gg (P from TMEM buffer gg % 2), whose first `valid` keys are real: only
-// ceil(valid / 16) k-steps are issued.
+struct MmaState {
+  uint32_t p_seen[2];   // P-full completions consumed, per softmax group
+  uint32_t items;       // items with key tiles issued so far
+  // Operand descriptors of the Q buffers and K / V stages (start address of the first k-step); a
+  // k-step adds a compile-time offset to the low bits (shared addresses stay below 256 KB, so the
+  // 14-bit field never carries). Scalars, selected by buffer index, so they stay in registers.
+  uint64_t q0, q1, k0, k1, v0, v1;
+};
+
+// Tensor-core issue is paced by execution (one 128x128x16 MMA takes about 64 cycles), so the issue
+// paths below keep the work between two MMAs minimal: precomputed descriptors, compile-time
+// offsets, and straight-line code for full tiles.
 template <int D>
-__device__ __forceinline__ bool issue_pv(uint32_t gg, int valid, bool first, uint32_t sbase,
+__device__ __forceinline__ void mma_qk(uint32_t d_tmem, uint64_t qa, uint64_t kb, uint32_t idesc) {
+  using C = Cfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < C::KSTEPS_QK; ++kk) {
+    const uint32_t off = ((kk / C::KSTEPS_PER_BLK) * C::BLK_BYTES +
+                          (kk % C::KSTEPS_PER_BLK) * 32) >> 4;
+    tc_mma(d_tmem, qa + off, kb + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_t vb, int ksteps,
+                                       bool overwrite) {
+  using C = Cfg<D>;
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(C::BM, D, false, true);
+  constexpr uint32_t kStep = (16 * C::SW) >> 4;   // 16 key rows of V per k-step
+  if (ksteps == C::KSTEPS_PV) {
+#pragma unroll
+    for (int kk = 0; kk < C::KSTEPS_PV; ++kk)
+      tc_mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u, vb + (uint64_t)(kk * kStep), kIdescPV,
+                (overwrite && kk == 0) ? 0u : 1u);
+  } else {
+    for (int kk = 0; kk < ksteps; ++kk)
+      tc_mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u, vb + (uint64_t)(kk * kStep), kIdescPV,
+                (overwrite && kk == 0) ? 0u : 1u);
+  }
+}
+
+// O_w += P_w V for tile j of the item (global tile gg: V stage), whose first `valid` keys are
+// real: only ceil(valid / 16) k-steps are issued. P_w is read from the first 64 TMEM columns of
+// S_w (bf16 pairs: 16 keys = 8 columns per k-step).
+template <int D>
+__device__ __forceinline__ bool issue_pv(uint32_t gg, int j, int valid, MmaState& st,
                                          uint32_t bars, uint32_t tmem, const AttnArgs& a,
                                          volatile int* abort_flag) {
   using C = Cfg<D>;
-  constexpr uint32_t kIdescPV = idesc_bf16_f32(C::BM, D, false, true);
+  const int w = j & 1;
   const int s = gg & 1;
   const uint32_t ph = (gg >> 1) & 1;
   if (!mbar_wait(bars + 8 * (kVFull + s), ph, abort_flag, a.status)) return false;
-  if (!mbar_wait(bars + 8 * (kPFull + s), ph, abort_flag, a.status)) return false;
+  if (!mbar_wait(bars + 8 * (kPFull + w), st.p_seen[w] & 1, abort_flag, a.status)) return false;
+  ++st.p_seen[w];
+  // The first PV of an item overwrites O0: both groups must have read the previous item's O.
+  if (j == 0 && st.items > 0 &&
+      !mbar_wait(bars + 8 * kOFree, (st.items - 1) & 1, abort_flag, a.status))
+    return false;
   tc_fence_after();
-  const uint32_t p_tmem = tmem + C::TMEM_P0 + (uint32_t)s * 64u;
-  const uint32_t v_base = sbase + C::OFF_V + s * C::TILE_BYTES;
-  const int ksteps = (valid + 15) >> 4;
-#pragma unroll
-  for (int kk = 0; kk < C::KSTEPS_PV; ++kk) {
-    if (kk >= ksteps) break;
-    // P: 16 keys = 8 TMEM columns per k-step; V: MN-major (head dim contiguous), 16 key rows.
-    const uint64_t bdesc =
-        smem_desc(v_base + kk * 16 * C::SW, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
-    tc_mma_ts(tmem + C::TMEM_O, p_tmem + (uint32_t)kk * 8u, bdesc, kIdescPV,
-              (first && kk == 0) ? 0u : 1u);
-  }
+  mma_pv<D>(tmem + (w ? C::TMEM_O1 : C::TMEM_O0), tmem + (w ? C::TMEM_S1 : C::TMEM_S0),
+            s ? st.v1 : st.v0, (valid + 15) >> 4, j < 2);
   tc_commit(bars + 8 * (kVEmpty + s));
-  tc_commit(bars + 8 * (kPVDone + s));
   return true;
 }
 
@@ -195,8 +250,18 @@ template <int D>
 __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          int n_items, volatile int* abort_flag) {
   using C = Cfg<D>;
-  // QK^T with N = keys of the tile rounded up to 16 (the last key tile of a user is trimmed).
-  constexpr uint32_t kIdescQK0 = idesc_bf16_f32(C::BM, 16, false, false) & ~(0x3Fu << 17);
+  constexpr uint32_t kIdescQKFull = idesc_bf16_f32(C::BM, C::BN, false, false);
+  // QK^T of a trimmed tile: N = keys of the tile rounded up to 16.
+  constexpr uint32_t kIdescQK0 = kIdescQKFull & ~(0x3Fu << 17);
+  MmaState st;
+  st.p_seen[0] = st.p_seen[1] = 0;
+  st.items = 0;
+  st.q0 = smem_desc(sbase + C::OFF_Q, 16, 8 * C::SW, C::LAYOUT);
+  st.q1 = smem_desc(sbase + C::OFF_Q + C::TILE_BYTES, 16, 8 * C::SW, C::LAYOUT);
+  st.k0 = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
+  st.k1 = smem_desc(sbase + C::OFF_K + C::TILE_BYTES, 16, 8 * C::SW, C::LAYOUT);
+  st.v0 = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
+  st.v1 = smem_desc(sbase + C::OFF_V + C::TILE_BYTES, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
   uint32_t g = 0, qi = 0;
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
@@ -206,40 +271,36 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     ok = mbar_wait(bars + 8 * (kQFull + qs), (qi >> 1) & 1, abort_flag, a.status);
     if (!ok) break;
     tc_fence_after();
-    const uint32_t q_base = sbase + C::OFF_Q + qs * C::TILE_BYTES;
+    const uint64_t qa = qs ? st.q1 : st.q0;
     int prev_valid = 0;
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = g & 1;
       const uint32_t ph = (g >> 1) & 1;
       const int valid = min(C::BN, w.kv_len - j * C::BN);
-      const uint32_t idesc_qk = kIdescQK0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17);
-      ok = mbar_wait(bars + 8 * (kKFull + s), ph, abort_flag, a.status) &&
-           mbar_wait(bars + 8 * (kSEmpty + s), ph ^ 1, abort_flag, a.status);
+      const uint32_t idesc_qk =
+          valid == C::BN ? kIdescQKFull
+                         : (kIdescQK0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17));
+      ok = mbar_wait(bars + 8 * (kKFull + s), ph, abort_flag, a.status);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t k_base = sbase + C::OFF_K + s * C::TILE_BYTES;
-      const uint32_t d_tmem = tmem + (s ? C::TMEM_S1 : C::TMEM_S0);
-#pragma unroll
-      for (int kk = 0; kk < C::KSTEPS_QK; ++kk) {
-        const uint32_t off =
-            (kk / C::KSTEPS_PER_BLK) * C::BLK_BYTES + (kk % C::KSTEPS_PER_BLK) * 32;
-        tc_mma(d_tmem, smem_desc(q_base + off, 16, 8 * C::SW, C::LAYOUT),
-               smem_desc(k_base + off, 16, 8 * C::SW, C::LAYOUT), idesc_qk, kk > 0 ? 1u : 0u);
-      }
+      mma_qk<D>(tmem + ((j & 1) ? C::TMEM_S1 : C::TMEM_S0), qa, s ? st.k1 : st.k0, idesc_qk);
       tc_commit(bars + 8 * (kKEmpty + s));
-      tc_commit(bars + 8 * (kSFull + s));
+      tc_commit(bars + 8 * (kSFull + (j & 1)));
+      // After the item's last QK the Q buffer may be refilled for a later item.
+      if (j == w.n_kv - 1) tc_commit(bars + 8 * (kQEmpty + qs));
       // PV of the previous key tile goes behind this QK, so the tensor core computes the next
-      // S while the softmax warps work on the previous one.
+      // S while the softmax groups work on earlier tiles.
       if (j > 0) {
-        ok = issue_pv<D>(g - 1, prev_valid, j == 1, sbase, bars, tmem, a, abort_flag);
+        ok = issue_pv<D>(g - 1, j - 1, prev_valid, st, bars, tmem, a, abort_flag);
         if (!ok) break;
       }
       prev_valid = valid;
     }
     if (!ok) break;
-    ok = issue_pv<D>(g - 1, prev_valid, w.n_kv == 1, sbase, bars, tmem, a, abort_flag);
+    ok = issue_pv<D>(g - 1, w.n_kv - 1, prev_valid, st, bars, tmem, a, abort_flag);
     if (!ok) break;
-    tc_commit(bars + 8 * (kQEmpty + qs));
+    tc_commit(bars + 8 * kOReady);
+    ++st.items;
     ++qi;
   }
   if (!ok) {
@@ -252,88 +313,161 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
 // ------------------------------------------------------------------------------------------
 // Softmax + epilogue
 // ------------------------------------------------------------------------------------------
-template <int D>
-__device__ __forceinline__ void rescale_o_row(uint32_t t_o, float alpha) {
-  if constexpr (D == 16) {
-    uint32_t r[16];
-    tmem_ld_x16(t_o, r);
-    tmem_wait_ld();
-    reg_fence16(r);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-    tmem_st_x16(t_o, r);
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t t, uint32_t* r) {
+  if constexpr (N == 8) {
+    tmem_ld_x8(t, r);
+  } else if constexpr (N == 16) {
+    tmem_ld_x16(t, r);
+  } else {
+    tmem_ld_x32(t, r);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t t, const uint32_t* r) {
+  if constexpr (N == 8) {
+    tmem_st_x8(t, r);
+  } else if constexpr (N == 16) {
+    tmem_st_x16(t, r);
+  } else {
+    tmem_st_x32(t, r);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void reg_fence_cols(uint32_t* r) {
+  if constexpr (N == 8) {
+    reg_fence8(r);
   } else {
 #pragma unroll
-    for (int c = 0; c < D; c += 32) {
-      uint32_t r[32];
-      tmem_ld_x32(t_o + c, r);
-      tmem_wait_ld();
-      reg_fence16(r);
-      reg_fence16(r + 16);
+    for (int i = 0; i < N; i += 16) reg_fence16(r + i);
+  }
+}
+
+// One O row (D columns) of this group, multiplied by alpha in place in TMEM.
+template <int D>
+__device__ __forceinline__ void rescale_o_row(uint32_t t_o, float alpha) {
+  constexpr int CW = D < 32 ? D : 32;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-      tmem_st_x32(t_o + c, r);
-    }
+  for (int c0 = 0; c0 < D; c0 += CW) {
+    uint32_t u[CW];
+    tmem_ld_cols<CW>(t_o + c0, u);
+    tmem_wait_ld();
+    reg_fence_cols<CW>(u);
+#pragma unroll
+    for (int i = 0; i < CW; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+    tmem_st_cols<CW>(t_o + c0, u);
   }
   tmem_wait_st();
 }
 
-// Epilogue of one query row: diagonal merge (a candidate's own key/value), normalisation and
-// store. Every lane of the warp calls this (the TMEM loads are warp-collective); rows outside the
-// tile only skip their memory accesses.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Epilogue of one query row, shared by the row's two threads (one per group): each thread handles
+// D / 2 output columns. They exchange (max, sum, partial diagonal dot) through shared memory
+// (bounded mbarrier wait), merge the two groups' partial softmax states
+//   M = max(m0, m1),  L = l0 2^(m0 - M) + l1 2^(m1 - M),  O = O0 2^(m0 - M) + O1 2^(m1 - M),
+// then merge the diagonal term of a candidate row (its own key and value), normalise and store.
+// Every softmax thread calls this (the exchange and the TMEM loads are collective); rows outside
+// the tile only skip their memory accesses. The candidate's q and k halves are loaded together,
+// and each O chunk of both groups is read behind one TMEM wait.
 template <int D>
-__device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int r, uint32_t t_o,
-                                           bool has_o, float m, float l) {
+__device__ __forceinline__ bool finish_row(const AttnArgs& a, const Item& w, int r, int grp,
+                                           uint32_t t_lane, float m, float l, float* xepi,
+                                           uint32_t ebar, uint32_t e, volatile int* abort_flag) {
+  using C = Cfg<D>;
+  constexpr int HD = D / 2;
+  constexpr int NV = HD / 8;                 // 16-byte vectors in this thread's half row
   const bool row_ok = r < w.nrows;
   const int row = w.q_row0 + (row_ok ? r : 0);
-  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
+  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D + (size_t)grp * HD;
   const int seg = row_ok ? (a.q_seg ? (int)a.q_seg[row] : -1) : 0;
-  float alpha = 1.f, beta = 0.f;
-  if (seg == -1) {
+  const bool cand = seg == -1;
+  float dot = 0.f;
+  if (cand) {
     const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
     const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
+    uint4 qv[NV], kv[NV];
+#pragma unroll
+    for (int c = 0; c < NV; ++c) {
+      qv[c] = ld_global_nc_v4(qp + c);
+      kv[c] = ld_global_nc_v4(kp + c);
+    }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int c = 0; c < D / 8; ++c) {
-      const uint4 qa = ld_global_nc_v4(qp + c);
-      const uint4 ka = ld_global_nc_v4(kp + c);
-      acc[0] = fmaf(bf16_lo(qa.x), bf16_lo(ka.x), fmaf(bf16_hi(qa.x), bf16_hi(ka.x), acc[0]));
-      acc[1] = fmaf(bf16_lo(qa.y), bf16_lo(ka.y), fmaf(bf16_hi(qa.y), bf16_hi(ka.y), acc[1]));
-      acc[2] = fmaf(bf16_lo(qa.z), bf16_lo(ka.z), fmaf(bf16_hi(qa.z), bf16_hi(ka.z), acc[2]));
-      acc[3] = fmaf(bf16_lo(qa.w), bf16_lo(ka.w), fmaf(bf16_hi(qa.w), bf16_hi(ka.w), acc[3]));
+    for (int c = 0; c < NV; ++c) {
+      acc[0] = fmaf(bf16_lo(qv[c].x), bf16_lo(kv[c].x), fmaf(bf16_hi(qv[c].x), bf16_hi(kv[c].x), acc[0]));
+      acc[1] = fmaf(bf16_lo(qv[c].y), bf16_lo(kv[c].y), fmaf(bf16_hi(qv[c].y), bf16_hi(kv[c].y), acc[1]));
+      acc[2] = fmaf(bf16_lo(qv[c].z), bf16_lo(kv[c].z), fmaf(bf16_hi(qv[c].z), bf16_hi(kv[c].z), acc[2]));
+      acc[3] = fmaf(bf16_lo(qv[c].w), bf16_lo(kv[c].w), fmaf(bf16_hi(qv[c].w), bf16_hi(kv[c].w), acc[3]));
     }
-    const float sd = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * a.scale_log2;
-    const float m_new = fmaxf(m, sd);
-    alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
+    dot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+  }
+  float* mine = xepi + ((e & 1) * 2 + grp) * 512 + 4 * r;
+  const float* other = xepi + ((e & 1) * 2 + (grp ^ 1)) * 512 + 4 * r;
+  mine[0] = m;
+  mine[1] = l;
+  mine[2] = dot;
+  mbar_arrive(ebar + 8 * (e & 1));
+  if (!__all_sync(0xffffffffu, mbar_wait(ebar + 8 * (e & 1), (e >> 1) & 1, abort_flag, a.status)))
+    return false;
+  // Index by group so that both threads evaluate the same expressions in the same order.
+  const float m0 = grp == 0 ? m : other[0], m1 = grp == 0 ? other[0] : m;
+  const float l0 = grp == 0 ? l : other[1], l1 = grp == 0 ? other[1] : l;
+  const float d0 = grp == 0 ? dot : other[2], d1 = grp == 0 ? other[2] : dot;
+  const float M = fmaxf(m0, m1);
+  float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M);
+  float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M);
+  float L = l0 * a0 + l1 * a1;
+  float beta = 0.f;
+  if (cand) {
+    const float sd = (d0 + d1) * a.scale_log2;
+    const float m_new = fmaxf(M, sd);
+    const float b = (M == -INFINITY) ? 0.f : fast_exp2(M - m_new);
     beta = fast_exp2(sd - m_new);
-    l = l * alpha + beta;
+    a0 *= b;
+    a1 *= b;
+    L = L * b + beta;
   }
   // Padding queries (segment 0) see no key and output 0.
-  const float inv = (seg != 0 && l > 0.f) ? 1.f / l : 0.f;
-  constexpr int CW = D < 32 ? D : 32;   // columns per TMEM load
+  const float inv = (seg != 0 && L > 0.f) ? 1.f / L : 0.f;
+  constexpr int CW = HD < 32 ? HD : 32;   // columns per TMEM load
 #pragma unroll
-  for (int c0 = 0; c0 < D; c0 += CW) {
-    float o[CW];
-    if (has_o) {
-      uint32_t u[CW];
-      if constexpr (CW == 32) {
-        tmem_ld_x32(t_o + c0, u);
-        tmem_wait_ld();
-        reg_fence16(u);
-        reg_fence16(u + 16);
-      } else {
-        tmem_ld_x16(t_o + c0, u);
-        tmem_wait_ld();
-        reg_fence16(u);
-      }
+  for (int c0 = 0; c0 < HD; c0 += CW) {
+    // o = a0 O0 + a1 O1 over this chunk; both groups' chunks are read behind one wait. Whether
+    // an item has key tiles of group 0 / 1 is warp-uniform (item-level), so the branches are too.
+    uint32_t o_bits[CW];
+    if (w.n_kv >= 2) {
+      uint32_t u1[CW];
+      tmem_ld_cols<CW>(t_lane + C::TMEM_O0 + grp * HD + c0, o_bits);
+      tmem_ld_cols<CW>(t_lane + C::TMEM_O1 + grp * HD + c0, u1);
+      tmem_wait_ld();
+      reg_fence_cols<CW>(o_bits);
+      reg_fence_cols<CW>(u1);
 #pragma unroll
-      for (int i = 0; i < CW; ++i) o[i] = __uint_as_float(u[i]);
+      for (int i = 0; i < CW; ++i)
+        o_bits[i] = __float_as_uint(
+            fmaf(__uint_as_float(u1[i]), a1, __uint_as_float(o_bits[i]) * a0));
+    } else if (w.n_kv == 1) {
+      tmem_ld_cols<CW>(t_lane + C::TMEM_O0 + grp * HD + c0, o_bits);
+      tmem_wait_ld();
+      reg_fence_cols<CW>(o_bits);
+#pragma unroll
+      for (int i = 0; i < CW; ++i) o_bits[i] = __float_as_uint(__uint_as_float(o_bits[i]) * a0);
     } else {
 #pragma unroll
-      for (int i = 0; i < CW; ++i) o[i] = 0.f;
+      for (int i = 0; i < CW; ++i) o_bits[i] = 0u;
     }
+    float o[CW];
+#pragma unroll
+    for (int i = 0; i < CW; ++i) o[i] = __uint_as_float(o_bits[i]);
     if (!row_ok) continue;
-    if (seg == -1) {
+    if (cand) {
       const uint4* vp = reinterpret_cast<const uint4*>(a.dv + base + c0);
 #pragma unroll
       for (int c = 0; c < CW / 8; ++c) {
@@ -341,8 +475,8 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int
         const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          o[8 * c + 2 * i] = fmaf(o[8 * c + 2 * i], alpha, beta * bf16_lo(vw[i]));
-          o[8 * c + 2 * i + 1] = fmaf(o[8 * c + 2 * i + 1], alpha, beta * bf16_hi(vw[i]));
+          o[8 * c + 2 * i] = fmaf(beta, bf16_lo(vw[i]), o[8 * c + 2 * i]);
+          o[8 * c + 2 * i + 1] = fmaf(beta, bf16_hi(vw[i]), o[8 * c + 2 * i + 1]);
         }
       }
     }
@@ -367,40 +501,49 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int
                            pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
     }
   }
+  return true;
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
+// Start moving a candidate row's q, k and v halves towards L2 at the beginning of an item, so that
+// the epilogue's loads of them do not wait on HBM.
+template <int D>
+__device__ __forceinline__ void prefetch_diag(const AttnArgs& a, const Item& w, int r, int grp) {
+  if (r >= w.nrows) return;
+  const int row = w.q_row0 + r;
+  if (a.q_seg && a.q_seg[row] != -1) return;
+  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D + (size_t)grp * (D / 2);
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a.q + base));
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dk + base));
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base));
 }
 
 template <int D>
-__device__ void softmax_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
+__device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, float* xepi,
                              int n_items, volatile int* abort_flag, int warp, int lane) {
   using C = Cfg<D>;
+  const int grp = (warp - 2) >> 2;            // softmax group: even (0) or odd (1) key tiles
   const int quarter = warp & 3;               // TMEM lane quarter this warp may access
   const int r = quarter * 32 + lane;          // query row of this thread inside the tile
   const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+  const uint32_t t_s = t_lane + (grp ? C::TMEM_S1 : C::TMEM_S0);
+  const uint32_t t_o = t_lane + (grp ? C::TMEM_O1 : C::TMEM_O0);
   const float sl2 = a.scale_log2;
-  uint32_t g = 0;
+  uint32_t lt = 0, oi = 0, e = 0;             // S_w fills seen, O-ready seen, exchanges done
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
-    float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
-    for (int j = 0; j < w.n_kv; ++j, ++g) {
-      const int s = g & 1;
-      const uint32_t ph = (g >> 1) & 1;
+    prefetch_diag<D>(a, w, r, grp);
+    float m = -INFINITY, l = 0.f;             // this group's running max (log2 units) and sum
+    for (int j = grp; j < w.n_kv; j += 2, ++lt) {
       const int valid = min(C::BN, w.kv_len - j * C::BN);
+      const int nchunks = (valid + 31) >> 5;
       // Edge tiles (the trimmed last tile, or any tile of a user with padding holes) are masked
       // column by column; interior tiles take the unmasked path.
       const bool edge = valid < C::BN || w.holes;
-      const int8_t* kseg = w.holes ? a.kv_seg + (w.kv_lo + j * C::BN) : nullptr;
-      const int nchunks = (valid + 31) >> 5;
-      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (kSFull + s), ph, abort_flag, a.status));
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bars + 8 * (kSFull + grp), lt & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-      const uint32_t t_s = t_lane + (s ? C::TMEM_S1 : C::TMEM_S0);
 
       // Pass 1: the whole S row in registers (four 32-column TMEM loads, one wait), then the
       // max of the raw scores (the scale is positive, so it commutes with max).
@@ -412,12 +555,10 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, u
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 128; c += 16) reg_fence16(x + c);
-      // S is in registers: the MMA warp may overwrite this buffer.
-      tc_fence_before();
-      mbar_arrive(bars + 8 * (kSEmpty + s));
       if (edge) {
         // Every row of the tile sees the same key columns: the warp builds the tile's 128-bit
         // column mask with one ballot per 32 columns (lane i tests column 32k + i).
+        const int8_t* kseg = w.holes ? a.kv_seg + (w.kv_lo + j * C::BN) : nullptr;
         uint32_t bits[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -445,16 +586,9 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, u
       const float m_use = rescale ? m_new : m;
       const float neg_m = (m_use == -INFINITY) ? 0.f : -m_use;
 
-      // P buffer s was last read by the PV of tile g - 2: it must have completed.
-      ok = __all_sync(0xffffffffu,
-                      mbar_wait(bars + 8 * (kPVDone + s), ph ^ 1, abort_flag, a.status));
-      if (!ok) break;
-      tc_fence_after();
-
-      // Pass 2: p = 2^(scale_log2 * s - m), streamed to TMEM 32 keys at a time as bf16 pairs
-      // (column k of the P buffer holds keys 2k, 2k+1). Chunks past the last real key are
-      // never read by the trimmed PV and are skipped.
-      const uint32_t t_p = t_lane + C::TMEM_P0 + (uint32_t)s * 64u;
+      // Pass 2: p = 2^(scale_log2 * s - m), written back over S_w as bf16 pairs (TMEM column k
+      // holds keys 2k, 2k+1) 32 keys at a time; chunks past the last real key are never read
+      // by the trimmed PV and are skipped.
       float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -473,34 +607,33 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, u
           pk[i / 2] = pack_bf16x2(p0, p1);
           pk[i / 2 + 1] = pack_bf16x2(p2, p3);
         }
-        tmem_st_x16(t_p + 16 * c, pk);
+        tmem_st_x16(t_s + 16 * c, pk);
       }
+      // O_w is stable here: its last PV was issued before the QK that filled S_w, and that
+      // QK's commit fired only after every earlier MMA completed. TMEM loads/stores are
+      // warp-collective: the warp rescales when any of its rows must.
       const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
-      // TMEM loads/stores are warp-collective: the warp rescales when any of its rows must.
-      // O must be stable, i.e. the PV of tile g - 1 complete.
-      if (__any_sync(0xffffffffu, rescale && j > 0)) {
-        const uint32_t gp = g - 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (kPVDone + (gp & 1)), (gp >> 1) & 1,
-                                               abort_flag, a.status));
-        if (!ok) break;
-        tc_fence_after();
-        rescale_o_row<D>(t_lane + C::TMEM_O, alpha);
-      }
+      if (__any_sync(0xffffffffu, rescale && j >= 2)) rescale_o_row<D>(t_o, alpha);
       l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
       m = m_use;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bars + 8 * (kPFull + s));
+      mbar_arrive(bars + 8 * (kPFull + grp));
     }
     if (!ok) break;
     if (w.n_kv > 0) {
-      const uint32_t gl = g - 1;   // last key tile of this item
-      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (kPVDone + (gl & 1)), (gl >> 1) & 1,
-                                             abort_flag, a.status));
+      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * kOReady, oi & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
     }
-    finish_row<D>(a, w, r, t_lane + C::TMEM_O, w.n_kv > 0, m, l);
+    ok = finish_row<D>(a, w, r, grp, t_lane, m, l, xepi, bars + 8 * kXEpi, e, abort_flag);
+    ++e;
+    if (ok && w.n_kv > 0) {
+      // O0 / O1 have been read: the next item's first PV may overwrite them.
+      tc_fence_before();
+      mbar_arrive(bars + 8 * kOFree);
+      ++oi;
+    }
   }
 }
 
@@ -521,6 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bars = sbase + C::OFF_BAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  float* xepi = reinterpret_cast<float*>(smem + C::OFF_XCH);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -532,10 +666,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (kVFull + i), 1);
       mbar_init(bars + 8 * (kVEmpty + i), 1);
       mbar_init(bars + 8 * (kSFull + i), 1);
-      mbar_init(bars + 8 * (kSEmpty + i), kSoftmaxThreads);
-      mbar_init(bars + 8 * (kPFull + i), kSoftmaxThreads);
-      mbar_init(bars + 8 * (kPVDone + i), 1);
+      mbar_init(bars + 8 * (kPFull + i), kSoftmaxThreads / 2);
+      mbar_init(bars + 8 * (kXEpi + i), kSoftmaxThreads);
     }
+    mbar_init(bars + 8 * kOReady, 1);
+    mbar_init(bars + 8 * kOFree, kSoftmaxThreads);
     mbar_init(bars + 8 * kDrain, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -557,11 +692,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_items = *a.n_items;
 
   if (warp == 0) {
-    if (lane == 0) producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag);
+    if (lane < 2)
+      producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag, lane == 1);
   } else if (warp == 1) {
     if (lane == 0) mma_role<D>(a, sbase, bars, tmem, n_items, abort_flag);
   } else {
-    softmax_role<D>(a, sbase, bars, tmem, n_items, abort_flag, warp, lane);
+    softmax_role<D>(a, bars, tmem, xepi, n_items, abort_flag, warp, lane);
   }
 
   tc_fence_before();
