@@ -9,21 +9,23 @@
 // (history x candidate and candidate x other-candidate pairs are skipped wholesale), and the
 // candidate's self term is merged into the online softmax as a diagonal epilogue on CUDA cores.
 //
-// Kernel structure (one persistent CTA per SM, 10 warps):
-//   warp 0      two TMA producer threads: lane 0 loads the Q tile (2 buffers) and K tiles, lane 1
-//               loads V tiles (2-stage rings each).
+// Kernel structure (one persistent CTA per SM, 10 warps). A work item is a block of up to 256 query
+// rows of one (user, head): two 128-row query tiles A and B that share every K/V tile load.
+//   warp 0      two TMA producer threads: lane 0 loads the item's Q tiles and the K tiles, lane 1
+//               loads the V tiles (2-stage rings each).
 //   warp 1      TMEM allocator and single-thread MMA issuer.
-//   warps 2..9  two softmax warpgroups, one query row per thread (TMEM lane = row). Group 0 takes
-//               the even key tiles of an item and group 1 the odd ones, each with its own S buffer
-//               in TMEM (P is written back over S as bf16 pairs and read from there by the PV MMA)
-//               and its own fp32 O accumulator and running max / sum. The two partial results are
-//               merged once per item in the epilogue, together with the diagonal term.
-// TMEM columns: S0 | S1 | O0 | O1 (128 each). MMA order per item: QK_0, QK_1, PV_0, QK_2, PV_1, ...
-// so the tensor core computes the next tile's S while a softmax group works on the previous one.
-// An MMA that overwrites S_w is issued after the PV that reads the P stored there, and MMAs from
-// one thread execute in issue order; a commit fires only when every earlier MMA has completed, so
-// once a group sees S_w full its previous PV into O_w is done and O_w may be rescaled in place.
-// Work items (user, head, 128-row query tile) come from the cost-sorted queue; CTA c takes items
+//   warps 2..9  two softmax warpgroups, one per query tile, one query row per thread (TMEM lane =
+//               row). Each group owns an S buffer in TMEM (P is written back over S as bf16 pairs
+//               and read from there by the PV MMA), an fp32 O accumulator and its rows' running
+//               max / sum, and finalises its own rows (diagonal term, 1/l, store).
+// TMEM columns: S_A | S_B | O_A | O_B (128 each). MMA order per key tile j:
+//   QK_A(j), PV_B(j-1), QK_B(j), PV_A(j)
+// so each group's chain (softmax -> PV -> next QK) is short and the tensor core works for one
+// group while the other runs its softmax. An MMA that overwrites S_w is issued after the PV that
+// reads the P stored there, and MMAs from one thread execute in issue order; a commit fires only
+// when every earlier MMA has completed, so once a group sees S_w full its previous PV into O_w is
+// done and O_w may be rescaled in place.
+// Work items (user, head, 256-row query block) come from the cost-sorted queue; CTA c takes items
 // c, c + grid, c + 2 grid, ... so the longest items start first.
 #include <climits>
 #include <cmath>
@@ -75,15 +77,11 @@ struct Cfg {
   static constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
   static constexpr int NUM_BARS = 24;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  // Epilogue exchange between the two groups' threads of a row: (max, sum, partial diagonal dot)
-  // as [2 parity][2 group][128 rows][4] fp32.
-  static constexpr int OFF_XCH = OFF_MISC + 16;
-  static constexpr int XCH_FLOATS = 2 * 2 * 128 * 4;
-  static constexpr int SMEM_USED = OFF_XCH + XCH_FLOATS * 4;
+  static constexpr int SMEM_USED = OFF_MISC + 16;
   static constexpr int SMEM_RAW = SMEM_USED + 1024;                // slack for 1 KB alignment
   // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
   static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
-  // TMEM columns: S0 | S1 (fp32 scores, then bf16 P over their first 64 columns) | O0 | O1.
+  // TMEM columns: S_A | S_B (fp32 scores, then bf16 P over their first 64 columns) | O_A | O_B.
   static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 384,
                             TMEM_COLS = 512;
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
@@ -91,17 +89,18 @@ struct Cfg {
 
 // Barrier slots.
 enum : int {
-  kQFull = 0, kQEmpty = 2, kKFull = 4, kKEmpty = 6, kVFull = 8, kVEmpty = 10,
+  kQFull = 0, kQEmpty = 2,   // per query tile (A, B)
+  kKFull = 4, kKEmpty = 6, kVFull = 8, kVEmpty = 10,   // per K / V stage
   kSFull = 12,   // per softmax group: S_w written by a QK
   kPFull = 14,   // per softmax group: P_w written (and S_w read) by the group
-  kOReady = 16,  // every MMA of an item complete: O0 / O1 final
-  kOFree = 17,   // both groups have read O0 / O1 of an item
-  kXEpi = 18,    // epilogue exchange, 2 parities
+  kOReady = 16,  // per group: the item's last PV into O_w complete
+  kOFree = 18,   // per group: O_w of the item read by the group
   kDrain = 20
 };
 
 // Warps: 0 TMA producers, 1 TMEM allocator + MMA issuer, 2..9 softmax/epilogue. Softmax warp w
-// belongs to group (w - 2) / 4 and owns TMEM lane quarter w % 4 (query rows 32 (w % 4) .. +31).
+// belongs to group (w - 2) / 4 (query tile A or B) and owns TMEM lane quarter w % 4 (rows
+// 32 (w % 4) .. +31 of its tile).
 constexpr int kThreads = 320;
 constexpr int kSoftmaxThreads = 256;
 
@@ -112,8 +111,8 @@ struct Item {
 __device__ __forceinline__ Item decode_item(int4 v) {
   Item w;
   w.q_row0 = v.x;
-  w.h = v.y >> 8;
-  w.nrows = v.y & 255;
+  w.h = v.y >> 9;
+  w.nrows = v.y & 511;
   w.kv_lo = v.z;
   w.kv_len = v.w & 0x7fffffff;
   w.holes = (int)((unsigned)v.w >> 31);
@@ -124,31 +123,35 @@ __device__ __forceinline__ Item decode_item(int4 v) {
 // ------------------------------------------------------------------------------------------
 // Producer
 // ------------------------------------------------------------------------------------------
-// Two producer threads in warp 0 walk the same item sequence: lane 0 loads Q and K tiles (slots
-// freed by QK completions), lane 1 loads V tiles (slots freed by PV completions), so a slow PV
-// never holds back the next K.
+// Two producer threads in warp 0 walk the same item sequence: lane 0 loads the Q tiles (one buffer
+// per query tile, refilled once the item's last QK of that tile completed) and the K tiles (slots
+// freed by QK completions), lane 1 loads the V tiles (slots freed by PV completions), so a slow
+// PV never holds back the next K.
 template <int D>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV, const AttnArgs& a, uint32_t sbase,
                               uint32_t bars, int n_items, volatile int* abort_flag, bool loads_v) {
   using C = Cfg<D>;
-  uint32_t armed[4] = {0, 0, 0, 0};  // Q or V stage 0, 1 | K stage 0, 1
-  uint32_t g = 0, qi = 0;
+  uint32_t armed[4] = {0, 0, 0, 0};  // Q A, Q B (or V stage 0, 1) | K stage 0, 1
+  uint32_t g = 0;
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
     if (w.n_kv == 0) continue;
     if (!loads_v) {
-      const int qs = qi & 1;
-      ok = mbar_wait(bars + 8 * (kQEmpty + qs), ((qi >> 1) & 1) ^ 1, abort_flag, a.status);
-      if (!ok) break;
-      mbar_arrive_expect_tx(bars + 8 * (kQFull + qs), C::TILE_BYTES);
-      ++armed[qs];
+      const int ntiles = w.nrows > C::BM ? 2 : 1;
+      for (int t = 0; ok && t < ntiles; ++t) {
+        // Load #n of Q buffer t waits for the release of load #n-1 (immediate the first time).
+        ok = mbar_wait(bars + 8 * (kQEmpty + t), (armed[t] & 1) ^ 1, abort_flag, a.status);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bars + 8 * (kQFull + t), C::TILE_BYTES);
+        ++armed[t];
 #pragma unroll
-      for (int c = 0; c < C::NBLK; ++c)
-        tma_load_3d(sbase + C::OFF_Q + qs * C::TILE_BYTES + c * C::BLK_BYTES, tmQ,
-                    bars + 8 * (kQFull + qs), c * C::BOX_X, w.h, w.q_row0);
-      ++qi;
+        for (int c = 0; c < C::NBLK; ++c)
+          tma_load_3d(sbase + C::OFF_Q + t * C::TILE_BYTES + c * C::BLK_BYTES, tmQ,
+                      bars + 8 * (kQFull + t), c * C::BOX_X, w.h, w.q_row0 + t * C::BM);
+      }
+      if (!ok) break;
     }
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = g & 1;
@@ -182,10 +185,11 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
 // ------------------------------------------------------------------------------------------
 struct MmaState {
   uint32_t p_seen[2];   // P-full completions consumed, per softmax group
-  uint32_t items;       // items with key tiles issued so far
+  uint32_t o_items[2];  // items whose O_w was written, per group (O-free completions expected)
+  uint32_t q_seen[2];   // Q-full completions consumed, per query tile
   // Operand descriptors of the Q buffers and K / V stages (start address of the first k-step); a
   // k-step adds a compile-time offset to the low bits (shared addresses stay below 256 KB, so the
-  // 14-bit field never carries). Scalars, selected by buffer index, so they stay in registers.
+  // 14-bit field never carries). Scalars, selected by index, so they stay in registers.
   uint64_t q0, q1, k0, k1, v0, v1;
 };
 
@@ -221,28 +225,26 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_
   }
 }
 
-// O_w += P_w V for tile j of the item (global tile gg: V stage), whose first `valid` keys are
+// O_w += P_w V for key tile jj of the item (global tile gg: V stage), whose first `valid` keys are
 // real: only ceil(valid / 16) k-steps are issued. P_w is read from the first 64 TMEM columns of
-// S_w (bf16 pairs: 16 keys = 8 columns per k-step).
+// S_w (bf16 pairs: 16 keys = 8 columns per k-step). The first PV of an item overwrites O_w, so it
+// waits until the group has read the previous item's O_w.
 template <int D>
-__device__ __forceinline__ bool issue_pv(uint32_t gg, int j, int valid, MmaState& st,
+__device__ __forceinline__ bool issue_pv(int grp, uint32_t gg, int jj, int valid, MmaState& st,
                                          uint32_t bars, uint32_t tmem, const AttnArgs& a,
                                          volatile int* abort_flag) {
   using C = Cfg<D>;
-  const int w = j & 1;
   const int s = gg & 1;
-  const uint32_t ph = (gg >> 1) & 1;
-  if (!mbar_wait(bars + 8 * (kVFull + s), ph, abort_flag, a.status)) return false;
-  if (!mbar_wait(bars + 8 * (kPFull + w), st.p_seen[w] & 1, abort_flag, a.status)) return false;
-  ++st.p_seen[w];
-  // The first PV of an item overwrites O0: both groups must have read the previous item's O.
-  if (j == 0 && st.items > 0 &&
-      !mbar_wait(bars + 8 * kOFree, (st.items - 1) & 1, abort_flag, a.status))
+  if (!mbar_wait(bars + 8 * (kVFull + s), (gg >> 1) & 1, abort_flag, a.status)) return false;
+  if (!mbar_wait(bars + 8 * (kPFull + grp), st.p_seen[grp] & 1, abort_flag, a.status))
+    return false;
+  ++st.p_seen[grp];
+  if (jj == 0 && st.o_items[grp] > 0 &&
+      !mbar_wait(bars + 8 * (kOFree + grp), (st.o_items[grp] - 1) & 1, abort_flag, a.status))
     return false;
   tc_fence_after();
-  mma_pv<D>(tmem + (w ? C::TMEM_O1 : C::TMEM_O0), tmem + (w ? C::TMEM_S1 : C::TMEM_S0),
-            s ? st.v1 : st.v0, (valid + 15) >> 4, j < 2);
-  tc_commit(bars + 8 * (kVEmpty + s));
+  mma_pv<D>(tmem + (grp ? C::TMEM_O1 : C::TMEM_O0), tmem + (grp ? C::TMEM_S1 : C::TMEM_S0),
+            s ? st.v1 : st.v0, (valid + 15) >> 4, jj == 0);
   return true;
 }
 
@@ -255,53 +257,77 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
   constexpr uint32_t kIdescQK0 = kIdescQKFull & ~(0x3Fu << 17);
   MmaState st;
   st.p_seen[0] = st.p_seen[1] = 0;
-  st.items = 0;
+  st.o_items[0] = st.o_items[1] = 0;
+  st.q_seen[0] = st.q_seen[1] = 0;
   st.q0 = smem_desc(sbase + C::OFF_Q, 16, 8 * C::SW, C::LAYOUT);
   st.q1 = smem_desc(sbase + C::OFF_Q + C::TILE_BYTES, 16, 8 * C::SW, C::LAYOUT);
   st.k0 = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
   st.k1 = smem_desc(sbase + C::OFF_K + C::TILE_BYTES, 16, 8 * C::SW, C::LAYOUT);
   st.v0 = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
   st.v1 = smem_desc(sbase + C::OFF_V + C::TILE_BYTES, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
-  uint32_t g = 0, qi = 0;
+  uint32_t g = 0;
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
     if (w.n_kv == 0) continue;
-    const int qs = qi & 1;
-    ok = mbar_wait(bars + 8 * (kQFull + qs), (qi >> 1) & 1, abort_flag, a.status);
+    const bool has_b = w.nrows > C::BM;
+    ok = mbar_wait(bars + 8 * kQFull, st.q_seen[0] & 1, abort_flag, a.status);
     if (!ok) break;
+    ++st.q_seen[0];
     tc_fence_after();
-    const uint64_t qa = qs ? st.q1 : st.q0;
     int prev_valid = 0;
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = g & 1;
       const uint32_t ph = (g >> 1) & 1;
+      const bool last = j == w.n_kv - 1;
       const int valid = min(C::BN, w.kv_len - j * C::BN);
       const uint32_t idesc_qk =
           valid == C::BN ? kIdescQKFull
                          : (kIdescQK0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17));
+      const uint64_t kb = s ? st.k1 : st.k0;
       ok = mbar_wait(bars + 8 * (kKFull + s), ph, abort_flag, a.status);
       if (!ok) break;
       tc_fence_after();
-      mma_qk<D>(tmem + ((j & 1) ? C::TMEM_S1 : C::TMEM_S0), qa, s ? st.k1 : st.k0, idesc_qk);
-      tc_commit(bars + 8 * (kKEmpty + s));
-      tc_commit(bars + 8 * (kSFull + (j & 1)));
-      // After the item's last QK the Q buffer may be refilled for a later item.
-      if (j == w.n_kv - 1) tc_commit(bars + 8 * (kQEmpty + qs));
-      // PV of the previous key tile goes behind this QK, so the tensor core computes the next
-      // S while the softmax groups work on earlier tiles.
-      if (j > 0) {
-        ok = issue_pv<D>(g - 1, j - 1, prev_valid, st, bars, tmem, a, abort_flag);
-        if (!ok) break;
+      // QK_A(j)
+      mma_qk<D>(tmem + C::TMEM_S0, st.q0, kb, idesc_qk);
+      tc_commit(bars + 8 * kSFull);
+      if (last) tc_commit(bars + 8 * kQEmpty);
+      if (has_b) {
+        // PV_B(j-1): the V stage of tile j-1 is released after both groups' PVs.
+        if (j > 0) {
+          ok = issue_pv<D>(1, g - 1, j - 1, prev_valid, st, bars, tmem, a, abort_flag);
+          if (!ok) break;
+          tc_commit(bars + 8 * (kVEmpty + ((g - 1) & 1)));
+        }
+        // QK_B(j)
+        if (j == 0) {
+          ok = mbar_wait(bars + 8 * (kQFull + 1), st.q_seen[1] & 1, abort_flag, a.status);
+          if (!ok) break;
+          ++st.q_seen[1];
+          tc_fence_after();
+        }
+        mma_qk<D>(tmem + C::TMEM_S1, st.q1, kb, idesc_qk);
+        tc_commit(bars + 8 * (kSFull + 1));
+        if (last) tc_commit(bars + 8 * (kQEmpty + 1));
       }
+      tc_commit(bars + 8 * (kKEmpty + s));
+      // PV_A(j)
+      ok = issue_pv<D>(0, g, j, valid, st, bars, tmem, a, abort_flag);
+      if (!ok) break;
+      if (!has_b) tc_commit(bars + 8 * (kVEmpty + s));
+      if (last) tc_commit(bars + 8 * kOReady);
       prev_valid = valid;
     }
     if (!ok) break;
-    ok = issue_pv<D>(g - 1, w.n_kv - 1, prev_valid, st, bars, tmem, a, abort_flag);
-    if (!ok) break;
-    tc_commit(bars + 8 * kOReady);
-    ++st.items;
-    ++qi;
+    ++st.o_items[0];
+    if (has_b) {
+      // PV_B of the item's last key tile.
+      ok = issue_pv<D>(1, g - 1, w.n_kv - 1, prev_valid, st, bars, tmem, a, abort_flag);
+      if (!ok) break;
+      tc_commit(bars + 8 * (kVEmpty + ((g - 1) & 1)));
+      tc_commit(bars + 8 * (kOReady + 1));
+      ++st.o_items[1];
+    }
   }
   if (!ok) {
     // Aborting: wait until every MMA this thread issued has completed.
@@ -368,109 +394,76 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Epilogue of one query row, shared by the row's two threads (one per group): each thread handles
-// D / 2 output columns. They exchange (max, sum, partial diagonal dot) through shared memory
-// (bounded mbarrier wait), merge the two groups' partial softmax states
-//   M = max(m0, m1),  L = l0 2^(m0 - M) + l1 2^(m1 - M),  O = O0 2^(m0 - M) + O1 2^(m1 - M),
-// then merge the diagonal term of a candidate row (its own key and value), normalise and store.
-// Every softmax thread calls this (the exchange and the TMEM loads are collective); rows outside
-// the tile only skip their memory accesses. The candidate's q and k halves are loaded together,
-// and each O chunk of both groups is read behind one TMEM wait.
+// Epilogue of one query row (every thread of a group calls this; the TMEM loads are collective and
+// rows outside the tile only skip their memory accesses): read O_w, release it to the MMA warp,
+// merge the diagonal term of a candidate row (its own key and value), normalise and store.
 template <int D>
-__device__ __forceinline__ bool finish_row(const AttnArgs& a, const Item& w, int r, int grp,
-                                           uint32_t t_lane, float m, float l, float* xepi,
-                                           uint32_t ebar, uint32_t e, volatile int* abort_flag) {
-  using C = Cfg<D>;
-  constexpr int HD = D / 2;
-  constexpr int NV = HD / 8;                 // 16-byte vectors in this thread's half row
-  const bool row_ok = r < w.nrows;
-  const int row = w.q_row0 + (row_ok ? r : 0);
-  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D + (size_t)grp * HD;
+__device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int row_in_item,
+                                           uint32_t t_o, bool has_o, float m, float l,
+                                           uint32_t o_free_bar) {
+  const bool row_ok = row_in_item < w.nrows;
+  const int row = w.q_row0 + (row_ok ? row_in_item : 0);
+  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
   const int seg = row_ok ? (a.q_seg ? (int)a.q_seg[row] : -1) : 0;
   const bool cand = seg == -1;
-  float dot = 0.f;
+  float alpha = 1.f, beta = 0.f;
   if (cand) {
     const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
     const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
-    uint4 qv[NV], kv[NV];
-#pragma unroll
-    for (int c = 0; c < NV; ++c) {
-      qv[c] = ld_global_nc_v4(qp + c);
-      kv[c] = ld_global_nc_v4(kp + c);
-    }
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    constexpr int HV = D / 16 > 0 ? D / 16 : 1;   // 16-byte vectors per half row (at least 1)
 #pragma unroll
-    for (int c = 0; c < NV; ++c) {
-      acc[0] = fmaf(bf16_lo(qv[c].x), bf16_lo(kv[c].x), fmaf(bf16_hi(qv[c].x), bf16_hi(kv[c].x), acc[0]));
-      acc[1] = fmaf(bf16_lo(qv[c].y), bf16_lo(kv[c].y), fmaf(bf16_hi(qv[c].y), bf16_hi(kv[c].y), acc[1]));
-      acc[2] = fmaf(bf16_lo(qv[c].z), bf16_lo(kv[c].z), fmaf(bf16_hi(qv[c].z), bf16_hi(kv[c].z), acc[2]));
-      acc[3] = fmaf(bf16_lo(qv[c].w), bf16_lo(kv[c].w), fmaf(bf16_hi(qv[c].w), bf16_hi(kv[c].w), acc[3]));
+    for (int h0 = 0; h0 < D / 8; h0 += HV) {
+      uint4 qv[HV], kv[HV];
+#pragma unroll
+      for (int c = 0; c < HV; ++c) {
+        qv[c] = ld_global_nc_v4(qp + h0 + c);
+        kv[c] = ld_global_nc_v4(kp + h0 + c);
+      }
+#pragma unroll
+      for (int c = 0; c < HV; ++c) {
+        acc[0] = fmaf(bf16_lo(qv[c].x), bf16_lo(kv[c].x), fmaf(bf16_hi(qv[c].x), bf16_hi(kv[c].x), acc[0]));
+        acc[1] = fmaf(bf16_lo(qv[c].y), bf16_lo(kv[c].y), fmaf(bf16_hi(qv[c].y), bf16_hi(kv[c].y), acc[1]));
+        acc[2] = fmaf(bf16_lo(qv[c].z), bf16_lo(kv[c].z), fmaf(bf16_hi(qv[c].z), bf16_hi(kv[c].z), acc[2]));
+        acc[3] = fmaf(bf16_lo(qv[c].w), bf16_lo(kv[c].w), fmaf(bf16_hi(qv[c].w), bf16_hi(kv[c].w), acc[3]));
+      }
     }
-    dot = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-  }
-  float* mine = xepi + ((e & 1) * 2 + grp) * 512 + 4 * r;
-  const float* other = xepi + ((e & 1) * 2 + (grp ^ 1)) * 512 + 4 * r;
-  mine[0] = m;
-  mine[1] = l;
-  mine[2] = dot;
-  mbar_arrive(ebar + 8 * (e & 1));
-  if (!__all_sync(0xffffffffu, mbar_wait(ebar + 8 * (e & 1), (e >> 1) & 1, abort_flag, a.status)))
-    return false;
-  // Index by group so that both threads evaluate the same expressions in the same order.
-  const float m0 = grp == 0 ? m : other[0], m1 = grp == 0 ? other[0] : m;
-  const float l0 = grp == 0 ? l : other[1], l1 = grp == 0 ? other[1] : l;
-  const float d0 = grp == 0 ? dot : other[2], d1 = grp == 0 ? other[2] : dot;
-  const float M = fmaxf(m0, m1);
-  float a0 = (m0 == -INFINITY) ? 0.f : fast_exp2(m0 - M);
-  float a1 = (m1 == -INFINITY) ? 0.f : fast_exp2(m1 - M);
-  float L = l0 * a0 + l1 * a1;
-  float beta = 0.f;
-  if (cand) {
-    const float sd = (d0 + d1) * a.scale_log2;
-    const float m_new = fmaxf(M, sd);
-    const float b = (M == -INFINITY) ? 0.f : fast_exp2(M - m_new);
+    const float sd = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * a.scale_log2;
+    const float m_new = fmaxf(m, sd);
+    alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
     beta = fast_exp2(sd - m_new);
-    a0 *= b;
-    a1 *= b;
-    L = L * b + beta;
+    l = l * alpha + beta;
   }
   // Padding queries (segment 0) see no key and output 0.
-  const float inv = (seg != 0 && L > 0.f) ? 1.f / L : 0.f;
-  constexpr int CW = HD < 32 ? HD : 32;   // columns per TMEM load
+  const float inv = (seg != 0 && l > 0.f) ? 1.f / l : 0.f;
+  constexpr int CW = D < 32 ? D : 32;            // columns per TMEM load
+  constexpr int PER = (D / CW) >= 2 ? 2 : 1;     // loads per TMEM wait
 #pragma unroll
-  for (int c0 = 0; c0 < HD; c0 += CW) {
-    // o = a0 O0 + a1 O1 over this chunk; both groups' chunks are read behind one wait. Whether
-    // an item has key tiles of group 0 / 1 is warp-uniform (item-level), so the branches are too.
-    uint32_t o_bits[CW];
-    if (w.n_kv >= 2) {
-      uint32_t u1[CW];
-      tmem_ld_cols<CW>(t_lane + C::TMEM_O0 + grp * HD + c0, o_bits);
-      tmem_ld_cols<CW>(t_lane + C::TMEM_O1 + grp * HD + c0, u1);
+  for (int c0 = 0; c0 < D; c0 += CW * PER) {
+    uint32_t u[CW * PER];
+    if (has_o) {
+#pragma unroll
+      for (int p = 0; p < PER; ++p) tmem_ld_cols<CW>(t_o + c0 + p * CW, u + p * CW);
       tmem_wait_ld();
-      reg_fence_cols<CW>(o_bits);
-      reg_fence_cols<CW>(u1);
 #pragma unroll
-      for (int i = 0; i < CW; ++i)
-        o_bits[i] = __float_as_uint(
-            fmaf(__uint_as_float(u1[i]), a1, __uint_as_float(o_bits[i]) * a0));
-    } else if (w.n_kv == 1) {
-      tmem_ld_cols<CW>(t_lane + C::TMEM_O0 + grp * HD + c0, o_bits);
-      tmem_wait_ld();
-      reg_fence_cols<CW>(o_bits);
-#pragma unroll
-      for (int i = 0; i < CW; ++i) o_bits[i] = __float_as_uint(__uint_as_float(o_bits[i]) * a0);
+      for (int p = 0; p < PER; ++p) reg_fence_cols<CW>(u + p * CW);
+      if (c0 + CW * PER >= D) {
+        // O_w has been read: the next item's first PV may overwrite it.
+        tc_fence_before();
+        mbar_arrive(o_free_bar);
+      }
     } else {
 #pragma unroll
-      for (int i = 0; i < CW; ++i) o_bits[i] = 0u;
+      for (int i = 0; i < CW * PER; ++i) u[i] = 0u;
     }
-    float o[CW];
-#pragma unroll
-    for (int i = 0; i < CW; ++i) o[i] = __uint_as_float(o_bits[i]);
     if (!row_ok) continue;
+    float o[CW * PER];
+#pragma unroll
+    for (int i = 0; i < CW * PER; ++i) o[i] = __uint_as_float(u[i]) * alpha;
     if (cand) {
       const uint4* vp = reinterpret_cast<const uint4*>(a.dv + base + c0);
 #pragma unroll
-      for (int c = 0; c < CW / 8; ++c) {
+      for (int c = 0; c < CW * PER / 8; ++c) {
         const uint4 va = ld_global_nc_v4(vp + c);
         const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
 #pragma unroll
@@ -482,59 +475,63 @@ __device__ __forceinline__ bool finish_row(const AttnArgs& a, const Item& w, int
     }
     if (seg == 0) {
 #pragma unroll
-      for (int i = 0; i < CW; ++i) o[i] = 0.f;
+      for (int i = 0; i < CW * PER; ++i) o[i] = 0.f;
     }
     if (a.out_fp32) {
       float4* op = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base + c0);
 #pragma unroll
-      for (int c = 0; c < CW / 4; ++c)
+      for (int c = 0; c < CW * PER / 4; ++c)
         op[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
                             o[4 * c + 3] * inv);
     } else {
       uint4* op =
           reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base + c0);
 #pragma unroll
-      for (int c = 0; c < CW / 8; ++c)
+      for (int c = 0; c < CW * PER / 8; ++c)
         op[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
                            pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
                            pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
                            pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
     }
   }
-  return true;
 }
 
-// Start moving a candidate row's q, k and v halves towards L2 at the beginning of an item, so that
-// the epilogue's loads of them do not wait on HBM.
+// Start moving a candidate row's q, k and v towards L2 at the beginning of an item, so that the
+// epilogue's loads of them do not wait on HBM.
 template <int D>
-__device__ __forceinline__ void prefetch_diag(const AttnArgs& a, const Item& w, int r, int grp) {
-  if (r >= w.nrows) return;
-  const int row = w.q_row0 + r;
+__device__ __forceinline__ void prefetch_diag(const AttnArgs& a, const Item& w, int row_in_item) {
+  if (row_in_item >= w.nrows) return;
+  const int row = w.q_row0 + row_in_item;
   if (a.q_seg && a.q_seg[row] != -1) return;
-  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D + (size_t)grp * (D / 2);
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(a.q + base));
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dk + base));
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base));
+  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
+#pragma unroll
+  for (int c = 0; c < D * 2; c += 128) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.q + base + c / 2));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dk + base + c / 2));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base + c / 2));
+  }
 }
 
 template <int D>
-__device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, float* xepi,
-                             int n_items, volatile int* abort_flag, int warp, int lane) {
+__device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, int n_items,
+                             volatile int* abort_flag, int warp, int lane) {
   using C = Cfg<D>;
-  const int grp = (warp - 2) >> 2;            // softmax group: even (0) or odd (1) key tiles
+  const int grp = (warp - 2) >> 2;            // query tile A (0) or B (1) of each item
   const int quarter = warp & 3;               // TMEM lane quarter this warp may access
-  const int r = quarter * 32 + lane;          // query row of this thread inside the tile
+  const int r = quarter * 32 + lane;          // query row of this thread inside its tile
+  const int row_in_item = grp * C::BM + r;
   const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
   const uint32_t t_s = t_lane + (grp ? C::TMEM_S1 : C::TMEM_S0);
   const uint32_t t_o = t_lane + (grp ? C::TMEM_O1 : C::TMEM_O0);
   const float sl2 = a.scale_log2;
-  uint32_t lt = 0, oi = 0, e = 0;             // S_w fills seen, O-ready seen, exchanges done
+  uint32_t lt = 0, oi = 0;                    // S_w fills and O_w-ready completions seen
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
-    prefetch_diag<D>(a, w, r, grp);
-    float m = -INFINITY, l = 0.f;             // this group's running max (log2 units) and sum
-    for (int j = grp; j < w.n_kv; j += 2, ++lt) {
+    if (grp == 1 && w.nrows <= C::BM) continue;   // the item has no tile B
+    prefetch_diag<D>(a, w, row_in_item);
+    float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
+    for (int j = 0; j < w.n_kv; ++j, ++lt) {
       const int valid = min(C::BN, w.kv_len - j * C::BN);
       const int nchunks = (valid + 31) >> 5;
       // Edge tiles (the trimmed last tile, or any tile of a user with padding holes) are masked
@@ -613,7 +610,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, fl
       // QK's commit fired only after every earlier MMA completed. TMEM loads/stores are
       // warp-collective: the warp rescales when any of its rows must.
       const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
-      if (__any_sync(0xffffffffu, rescale && j >= 2)) rescale_o_row<D>(t_o, alpha);
+      if (__any_sync(0xffffffffu, rescale && j >= 1)) rescale_o_row<D>(t_o, alpha);
       l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
       m = m_use;
       tmem_wait_st();
@@ -622,18 +619,13 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, fl
     }
     if (!ok) break;
     if (w.n_kv > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * kOReady, oi & 1, abort_flag, a.status));
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bars + 8 * (kOReady + grp), oi & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
-    }
-    ok = finish_row<D>(a, w, r, grp, t_lane, m, l, xepi, bars + 8 * kXEpi, e, abort_flag);
-    ++e;
-    if (ok && w.n_kv > 0) {
-      // O0 / O1 have been read: the next item's first PV may overwrite them.
-      tc_fence_before();
-      mbar_arrive(bars + 8 * kOFree);
       ++oi;
     }
+    finish_row<D>(a, w, row_in_item, t_o, w.n_kv > 0, m, l, bars + 8 * (kOFree + grp));
   }
 }
 
@@ -654,7 +646,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bars = sbase + C::OFF_BAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  float* xepi = reinterpret_cast<float*>(smem + C::OFF_XCH);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
@@ -667,10 +658,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (kVEmpty + i), 1);
       mbar_init(bars + 8 * (kSFull + i), 1);
       mbar_init(bars + 8 * (kPFull + i), kSoftmaxThreads / 2);
-      mbar_init(bars + 8 * (kXEpi + i), kSoftmaxThreads);
+      mbar_init(bars + 8 * (kOReady + i), 1);
+      mbar_init(bars + 8 * (kOFree + i), kSoftmaxThreads / 2);
     }
-    mbar_init(bars + 8 * kOReady, 1);
-    mbar_init(bars + 8 * kOFree, kSoftmaxThreads);
     mbar_init(bars + 8 * kDrain, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -697,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) mma_role<D>(a, sbase, bars, tmem, n_items, abort_flag);
   } else {
-    softmax_role<D>(a, bars, tmem, xepi, n_items, abort_flag, warp, lane);
+    softmax_role<D>(a, bars, tmem, n_items, abort_flag, warp, lane);
   }
 
   tc_fence_before();

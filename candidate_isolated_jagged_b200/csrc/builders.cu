@@ -179,7 +179,8 @@ __global__ void bounds_kernel(const int8_t* __restrict__ seg, const IdxT* __rest
 }
 
 // ---------------------------------------------------------------------------------------------
-// Work queue: counting sort of (user, head, query tile) items by key-tile count, descending.
+// Work queue: counting sort of (user, head, 256-row query pair) items by key-tile count,
+// descending.
 // A single block: pass 1 validates and histograms, a block scan turns bucket sizes into start
 // positions (largest cost first), pass 2 emits each user's items contiguously (head-major, then
 // query tile) at a position claimed with an atomic on its bucket cursor.
@@ -209,7 +210,7 @@ __global__ void __launch_bounds__(1024) work_queue_kernel(
       s_bad = 1;
       continue;
     }
-    const long long nq = (e - s + kTileM - 1) / kTileM;
+    const long long nq = (e - s + kItemRows - 1) / kItemRows;
     const long long nkv = (hi - lo + kTileN - 1) / kTileN;
     const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
     if (nq) atomicAdd(&s_cnt[key], (unsigned long long)(nq * H));
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(1024) work_queue_kernel(
   for (int64_t b = tid; b < B; b += blockDim.x) {
     const long long s = (long long)qoff[b], e = (long long)qoff[b + 1];
     const long long lo = (long long)kvlo[b], hi = (long long)kvhi[b];
-    const long long nq = (e - s + kTileM - 1) / kTileM;
+    const long long nq = (e - s + kItemRows - 1) / kItemRows;
     if (nq == 0) continue;
     const long long nkv = (hi - lo + kTileN - 1) / kTileN;
     const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
@@ -267,9 +268,9 @@ __global__ void __launch_bounds__(1024) work_queue_kernel(
     const int w = (int)(hi - lo) | (holes << 31);
     for (int h = 0; h < H; ++h) {
       for (long long t = 0; t < nq; ++t) {
-        const long long row0 = s + t * kTileM;
-        const int rows = (int)min((long long)kTileM, e - row0);
-        items[pos + (unsigned long long)h * nq + t] = make_int4((int)row0, h * 256 + rows, (int)lo, w);
+        const long long row0 = s + t * kItemRows;
+        const int rows = (int)min((long long)kItemRows, e - row0);
+        items[pos + (unsigned long long)h * nq + t] = make_int4((int)row0, (h << 9) | rows, (int)lo, w);
       }
     }
   }
@@ -281,7 +282,7 @@ inline int grid_for_rows(int64_t B) { return (int)(B < (1 << 20) ? B : (1 << 20)
 }  // namespace
 
 int64_t max_work_items(int64_t B, int64_t rows, int H) {
-  return ((rows + kTileM - 1) / kTileM + B) * (int64_t)H;
+  return ((rows + kItemRows - 1) / kItemRows + B) * (int64_t)H;
 }
 
 WorkspaceLayout workspace_layout(int64_t B, int64_t rows, int H) {

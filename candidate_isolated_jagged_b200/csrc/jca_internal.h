@@ -9,7 +9,8 @@
 
 namespace jca {
 
-constexpr int kTileM = 128;          // query rows per work item
+constexpr int kTileM = 128;          // query rows per MMA tile (one softmax group)
+constexpr int kItemRows = 256;       // query rows per work item: two tiles sharing every K/V load
 constexpr int kTileN = 128;          // keys per key tile
 constexpr int kQueueBuckets = 1024;  // cost buckets of the work-queue counting sort
 

@@ -119,7 +119,7 @@ int jca_bounds_from_segment_ids(const int8_t* seg, const void* offsets, int64_t 
                                 void* cand_hi, int32_t* status, jca_stream_t stream);
 
 /*
- * Work queue of the attention kernels: one item per (user b, head h, 128-row query tile t),
+ * Work queue of the attention kernels: one item per (user b, head h, 256-row query block t),
  * ordered by cost (the number of 128-key tiles over the user's key interval), largest first,
  * so that a persistent kernel taking items in order approximates longest-processing-time-first.
  * Items of equal cost may come in any order.
@@ -127,8 +127,8 @@ int jca_bounds_from_segment_ids(const int8_t* seg, const void* offsets, int64_t 
  *   interval of user b is [kv_lo[b], kv_hi[b])).
  *   kv_count [B] int32 or NULL: number of valid keys inside the interval; when it differs from
  *   kv_hi - kv_lo the user's key tiles are masked key by key.
- *   items [max_items * 4] int32, written; item i = {first query row, h * 256 + rows in the
- *   tile, kv_lo, (kv_hi - kv_lo) | (holes << 31)}.
+ *   items [max_items * 4] int32, written; item i = {first query row, (h << 9) | rows in the
+ *   block (1..256), kv_lo, (kv_hi - kv_lo) | (holes << 31)}.
  *   n_items [1] int32, written.
  *   q_rows / kv_rows: rows of the query and key tensors (q_offsets[B] must equal q_rows;
  *   every key interval must lie inside [0, kv_rows)).

@@ -311,8 +311,8 @@ def allowed_pairs(offsets, seg, mask_fn=history_candidate_mask) -> int:
     return total
 
 
-def work_items(offsets, seg, H: int, tile_m: int = 128, tile_n: int = 128):
-    """The set of (user, head, query tile) items a tiled kernel must process, with each item's
+def work_items(offsets, seg, H: int, tile_m: int = 256, tile_n: int = 128):
+    """The set of (user, head, query block) items a tiled kernel must process, with each item's
     cost in key tiles over the user's history interval. Used to check the GPU work queue holds
     exactly these items (any order of equal costs, non-increasing cost)."""
     hist_lo, hist_hi, _, _, _ = bounds_from_segment_ids(seg, offsets)

@@ -55,7 +55,7 @@ def test_workspace_and_queue_bounds(L):
     assert L.jca_workspace_bytes(3, 20, 2, 16) > 0
     assert L.jca_workspace_bytes(3, 20, 2, 48) == 0       # unsupported head dim
     assert L.jca_workspace_bytes(-1, 20, 2, 16) == 0
-    assert L.jca_max_work_items(3, 1222, 4) == (10 + 3) * 4
+    assert L.jca_max_work_items(3, 1222, 4) == (5 + 3) * 4
     ws = L.jca_workspace_bytes(256, 131072, 8, 128)
     assert ws % 256 == 0 and ws >= 16 * L.jca_max_work_items(256, 131072, 8)
 

@@ -157,13 +157,13 @@ def test_work_queue_matches_item_set(idx, name):
     assert np.all(np.diff(costs) <= 0), "items must come largest cost first"
     # decode and compare as a set with the oracle's items
     users = np.searchsorted(off_np, got[:, 0], side="right") - 1
-    tiles = (got[:, 0] - off_np[users]) // 128
-    heads = got[:, 1] >> 8
+    tiles = (got[:, 0] - off_np[users]) // 256
+    heads = got[:, 1] >> 9
     decoded = sorted(zip(users.tolist(), heads.tolist(), tiles.tolist(), costs.tolist()))
     assert decoded == sorted(ref)
-    rows = got[:, 1] & 255
+    rows = got[:, 1] & 511
     L = (off_np[users + 1] - off_np[users])
-    assert np.array_equal(rows, np.minimum(128, L - tiles * 128))
+    assert np.array_equal(rows, np.minimum(256, L - tiles * 256))
     assert np.array_equal(got[:, 2], hl[users])
     holes = (got[:, 3] >> 31) & 1
     assert np.array_equal(holes, (cnt[users] != (hh - hl)[users]).astype(np.int64))

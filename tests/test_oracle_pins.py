@@ -329,7 +329,7 @@ def test_work_items_cover_every_tile():
     b = synth.three_users()
     off, seg = batch_seg(b)
     items = oracle.work_items(off, seg, b.H)
-    assert len(items) == b.H * sum(-(-int(L) // 128) for L in b.row_lengths)
+    assert len(items) == b.H * sum(-(-int(L) // 256) for L in b.row_lengths)
     costs = {(it[0]): it[3] for it in items}
     assert costs == {0: 1, 1: 1, 2: 8}
 
