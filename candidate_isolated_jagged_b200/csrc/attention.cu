@@ -54,6 +54,7 @@ struct AttnArgs {
   int32_t* status;
   int H;
   int out_fp32;
+  int out_v8;               // out is 32-byte aligned: rows are written with 32-byte stores
   float scale_log2;         // softmax scale * log2(e)
 };
 
@@ -394,41 +395,79 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Epilogue of one query row (every thread of a group calls this; the TMEM loads are collective and
-// rows outside the tile only skip their memory accesses): read O_w, release it to the MMA warp,
-// merge the diagonal term of a candidate row (its own key and value), normalise and store.
+// Score of a candidate row against its own key, scaled to log2 units (the diagonal term of the
+// mask). Plain CUDA-core dot product over 16-byte loads, half a row at a time.
 template <int D>
-__device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int row_in_item,
-                                           uint32_t t_o, bool has_o, float m, float l,
-                                           uint32_t o_free_bar) {
-  const bool row_ok = row_in_item < w.nrows;
-  const int row = w.q_row0 + (row_ok ? row_in_item : 0);
-  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
-  const int seg = row_ok ? (a.q_seg ? (int)a.q_seg[row] : -1) : 0;
+__device__ __forceinline__ float diag_score(const AttnArgs& a, size_t base) {
+  const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
+  const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  constexpr int HV = D / 16 > 0 ? D / 16 : 1;   // 16-byte vectors per half row (at least 1)
+#pragma unroll
+  for (int h0 = 0; h0 < D / 8; h0 += HV) {
+    uint4 qv[HV], kv[HV];
+#pragma unroll
+    for (int c = 0; c < HV; ++c) {
+      qv[c] = ld_global_nc_v4(qp + h0 + c);
+      kv[c] = ld_global_nc_v4(kp + h0 + c);
+    }
+#pragma unroll
+    for (int c = 0; c < HV; ++c) {
+      acc[0] = fmaf(bf16_lo(qv[c].x), bf16_lo(kv[c].x), fmaf(bf16_hi(qv[c].x), bf16_hi(kv[c].x), acc[0]));
+      acc[1] = fmaf(bf16_lo(qv[c].y), bf16_lo(kv[c].y), fmaf(bf16_hi(qv[c].y), bf16_hi(kv[c].y), acc[1]));
+      acc[2] = fmaf(bf16_lo(qv[c].z), bf16_lo(kv[c].z), fmaf(bf16_hi(qv[c].z), bf16_hi(kv[c].z), acc[2]));
+      acc[3] = fmaf(bf16_lo(qv[c].w), bf16_lo(kv[c].w), fmaf(bf16_hi(qv[c].w), bf16_hi(kv[c].w), acc[3]));
+    }
+  }
+  return ((acc[0] + acc[1]) + (acc[2] + acc[3])) * a.scale_log2;
+}
+
+// Writes 8 consecutive output values of a row (bf16 or fp32 per a.out_fp32), already normalised.
+__device__ __forceinline__ void store8(const AttnArgs& a, size_t idx, const float* o) {
+  if (a.out_fp32) {
+    float* op = reinterpret_cast<float*>(a.out) + idx;
+    if (a.out_v8) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(o[i]);
+      st_global_v8(op, w);
+    } else {
+      reinterpret_cast<float4*>(op)[0] = make_float4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<float4*>(op)[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  } else {
+    reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + idx)[0] =
+        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                   pack_bf16x2(o[6], o[7]));
+  }
+}
+
+// Writes 16 consecutive bf16 output values of a row with one 32-byte store when allowed.
+__device__ __forceinline__ void store16_bf16(const AttnArgs& a, size_t idx, const float* o) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
+  __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.out) + idx;
+  if (a.out_v8) {
+    st_global_v8(op, w);
+  } else {
+    reinterpret_cast<uint4*>(op)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(op)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+// Epilogue of one query row (every thread of a group calls this; the TMEM loads are collective and
+// rows outside the tile only skip their memory accesses). The diagonal score sd and the row's own
+// value vv were fetched before O_w was complete, so that after it completes only the TMEM reads,
+// the merge, the normalisation and the stores remain: read O_w, release it to the MMA warp, merge
+// the diagonal term of a candidate row, normalise and store.
+template <int D>
+__device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int seg, size_t base,
+                                           uint32_t t_o, bool has_o, float m, float l, float sd,
+                                           const uint4 (&vv)[D / 8], uint32_t o_free_bar) {
   const bool cand = seg == -1;
   float alpha = 1.f, beta = 0.f;
   if (cand) {
-    const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
-    const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    constexpr int HV = D / 16 > 0 ? D / 16 : 1;   // 16-byte vectors per half row (at least 1)
-#pragma unroll
-    for (int h0 = 0; h0 < D / 8; h0 += HV) {
-      uint4 qv[HV], kv[HV];
-#pragma unroll
-      for (int c = 0; c < HV; ++c) {
-        qv[c] = ld_global_nc_v4(qp + h0 + c);
-        kv[c] = ld_global_nc_v4(kp + h0 + c);
-      }
-#pragma unroll
-      for (int c = 0; c < HV; ++c) {
-        acc[0] = fmaf(bf16_lo(qv[c].x), bf16_lo(kv[c].x), fmaf(bf16_hi(qv[c].x), bf16_hi(kv[c].x), acc[0]));
-        acc[1] = fmaf(bf16_lo(qv[c].y), bf16_lo(kv[c].y), fmaf(bf16_hi(qv[c].y), bf16_hi(kv[c].y), acc[1]));
-        acc[2] = fmaf(bf16_lo(qv[c].z), bf16_lo(kv[c].z), fmaf(bf16_hi(qv[c].z), bf16_hi(kv[c].z), acc[2]));
-        acc[3] = fmaf(bf16_lo(qv[c].w), bf16_lo(kv[c].w), fmaf(bf16_hi(qv[c].w), bf16_hi(kv[c].w), acc[3]));
-      }
-    }
-    const float sd = ((acc[0] + acc[1]) + (acc[2] + acc[3])) * a.scale_log2;
     const float m_new = fmaxf(m, sd);
     alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
     beta = fast_exp2(sd - m_new);
@@ -436,6 +475,7 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int
   }
   // Padding queries (segment 0) see no key and output 0.
   const float inv = (seg != 0 && l > 0.f) ? 1.f / l : 0.f;
+  const float scale_o = alpha * inv, scale_v = beta * inv;
   constexpr int CW = D < 32 ? D : 32;            // columns per TMEM load
   constexpr int PER = (D / CW) >= 2 ? 2 : 1;     // loads per TMEM wait
 #pragma unroll
@@ -459,39 +499,25 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, const Item& w, int
     if (!row_ok) continue;
     float o[CW * PER];
 #pragma unroll
-    for (int i = 0; i < CW * PER; ++i) o[i] = __uint_as_float(u[i]) * alpha;
+    for (int i = 0; i < CW * PER; ++i) o[i] = __uint_as_float(u[i]) * scale_o;
     if (cand) {
-      const uint4* vp = reinterpret_cast<const uint4*>(a.dv + base + c0);
 #pragma unroll
       for (int c = 0; c < CW * PER / 8; ++c) {
-        const uint4 va = ld_global_nc_v4(vp + c);
+        const uint4 va = vv[c0 / 8 + c];
         const uint32_t vw[4] = {va.x, va.y, va.z, va.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          o[8 * c + 2 * i] = fmaf(beta, bf16_lo(vw[i]), o[8 * c + 2 * i]);
-          o[8 * c + 2 * i + 1] = fmaf(beta, bf16_hi(vw[i]), o[8 * c + 2 * i + 1]);
+          o[8 * c + 2 * i] = fmaf(scale_v, bf16_lo(vw[i]), o[8 * c + 2 * i]);
+          o[8 * c + 2 * i + 1] = fmaf(scale_v, bf16_hi(vw[i]), o[8 * c + 2 * i + 1]);
         }
       }
     }
-    if (seg == 0) {
-#pragma unroll
-      for (int i = 0; i < CW * PER; ++i) o[i] = 0.f;
-    }
     if (a.out_fp32) {
-      float4* op = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + base + c0);
 #pragma unroll
-      for (int c = 0; c < CW * PER / 4; ++c)
-        op[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv, o[4 * c + 2] * inv,
-                            o[4 * c + 3] * inv);
+      for (int c = 0; c < CW * PER; c += 8) store8(a, base + c0 + c, o + c);
     } else {
-      uint4* op =
-          reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + base + c0);
 #pragma unroll
-      for (int c = 0; c < CW * PER / 8; ++c)
-        op[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
-                           pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
-                           pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
-                           pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+      for (int c = 0; c < CW * PER; c += 16) store16_bf16(a, base + c0 + c, o + c);
     }
   }
 }
@@ -530,6 +556,12 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, in
     const Item w = decode_item(a.items[it]);
     if (grp == 1 && w.nrows <= C::BM) continue;   // the item has no tile B
     prefetch_diag<D>(a, w, row_in_item);
+    const bool row_ok = row_in_item < w.nrows;
+    const int row = w.q_row0 + (row_ok ? row_in_item : 0);
+    const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
+    const int seg = row_ok ? (a.q_seg ? (int)a.q_seg[row] : -1) : 0;
+    float sd = -INFINITY;                     // diagonal score of a candidate row
+    if (w.n_kv == 0 && seg == -1) sd = diag_score<D>(a, base);
     float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
     for (int j = 0; j < w.n_kv; ++j, ++lt) {
       const int valid = min(C::BN, w.kv_len - j * C::BN);
@@ -616,8 +648,19 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, in
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars + 8 * (kPFull + grp));
+      // The diagonal score needs no TMEM: a candidate row computes it while the next S_w (or, for
+      // a one-tile item, O_w) is being produced.
+      if (j == 0 && seg == -1) sd = diag_score<D>(a, base);
     }
     if (!ok) break;
+    // The row's own value is fetched while the item's last PV runs.
+    uint4 vv[D / 8];
+    {
+      const uint4* vp = reinterpret_cast<const uint4*>(a.dv + base);
+#pragma unroll
+      for (int c = 0; c < D / 8; ++c)
+        vv[c] = seg == -1 ? ld_global_nc_v4(vp + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
     if (w.n_kv > 0) {
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bars + 8 * (kOReady + grp), oi & 1, abort_flag, a.status));
@@ -625,7 +668,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, in
       tc_fence_after();
       ++oi;
     }
-    finish_row<D>(a, w, row_in_item, t_o, w.n_kv > 0, m, l, bars + 8 * (kOFree + grp));
+    finish_row<D>(a, row_ok, seg, base, t_o, w.n_kv > 0, m, l, sd, vv, bars + 8 * (kOFree + grp));
   }
 }
 
@@ -778,7 +821,9 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
   if (!make_map<D>(&tmQ, q, Tq, a.H) || !make_map<D>(&tmK, k, Tkv, a.H) ||
       !make_map<D>(&tmV, v, Tkv, a.H))
     return JCA_ERR_CUDA;
-  jagged_attn_kernel<D><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, a);
+  AttnArgs args = a;
+  args.out_v8 = aligned(a.out, 32) ? 1 : 0;
+  jagged_attn_kernel<D><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, args);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }
 
