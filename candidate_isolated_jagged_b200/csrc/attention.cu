@@ -76,9 +76,11 @@ struct Cfg {
   static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
-  static constexpr int NUM_BARS = 24;
+  static constexpr int NUM_BARS = 26;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_USED = OFF_MISC + 16;
+  // Diagonal scores of the candidate rows: two item slots of kItemRows floats.
+  static constexpr int OFF_DIAG = OFF_MISC + 16;
+  static constexpr int SMEM_USED = OFF_DIAG + 2 * kItemRows * 4;
   static constexpr int SMEM_RAW = SMEM_USED + 1024;                // slack for 1 KB alignment
   // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
   static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
@@ -96,14 +98,17 @@ enum : int {
   kPFull = 14,   // per softmax group: P_w written (and S_w read) by the group
   kOReady = 16,  // per group: the item's last PV into O_w complete
   kOFree = 18,   // per group: O_w of the item read by the group
-  kDrain = 20
+  kDrain = 20,
+  kDiagFull = 22,   // per slot: an item's diagonal scores written by the diagonal warps
+  kDiagEmpty = 24   // per slot: the item's scores taken by every softmax thread
 };
 
-// Warps: 0 TMA producers, 1 TMEM allocator + MMA issuer, 2..9 softmax/epilogue. Softmax warp w
-// belongs to group (w - 2) / 4 (query tile A or B) and owns TMEM lane quarter w % 4 (rows
-// 32 (w % 4) .. +31 of its tile).
-constexpr int kThreads = 320;
+// Warps: 0 TMA producers, 1 TMEM allocator + MMA issuer, 2..9 softmax/epilogue, 10..11 diagonal
+// scores. Softmax warp w belongs to group (w - 2) / 4 (query tile A or B) and owns TMEM lane
+// quarter w % 4 (rows 32 (w % 4) .. +31 of its tile).
+constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
+constexpr int kDiagThreads = 64;
 
 struct Item {
   int q_row0, h, nrows, kv_lo, kv_len, holes, n_kv;
@@ -522,25 +527,43 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int s
   }
 }
 
-// Start moving a candidate row's q, k and v towards L2 at the beginning of an item, so that the
-// epilogue's loads of them do not wait on HBM.
+// Diagonal scores, computed by two warps up to one item ahead of the softmax warps so that no
+// softmax thread waits on the q / k loads: thread t covers rows t, t + 64, t + 128 and t + 192 of
+// each item and deposits the score (-inf for a row without a diagonal term) in the item's slot of
+// a two-slot shared array; it also starts moving each candidate row's own value towards L2 for
+// the epilogue. Slot s is reused for the item after next once all 256 softmax threads have taken
+// the scores out of it.
 template <int D>
-__device__ __forceinline__ void prefetch_diag(const AttnArgs& a, const Item& w, int row_in_item) {
-  if (row_in_item >= w.nrows) return;
-  const int row = w.q_row0 + row_in_item;
-  if (a.q_seg && a.q_seg[row] != -1) return;
-  const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
+__device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars, int n_items,
+                          volatile int* abort_flag, int t) {
+  uint32_t n = 0;
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n) {
+    const Item w = decode_item(a.items[it]);
+    const int slot = n & 1;
+    if (!mbar_wait(bars + 8 * (kDiagEmpty + slot), ((n >> 1) & 1) ^ 1, abort_flag, a.status))
+      return;
+    for (int rr = t; rr < kItemRows; rr += kDiagThreads) {
+      float sd = -INFINITY;
+      if (rr < w.nrows) {
+        const int row = w.q_row0 + rr;
+        if (!a.q_seg || a.q_seg[row] == -1) {
+          const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
 #pragma unroll
-  for (int c = 0; c < D * 2; c += 128) {
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.q + base + c / 2));
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dk + base + c / 2));
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base + c / 2));
+          for (int c = 0; c < D * 2; c += 128)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base + c / 2));
+          sd = diag_score<D>(a, base);
+        }
+      }
+      sd_buf[slot * kItemRows + rr] = sd;
+    }
+    mbar_arrive(bars + 8 * (kDiagFull + slot));
   }
 }
 
 template <int D>
-__device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, int n_items,
-                             volatile int* abort_flag, int warp, int lane) {
+__device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
+                             const float* sd_buf, int n_items, volatile int* abort_flag, int warp,
+                             int lane) {
   using C = Cfg<D>;
   const int grp = (warp - 2) >> 2;            // query tile A (0) or B (1) of each item
   const int quarter = warp & 3;               // TMEM lane quarter this warp may access
@@ -552,16 +575,22 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, in
   const float sl2 = a.scale_log2;
   uint32_t lt = 0, oi = 0;                    // S_w fills and O_w-ready completions seen
   bool ok = true;
-  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+  uint32_t n = 0;                             // items walked (diagonal-score slot sequence)
+  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++n) {
     const Item w = decode_item(a.items[it]);
-    if (grp == 1 && w.nrows <= C::BM) continue;   // the item has no tile B
-    prefetch_diag<D>(a, w, row_in_item);
+    const int slot = n & 1;
+    if (grp == 1 && w.nrows <= C::BM) {
+      // The item has no tile B; its diagonal-score slot is still released (after it was filled,
+      // so that this release cannot count toward the slot's previous use).
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bars + 8 * (kDiagFull + slot), (n >> 1) & 1, abort_flag, a.status));
+      if (ok) mbar_arrive(bars + 8 * (kDiagEmpty + slot));
+      continue;
+    }
     const bool row_ok = row_in_item < w.nrows;
     const int row = w.q_row0 + (row_ok ? row_in_item : 0);
     const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
     const int seg = row_ok ? (a.q_seg ? (int)a.q_seg[row] : -1) : 0;
-    float sd = -INFINITY;                     // diagonal score of a candidate row
-    if (w.n_kv == 0 && seg == -1) sd = diag_score<D>(a, base);
     float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
     for (int j = 0; j < w.n_kv; ++j, ++lt) {
       const int valid = min(C::BN, w.kv_len - j * C::BN);
@@ -648,9 +677,6 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, in
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bars + 8 * (kPFull + grp));
-      // The diagonal score needs no TMEM: a candidate row computes it while the next S_w (or, for
-      // a one-tile item, O_w) is being produced.
-      if (j == 0 && seg == -1) sd = diag_score<D>(a, base);
     }
     if (!ok) break;
     // The row's own value is fetched while the item's last PV runs.
@@ -661,6 +687,11 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem, in
       for (int c = 0; c < D / 8; ++c)
         vv[c] = seg == -1 ? ld_global_nc_v4(vp + c) : make_uint4(0u, 0u, 0u, 0u);
     }
+    ok = __all_sync(0xffffffffu,
+                    mbar_wait(bars + 8 * (kDiagFull + slot), (n >> 1) & 1, abort_flag, a.status));
+    if (!ok) break;
+    const float sd = sd_buf[slot * kItemRows + row_in_item];   // diagonal score (candidates)
+    mbar_arrive(bars + 8 * (kDiagEmpty + slot));
     if (w.n_kv > 0) {
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bars + 8 * (kOReady + grp), oi & 1, abort_flag, a.status));
@@ -705,6 +736,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (kOFree + i), kSoftmaxThreads / 2);
     }
     mbar_init(bars + 8 * kDrain, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars + 8 * (kDiagFull + i), kDiagThreads);
+      mbar_init(bars + 8 * (kDiagEmpty + i), kSoftmaxThreads);
+    }
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
@@ -729,8 +764,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag, lane == 1);
   } else if (warp == 1) {
     if (lane == 0) mma_role<D>(a, sbase, bars, tmem, n_items, abort_flag);
+  } else if (warp < 10) {
+    softmax_role<D>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG), n_items,
+                    abort_flag, warp, lane);
   } else {
-    softmax_role<D>(a, bars, tmem, n_items, abort_flag, warp, lane);
+    diag_role<D>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), bars, n_items, abort_flag,
+                 threadIdx.x - 320);
   }
 
   tc_fence_before();
