@@ -109,6 +109,12 @@ enum : int {
 constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kDiagThreads = 64;
+// Key pairs (of every 16 in a 32-key chunk) whose 2^x is evaluated on the FMA pipe; even.
+#ifndef JCA_EMU_PAIRS
+#define JCA_EMU_PAIRS 0
+#endif
+constexpr int kEmuPairs = JCA_EMU_PAIRS;
+static_assert(kEmuPairs % 2 == 0 && kEmuPairs >= 0 && kEmuPairs <= 16, "emulated pairs per chunk");
 
 struct Item {
   int q_row0, h, nrows, kv_lo, kv_len, holes, n_kv;
@@ -646,33 +652,43 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
 
       // Pass 2: p = 2^(scale_log2 * s - m), written back over S_w as bf16 pairs (TMEM column k
       // holds keys 2k, 2k+1) 32 keys at a time; chunks past the last real key are never read
-      // by the trimmed PV and are skipped.
-      float sum0 = 0.f, sum1 = 0.f, sum2 = 0.f, sum3 = 0.f;
+      // by the trimmed PV and are skipped. Arithmetic runs on key pairs (packed fp32 FMA/add), and
+      // kEmuPairs of every 16 pairs take 2^x on the FMA pipe instead of the special-function
+      // unit, whose 16 results per clock would otherwise set the pace of the softmax.
+      const float2 sl2v = make_float2(sl2, sl2), negv = make_float2(neg_m, neg_m);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         if (c >= nchunks) break;
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i]), sl2, neg_m));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i + 1]), sl2, neg_m));
-          const float p2 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i + 2]), sl2, neg_m));
-          const float p3 = fast_exp2(fmaf(__uint_as_float(x[32 * c + i + 3]), sl2, neg_m));
-          sum0 += p0;
-          sum1 += p1;
-          sum2 += p2;
-          sum3 += p3;
-          pk[i / 2] = pack_bf16x2(p0, p1);
-          pk[i / 2 + 1] = pack_bf16x2(p2, p3);
+        for (int i = 0; i < 16; ++i) {
+          const float2 xs = __ffma2_rn(make_float2(__uint_as_float(x[32 * c + 2 * i]),
+                                                   __uint_as_float(x[32 * c + 2 * i + 1])),
+                                       sl2v, negv);
+          float2 p;
+          if ((i & 7) >= 8 - kEmuPairs / 2) {
+            p = exp2_fma2(xs);
+          } else {
+            p.x = fast_exp2(xs.x);
+            p.y = fast_exp2(xs.y);
+          }
+          if ((i & 3) == 0) acc0 = __fadd2_rn(acc0, p);
+          if ((i & 3) == 1) acc1 = __fadd2_rn(acc1, p);
+          if ((i & 3) == 2) acc2 = __fadd2_rn(acc2, p);
+          if ((i & 3) == 3) acc3 = __fadd2_rn(acc3, p);
+          pk[i] = pack_bf16x2(p.x, p.y);
         }
         tmem_st_x16(t_s + 16 * c, pk);
       }
+      const float2 acc01 = __fadd2_rn(acc0, acc1), acc23 = __fadd2_rn(acc2, acc3);
+      const float tile_sum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
       // O_w is stable here: its last PV was issued before the QK that filled S_w, and that
       // QK's commit fired only after every earlier MMA completed. TMEM loads/stores are
       // warp-collective: the warp rescales when any of its rows must.
       const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
       if (__any_sync(0xffffffffu, rescale && j >= 1)) rescale_o_row<D>(t_o, alpha);
-      l = l * alpha + ((sum0 + sum1) + (sum2 + sum3));
+      l = l * alpha + tile_sum;
       m = m_use;
       tmem_wait_st();
       tc_fence_before();
