@@ -72,11 +72,30 @@ struct Cfg {
   static constexpr int KSTEPS_QK = D / 16;
   static constexpr int KSTEPS_PER_BLK = SW / 32;
   static constexpr int KSTEPS_PV = BN / 16;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + 2 * TILE_BYTES;
-  static constexpr int OFF_V = OFF_K + 2 * TILE_BYTES;
-  static constexpr int OFF_BAR = OFF_V + 2 * TILE_BYTES;
-  static constexpr int NUM_BARS = 26;
+  // Ring depths: query-tile buffers per group and K / V stages. Small heads make short items
+  // (a few key tiles) whose loads must be issued an item ahead to hide HBM latency; their tiles are
+  // small, so the rings are deeper there. D = 128 fills shared memory with one Q buffer per group.
+  static constexpr int QS = D >= 128 ? 1 : (D == 64 ? 2 : 4);
+  static constexpr int KVS = D >= 128 ? 2 : (D == 64 ? 3 : 4);
+  static constexpr int OFF_Q = 0;                          // [group][QS] tiles
+  static constexpr int OFF_K = OFF_Q + 2 * QS * TILE_BYTES;
+  static constexpr int OFF_V = OFF_K + KVS * TILE_BYTES;
+  static constexpr int OFF_BAR = OFF_V + KVS * TILE_BYTES;
+  // Barrier slots.
+  static constexpr int B_QFULL = 0;                        // [group][QS]
+  static constexpr int B_QEMPTY = B_QFULL + 2 * QS;        // [group][QS]
+  static constexpr int B_KFULL = B_QEMPTY + 2 * QS;        // [KVS]
+  static constexpr int B_KEMPTY = B_KFULL + KVS;
+  static constexpr int B_VFULL = B_KEMPTY + KVS;
+  static constexpr int B_VEMPTY = B_VFULL + KVS;
+  static constexpr int B_SFULL = B_VEMPTY + KVS;           // [group]: S_w written by a QK
+  static constexpr int B_PFULL = B_SFULL + 2;              // [group]: P_w written, S_w read
+  static constexpr int B_OREADY = B_PFULL + 2;             // [group]: item's last PV complete
+  static constexpr int B_OFREE = B_OREADY + 2;             // [group]: O_w read by the group
+  static constexpr int B_DRAIN = B_OFREE + 2;
+  static constexpr int B_DIAGFULL = B_DRAIN + 1;           // [slot]: scores written
+  static constexpr int B_DIAGEMPTY = B_DIAGFULL + 2;       // [slot]: scores taken
+  static constexpr int NUM_BARS = B_DIAGEMPTY + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // Diagonal scores of the candidate rows: two item slots of kItemRows floats.
   static constexpr int OFF_DIAG = OFF_MISC + 16;
@@ -88,19 +107,6 @@ struct Cfg {
   static constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 384,
                             TMEM_COLS = 512;
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
-};
-
-// Barrier slots.
-enum : int {
-  kQFull = 0, kQEmpty = 2,   // per query tile (A, B)
-  kKFull = 4, kKEmpty = 6, kVFull = 8, kVEmpty = 10,   // per K / V stage
-  kSFull = 12,   // per softmax group: S_w written by a QK
-  kPFull = 14,   // per softmax group: P_w written (and S_w read) by the group
-  kOReady = 16,  // per group: the item's last PV into O_w complete
-  kOFree = 18,   // per group: O_w of the item read by the group
-  kDrain = 20,
-  kDiagFull = 22,   // per slot: an item's diagonal scores written by the diagonal warps
-  kDiagEmpty = 24   // per slot: the item's scores taken by every softmax thread
 };
 
 // Warps: 0 TMA producers, 1 TMEM allocator + MMA issuer, 2..9 softmax/epilogue, 10..11 diagonal
@@ -135,17 +141,17 @@ __device__ __forceinline__ Item decode_item(int4 v) {
 // ------------------------------------------------------------------------------------------
 // Producer
 // ------------------------------------------------------------------------------------------
-// Two producer threads in warp 0 walk the same item sequence: lane 0 loads the Q tiles (one buffer
-// per query tile, refilled once the item's last QK of that tile completed) and the K tiles (slots
-// freed by QK completions), lane 1 loads the V tiles (slots freed by PV completions), so a slow
-// PV never holds back the next K.
+// Two producer threads in warp 0 walk the same item sequence: lane 0 loads the Q tiles (a ring of
+// QS buffers per query tile, each refilled once the last QK of the item that used it completed)
+// and the K tiles (stages freed by QK completions), lane 1 loads the V tiles (stages freed by PV
+// completions), so a slow PV never holds back the next K.
 template <int D>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV, const AttnArgs& a, uint32_t sbase,
                               uint32_t bars, int n_items, volatile int* abort_flag, bool loads_v) {
   using C = Cfg<D>;
-  uint32_t armed[4] = {0, 0, 0, 0};  // Q A, Q B (or V stage 0, 1) | K stage 0, 1
-  uint32_t g = 0;
+  uint32_t nq[2] = {0, 0};   // Q loads per query tile
+  uint32_t g = 0;            // K (or V) loads
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
@@ -153,30 +159,31 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
     if (!loads_v) {
       const int ntiles = w.nrows > C::BM ? 2 : 1;
       for (int t = 0; ok && t < ntiles; ++t) {
-        // Load #n of Q buffer t waits for the release of load #n-1 (immediate the first time).
-        ok = mbar_wait(bars + 8 * (kQEmpty + t), (armed[t] & 1) ^ 1, abort_flag, a.status);
+        // Load n of a buffer waits for the release of load n - 1 (immediate the first time).
+        const int slot = t * C::QS + (int)(nq[t] % C::QS);
+        ok = mbar_wait(bars + 8 * (C::B_QEMPTY + slot), ((nq[t] / C::QS) & 1) ^ 1, abort_flag,
+                       a.status);
         if (!ok) break;
-        mbar_arrive_expect_tx(bars + 8 * (kQFull + t), C::TILE_BYTES);
-        ++armed[t];
+        mbar_arrive_expect_tx(bars + 8 * (C::B_QFULL + slot), C::TILE_BYTES);
+        ++nq[t];
 #pragma unroll
         for (int c = 0; c < C::NBLK; ++c)
-          tma_load_3d(sbase + C::OFF_Q + t * C::TILE_BYTES + c * C::BLK_BYTES, tmQ,
-                      bars + 8 * (kQFull + t), c * C::BOX_X, w.h, w.q_row0 + t * C::BM);
+          tma_load_3d(sbase + C::OFF_Q + slot * C::TILE_BYTES + c * C::BLK_BYTES, tmQ,
+                      bars + 8 * (C::B_QFULL + slot), c * C::BOX_X, w.h, w.q_row0 + t * C::BM);
       }
       if (!ok) break;
     }
+    const int empty = loads_v ? C::B_VEMPTY : C::B_KEMPTY;
+    const int full = loads_v ? C::B_VFULL : C::B_KFULL;
+    const CUtensorMap* map = loads_v ? tmV : tmK;
+    const int off = loads_v ? C::OFF_V : C::OFF_K;
     for (int j = 0; j < w.n_kv; ++j, ++g) {
-      const int s = g & 1;
-      const uint32_t ph = (g >> 1) & 1;
+      const int s = (int)(g % C::KVS);
+      const uint32_t ph = (g / C::KVS) & 1;
       const int row = w.kv_lo + j * C::BN;
-      const int empty = loads_v ? kVEmpty : kKEmpty;
-      const int full = loads_v ? kVFull : kKFull;
-      const CUtensorMap* map = loads_v ? tmV : tmK;
-      const int off = loads_v ? C::OFF_V : C::OFF_K;
       ok = mbar_wait(bars + 8 * (empty + s), ph ^ 1, abort_flag, a.status);
       if (!ok) break;
       mbar_arrive_expect_tx(bars + 8 * (full + s), C::TILE_BYTES);
-      ++armed[loads_v ? s : 2 + s];
 #pragma unroll
       for (int c = 0; c < C::NBLK; ++c)
         tma_load_3d(sbase + off + s * C::TILE_BYTES + c * C::BLK_BYTES, map,
@@ -184,11 +191,17 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
     }
   }
   if (!ok) {
-    // Aborting: let every copy this thread started land before the CTA exits.
-    const int slot[4] = {loads_v ? kVFull : kQFull, loads_v ? kVFull + 1 : kQFull + 1, kKFull,
-                         kKFull + 1};
-    for (int i = 0; i < 4; ++i)
-      if (armed[i]) mbar_wait_drain(bars + 8 * slot[i], (armed[i] - 1) & 1);
+    // Aborting: let every copy this thread started land before the CTA exits. Load n of a slot
+    // completes phase n of its full barrier; the last one issued is the newest.
+    if (!loads_v) {
+      for (int t = 0; t < 2; ++t)
+        for (uint32_t n = nq[t] > (uint32_t)C::QS ? nq[t] - C::QS : 0; n < nq[t]; ++n)
+          mbar_wait_drain(bars + 8 * (C::B_QFULL + t * C::QS + (int)(n % C::QS)),
+                          (n / C::QS) & 1);
+    }
+    const int full = loads_v ? C::B_VFULL : C::B_KFULL;
+    for (uint32_t n = g > (uint32_t)C::KVS ? g - C::KVS : 0; n < g; ++n)
+      mbar_wait_drain(bars + 8 * (full + (int)(n % C::KVS)), (n / C::KVS) & 1);
   }
 }
 
@@ -199,10 +212,10 @@ struct MmaState {
   uint32_t p_seen[2];   // P-full completions consumed, per softmax group
   uint32_t o_items[2];  // items whose O_w was written, per group (O-free completions expected)
   uint32_t q_seen[2];   // Q-full completions consumed, per query tile
-  // Operand descriptors of the Q buffers and K / V stages (start address of the first k-step); a
-  // k-step adds a compile-time offset to the low bits (shared addresses stay below 256 KB, so the
-  // 14-bit field never carries). Scalars, selected by index, so they stay in registers.
-  uint64_t q0, q1, k0, k1, v0, v1;
+  // Operand descriptors of Q buffer 0 and of K / V stage 0 (start address of the first k-step);
+  // a buffer, stage or k-step adds an offset to the low bits (shared addresses stay below 256 KB,
+  // so the 14-bit field never carries).
+  uint64_t q, k, v;
 };
 
 // Tensor-core issue is paced by execution (one 128x128x16 MMA takes about 64 cycles), so the issue
@@ -246,17 +259,18 @@ __device__ __forceinline__ bool issue_pv(int grp, uint32_t gg, int jj, int valid
                                          uint32_t bars, uint32_t tmem, const AttnArgs& a,
                                          volatile int* abort_flag) {
   using C = Cfg<D>;
-  const int s = gg & 1;
-  if (!mbar_wait(bars + 8 * (kVFull + s), (gg >> 1) & 1, abort_flag, a.status)) return false;
-  if (!mbar_wait(bars + 8 * (kPFull + grp), st.p_seen[grp] & 1, abort_flag, a.status))
+  const int s = (int)(gg % C::KVS);
+  if (!mbar_wait(bars + 8 * (C::B_VFULL + s), (gg / C::KVS) & 1, abort_flag, a.status))
+    return false;
+  if (!mbar_wait(bars + 8 * (C::B_PFULL + grp), st.p_seen[grp] & 1, abort_flag, a.status))
     return false;
   ++st.p_seen[grp];
   if (jj == 0 && st.o_items[grp] > 0 &&
-      !mbar_wait(bars + 8 * (kOFree + grp), (st.o_items[grp] - 1) & 1, abort_flag, a.status))
+      !mbar_wait(bars + 8 * (C::B_OFREE + grp), (st.o_items[grp] - 1) & 1, abort_flag, a.status))
     return false;
   tc_fence_after();
   mma_pv<D>(tmem + (grp ? C::TMEM_O1 : C::TMEM_O0), tmem + (grp ? C::TMEM_S1 : C::TMEM_S0),
-            s ? st.v1 : st.v0, (valid + 15) >> 4, jj == 0);
+            st.v + (uint64_t)((s * C::TILE_BYTES) >> 4), (valid + 15) >> 4, jj == 0);
   return true;
 }
 
@@ -271,63 +285,67 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
   st.p_seen[0] = st.p_seen[1] = 0;
   st.o_items[0] = st.o_items[1] = 0;
   st.q_seen[0] = st.q_seen[1] = 0;
-  st.q0 = smem_desc(sbase + C::OFF_Q, 16, 8 * C::SW, C::LAYOUT);
-  st.q1 = smem_desc(sbase + C::OFF_Q + C::TILE_BYTES, 16, 8 * C::SW, C::LAYOUT);
-  st.k0 = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
-  st.k1 = smem_desc(sbase + C::OFF_K + C::TILE_BYTES, 16, 8 * C::SW, C::LAYOUT);
-  st.v0 = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
-  st.v1 = smem_desc(sbase + C::OFF_V + C::TILE_BYTES, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
+  st.q = smem_desc(sbase + C::OFF_Q, 16, 8 * C::SW, C::LAYOUT);
+  st.k = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
+  st.v = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
   uint32_t g = 0;
   bool ok = true;
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
     if (w.n_kv == 0) continue;
     const bool has_b = w.nrows > C::BM;
-    ok = mbar_wait(bars + 8 * kQFull, st.q_seen[0] & 1, abort_flag, a.status);
+    // This item's Q buffers (one per query tile) in the per-group rings.
+    const int qslot_a = (int)(st.q_seen[0] % C::QS);
+    const int qslot_b = C::QS + (int)(st.q_seen[1] % C::QS);
+    const uint64_t qa = st.q + (uint64_t)((qslot_a * C::TILE_BYTES) >> 4);
+    const uint64_t qb = st.q + (uint64_t)((qslot_b * C::TILE_BYTES) >> 4);
+    ok = mbar_wait(bars + 8 * (C::B_QFULL + qslot_a), (st.q_seen[0] / C::QS) & 1, abort_flag,
+                   a.status);
     if (!ok) break;
     ++st.q_seen[0];
     tc_fence_after();
     int prev_valid = 0;
     for (int j = 0; j < w.n_kv; ++j, ++g) {
-      const int s = g & 1;
-      const uint32_t ph = (g >> 1) & 1;
+      const int s = (int)(g % C::KVS);
+      const uint32_t ph = (g / C::KVS) & 1;
       const bool last = j == w.n_kv - 1;
       const int valid = min(C::BN, w.kv_len - j * C::BN);
       const uint32_t idesc_qk =
           valid == C::BN ? kIdescQKFull
                          : (kIdescQK0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17));
-      const uint64_t kb = s ? st.k1 : st.k0;
-      ok = mbar_wait(bars + 8 * (kKFull + s), ph, abort_flag, a.status);
+      const uint64_t kb = st.k + (uint64_t)((s * C::TILE_BYTES) >> 4);
+      ok = mbar_wait(bars + 8 * (C::B_KFULL + s), ph, abort_flag, a.status);
       if (!ok) break;
       tc_fence_after();
       // QK_A(j)
-      mma_qk<D>(tmem + C::TMEM_S0, st.q0, kb, idesc_qk);
-      tc_commit(bars + 8 * kSFull);
-      if (last) tc_commit(bars + 8 * kQEmpty);
+      mma_qk<D>(tmem + C::TMEM_S0, qa, kb, idesc_qk);
+      tc_commit(bars + 8 * C::B_SFULL);
+      if (last) tc_commit(bars + 8 * (C::B_QEMPTY + qslot_a));
       if (has_b) {
         // PV_B(j-1): the V stage of tile j-1 is released after both groups' PVs.
         if (j > 0) {
           ok = issue_pv<D>(1, g - 1, j - 1, prev_valid, st, bars, tmem, a, abort_flag);
           if (!ok) break;
-          tc_commit(bars + 8 * (kVEmpty + ((g - 1) & 1)));
+          tc_commit(bars + 8 * (C::B_VEMPTY + (int)((g - 1) % C::KVS)));
         }
         // QK_B(j)
         if (j == 0) {
-          ok = mbar_wait(bars + 8 * (kQFull + 1), st.q_seen[1] & 1, abort_flag, a.status);
+          ok = mbar_wait(bars + 8 * (C::B_QFULL + qslot_b), (st.q_seen[1] / C::QS) & 1,
+                         abort_flag, a.status);
           if (!ok) break;
           ++st.q_seen[1];
           tc_fence_after();
         }
-        mma_qk<D>(tmem + C::TMEM_S1, st.q1, kb, idesc_qk);
-        tc_commit(bars + 8 * (kSFull + 1));
-        if (last) tc_commit(bars + 8 * (kQEmpty + 1));
+        mma_qk<D>(tmem + C::TMEM_S1, qb, kb, idesc_qk);
+        tc_commit(bars + 8 * (C::B_SFULL + 1));
+        if (last) tc_commit(bars + 8 * (C::B_QEMPTY + qslot_b));
       }
-      tc_commit(bars + 8 * (kKEmpty + s));
+      tc_commit(bars + 8 * (C::B_KEMPTY + s));
       // PV_A(j)
       ok = issue_pv<D>(0, g, j, valid, st, bars, tmem, a, abort_flag);
       if (!ok) break;
-      if (!has_b) tc_commit(bars + 8 * (kVEmpty + s));
-      if (last) tc_commit(bars + 8 * kOReady);
+      if (!has_b) tc_commit(bars + 8 * (C::B_VEMPTY + s));
+      if (last) tc_commit(bars + 8 * C::B_OREADY);
       prev_valid = valid;
     }
     if (!ok) break;
@@ -336,15 +354,15 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
       // PV_B of the item's last key tile.
       ok = issue_pv<D>(1, g - 1, w.n_kv - 1, prev_valid, st, bars, tmem, a, abort_flag);
       if (!ok) break;
-      tc_commit(bars + 8 * (kVEmpty + ((g - 1) & 1)));
-      tc_commit(bars + 8 * (kOReady + 1));
+      tc_commit(bars + 8 * (C::B_VEMPTY + (int)((g - 1) % C::KVS)));
+      tc_commit(bars + 8 * (C::B_OREADY + 1));
       ++st.o_items[1];
     }
   }
   if (!ok) {
     // Aborting: wait until every MMA this thread issued has completed.
-    tc_commit(bars + 8 * kDrain);
-    mbar_wait_drain(bars + 8 * kDrain, 0);
+    tc_commit(bars + 8 * C::B_DRAIN);
+    mbar_wait_drain(bars + 8 * C::B_DRAIN, 0);
   }
 }
 
@@ -542,11 +560,12 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int s
 template <int D>
 __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars, int n_items,
                           volatile int* abort_flag, int t) {
+  using C = Cfg<D>;
   uint32_t n = 0;
   for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n) {
     const Item w = decode_item(a.items[it]);
     const int slot = n & 1;
-    if (!mbar_wait(bars + 8 * (kDiagEmpty + slot), ((n >> 1) & 1) ^ 1, abort_flag, a.status))
+    if (!mbar_wait(bars + 8 * (C::B_DIAGEMPTY + slot), ((n >> 1) & 1) ^ 1, abort_flag, a.status))
       return;
     for (int rr = t; rr < kItemRows; rr += kDiagThreads) {
       float sd = -INFINITY;
@@ -562,7 +581,7 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars, int n
       }
       sd_buf[slot * kItemRows + rr] = sd;
     }
-    mbar_arrive(bars + 8 * (kDiagFull + slot));
+    mbar_arrive(bars + 8 * (C::B_DIAGFULL + slot));
   }
 }
 
@@ -589,8 +608,8 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       // The item has no tile B; its diagonal-score slot is still released (after it was filled,
       // so that this release cannot count toward the slot's previous use).
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bars + 8 * (kDiagFull + slot), (n >> 1) & 1, abort_flag, a.status));
-      if (ok) mbar_arrive(bars + 8 * (kDiagEmpty + slot));
+                      mbar_wait(bars + 8 * (C::B_DIAGFULL + slot), (n >> 1) & 1, abort_flag, a.status));
+      if (ok) mbar_arrive(bars + 8 * (C::B_DIAGEMPTY + slot));
       continue;
     }
     const bool row_ok = row_in_item < w.nrows;
@@ -605,7 +624,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       // column by column; interior tiles take the unmasked path.
       const bool edge = valid < C::BN || w.holes;
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bars + 8 * (kSFull + grp), lt & 1, abort_flag, a.status));
+                      mbar_wait(bars + 8 * (C::B_SFULL + grp), lt & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
 
@@ -692,7 +711,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       m = m_use;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bars + 8 * (kPFull + grp));
+      mbar_arrive(bars + 8 * (C::B_PFULL + grp));
     }
     if (!ok) break;
     // The row's own value is fetched while the item's last PV runs.
@@ -704,18 +723,18 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
         vv[c] = seg == -1 ? ld_global_nc_v4(vp + c) : make_uint4(0u, 0u, 0u, 0u);
     }
     ok = __all_sync(0xffffffffu,
-                    mbar_wait(bars + 8 * (kDiagFull + slot), (n >> 1) & 1, abort_flag, a.status));
+                    mbar_wait(bars + 8 * (C::B_DIAGFULL + slot), (n >> 1) & 1, abort_flag, a.status));
     if (!ok) break;
     const float sd = sd_buf[slot * kItemRows + row_in_item];   // diagonal score (candidates)
-    mbar_arrive(bars + 8 * (kDiagEmpty + slot));
+    mbar_arrive(bars + 8 * (C::B_DIAGEMPTY + slot));
     if (w.n_kv > 0) {
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(bars + 8 * (kOReady + grp), oi & 1, abort_flag, a.status));
+                      mbar_wait(bars + 8 * (C::B_OREADY + grp), oi & 1, abort_flag, a.status));
       if (!ok) break;
       tc_fence_after();
       ++oi;
     }
-    finish_row<D>(a, row_ok, seg, base, t_o, w.n_kv > 0, m, l, sd, vv, bars + 8 * (kOFree + grp));
+    finish_row<D>(a, row_ok, seg, base, t_o, w.n_kv > 0, m, l, sd, vv, bars + 8 * (C::B_OFREE + grp));
   }
 }
 
@@ -739,23 +758,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bars + 8 * (kQFull + i), 1);
-      mbar_init(bars + 8 * (kQEmpty + i), 1);
-      mbar_init(bars + 8 * (kKFull + i), 1);
-      mbar_init(bars + 8 * (kKEmpty + i), 1);
-      mbar_init(bars + 8 * (kVFull + i), 1);
-      mbar_init(bars + 8 * (kVEmpty + i), 1);
-      mbar_init(bars + 8 * (kSFull + i), 1);
-      mbar_init(bars + 8 * (kPFull + i), kSoftmaxThreads / 2);
-      mbar_init(bars + 8 * (kOReady + i), 1);
-      mbar_init(bars + 8 * (kOFree + i), kSoftmaxThreads / 2);
+    for (int i = 0; i < 2 * C::QS; ++i) {
+      mbar_init(bars + 8 * (C::B_QFULL + i), 1);
+      mbar_init(bars + 8 * (C::B_QEMPTY + i), 1);
     }
-    mbar_init(bars + 8 * kDrain, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bars + 8 * (kDiagFull + i), kDiagThreads);
-      mbar_init(bars + 8 * (kDiagEmpty + i), kSoftmaxThreads);
+    for (int i = 0; i < C::KVS; ++i) {
+      mbar_init(bars + 8 * (C::B_KFULL + i), 1);
+      mbar_init(bars + 8 * (C::B_KEMPTY + i), 1);
+      mbar_init(bars + 8 * (C::B_VFULL + i), 1);
+      mbar_init(bars + 8 * (C::B_VEMPTY + i), 1);
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bars + 8 * (C::B_SFULL + i), 1);
+      mbar_init(bars + 8 * (C::B_PFULL + i), kSoftmaxThreads / 2);
+      mbar_init(bars + 8 * (C::B_OREADY + i), 1);
+      mbar_init(bars + 8 * (C::B_OFREE + i), kSoftmaxThreads / 2);
+      mbar_init(bars + 8 * (C::B_DIAGFULL + i), kDiagThreads);
+      mbar_init(bars + 8 * (C::B_DIAGEMPTY + i), kSoftmaxThreads);
+    }
+    mbar_init(bars + 8 * C::B_DRAIN, 1);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
