@@ -274,6 +274,18 @@ __device__ __forceinline__ bool issue_pv(int grp, uint32_t gg, int jj, int valid
   return true;
 }
 
+// The issue order is one stream over the key tiles of all the CTA's items: per key tile t,
+//   QK_A(t), PV_B(t-1), QK_B(t), PV_A(t),
+// where t-1 may be the last tile of the previous item. The next item's first QK therefore starts
+// while the previous item's tile-B softmax is still running, and the two groups stay a half tile
+// apart across item boundaries instead of starting every item in step.
+struct PendingPV {
+  uint32_t gg;   // global key tile (V stage)
+  int jj;        // key tile within its item (0: overwrite O)
+  int valid;     // real keys in the tile; 0 = nothing pending
+  bool last;     // the item's last key tile: its completion makes O ready
+};
+
 template <int D>
 __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          int n_items, volatile int* abort_flag) {
@@ -289,7 +301,20 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
   st.k = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
   st.v = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
   uint32_t g = 0;
+  PendingPV pend{0, 0, 0, false};
   bool ok = true;
+  // PV_B of the pending tile, its V-stage release and, for an item's last tile, O_B ready.
+  auto flush_b = [&]() -> bool {
+    if (pend.valid == 0) return true;
+    if (!issue_pv<D>(1, pend.gg, pend.jj, pend.valid, st, bars, tmem, a, abort_flag)) return false;
+    tc_commit(bars + 8 * (C::B_VEMPTY + (int)(pend.gg % C::KVS)));
+    if (pend.last) {
+      tc_commit(bars + 8 * (C::B_OREADY + 1));
+      ++st.o_items[1];
+    }
+    pend.valid = 0;
+    return true;
+  };
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const Item w = decode_item(a.items[it]);
     if (w.n_kv == 0) continue;
@@ -304,7 +329,6 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     if (!ok) break;
     ++st.q_seen[0];
     tc_fence_after();
-    int prev_valid = 0;
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = (int)(g % C::KVS);
       const uint32_t ph = (g / C::KVS) & 1;
@@ -317,18 +341,15 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
       ok = mbar_wait(bars + 8 * (C::B_KFULL + s), ph, abort_flag, a.status);
       if (!ok) break;
       tc_fence_after();
-      // QK_A(j)
+      // QK_A(t)
       mma_qk<D>(tmem + C::TMEM_S0, qa, kb, idesc_qk);
       tc_commit(bars + 8 * C::B_SFULL);
       if (last) tc_commit(bars + 8 * (C::B_QEMPTY + qslot_a));
+      // PV_B(t-1), possibly of the previous item
+      ok = flush_b();
+      if (!ok) break;
       if (has_b) {
-        // PV_B(j-1): the V stage of tile j-1 is released after both groups' PVs.
-        if (j > 0) {
-          ok = issue_pv<D>(1, g - 1, j - 1, prev_valid, st, bars, tmem, a, abort_flag);
-          if (!ok) break;
-          tc_commit(bars + 8 * (C::B_VEMPTY + (int)((g - 1) % C::KVS)));
-        }
-        // QK_B(j)
+        // QK_B(t)
         if (j == 0) {
           ok = mbar_wait(bars + 8 * (C::B_QFULL + qslot_b), (st.q_seen[1] / C::QS) & 1,
                          abort_flag, a.status);
@@ -341,24 +362,18 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
         if (last) tc_commit(bars + 8 * (C::B_QEMPTY + qslot_b));
       }
       tc_commit(bars + 8 * (C::B_KEMPTY + s));
-      // PV_A(j)
+      // PV_A(t); the V stage is released here when the item has no tile B, else after PV_B(t).
       ok = issue_pv<D>(0, g, j, valid, st, bars, tmem, a, abort_flag);
       if (!ok) break;
       if (!has_b) tc_commit(bars + 8 * (C::B_VEMPTY + s));
-      if (last) tc_commit(bars + 8 * C::B_OREADY);
-      prev_valid = valid;
-    }
-    if (!ok) break;
-    ++st.o_items[0];
-    if (has_b) {
-      // PV_B of the item's last key tile.
-      ok = issue_pv<D>(1, g - 1, w.n_kv - 1, prev_valid, st, bars, tmem, a, abort_flag);
-      if (!ok) break;
-      tc_commit(bars + 8 * (C::B_VEMPTY + (int)((g - 1) % C::KVS)));
-      tc_commit(bars + 8 * (C::B_OREADY + 1));
-      ++st.o_items[1];
+      if (last) {
+        tc_commit(bars + 8 * C::B_OREADY);
+        ++st.o_items[0];
+      }
+      if (has_b) pend = PendingPV{g, j, valid, last};
     }
   }
+  if (ok) ok = flush_b();
   if (!ok) {
     // Aborting: wait until every MMA this thread issued has completed.
     tc_commit(bars + 8 * C::B_DRAIN);
