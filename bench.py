@@ -241,7 +241,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     out = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
     ws = torch.empty(jca.jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=dev)
     status = jca.new_status(dev)
-    launches_per_step = 5  # offsets, segment IDs, bounds, work queue, attention
+    launches_per_step = 4  # offsets, segment IDs + bounds (one pass), work queue, attention
 
     def step(ev=None):
         jca.jca_offsets_from_lengths(lengths, offsets, status, stream)

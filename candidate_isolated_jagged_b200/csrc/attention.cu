@@ -981,11 +981,11 @@ extern "C" int jagged_cand_attn_plan(const void* offsets, const void* candidate_
   char* ws = static_cast<char*>(workspace);
   int8_t* segp = seg ? const_cast<int8_t*>(seg) : reinterpret_cast<int8_t*>(ws + L.seg);
   int32_t* kv_count = reinterpret_cast<int32_t*>(ws + L.kv_count);
-  if (!seg && launch_segment_ids(offsets, candidate_start, nullptr, 0, B, T, idx_bits, segp,
-                                 status, st) != cudaSuccess)
-    return JCA_ERR_CUDA;
+  // Without a caller's segment IDs, one pass builds them from the candidate starts and reduces
+  // the bounds.
   if (launch_bounds(segp, offsets, B, T, idx_bits, ws + L.hist_lo, ws + L.hist_hi, ws + L.cand_lo,
-                    ws + L.cand_hi, kv_count, 0, status, st) != cudaSuccess)
+                    ws + L.cand_hi, kv_count, 0, status, st, seg ? nullptr : candidate_start,
+                    seg ? nullptr : segp) != cudaSuccess)
     return JCA_ERR_CUDA;
   if (launch_work_queue(offsets, ws + L.hist_lo, ws + L.hist_hi, kv_count, B, T, T, H, idx_bits,
                         reinterpret_cast<int32_t*>(ws + L.items), L.max_items,

@@ -108,71 +108,92 @@ __global__ void segment_ids_kernel(const IdxT* __restrict__ off, const IdxT* __r
 
 // ---------------------------------------------------------------------------------------------
 // Bounds (候选隔离注意力掩码, section 段 ID：掩码的表达方式, bounds_from_segment_ids): one block per
-// user row reduces first/last positions of segment 1 and -1 and counts the segment-1 tokens.
+// user row reduces first/last positions of segment 1 and -1 and counts the segment-1 tokens, with
+// warp reductions and one shared-memory combine. With FUSED, the block also builds the row's
+// segment IDs from its candidate start (all tokens valid) and writes them, so that the plan makes
+// one pass over the rows instead of two.
 // ---------------------------------------------------------------------------------------------
-template <typename IdxT>
-__global__ void bounds_kernel(const int8_t* __restrict__ seg, const IdxT* __restrict__ off,
-                              int64_t B, int64_t T, IdxT* __restrict__ hist_lo,
-                              IdxT* __restrict__ hist_hi, IdxT* __restrict__ cand_lo,
-                              IdxT* __restrict__ cand_hi, int32_t* __restrict__ kv_count,
-                              int history_only, int32_t* status) {
+template <typename IdxT, bool FUSED>
+__global__ void __launch_bounds__(256) bounds_kernel(
+    int8_t* __restrict__ seg, const IdxT* __restrict__ off, const IdxT* __restrict__ cs, int64_t B,
+    int64_t T, IdxT* __restrict__ hist_lo, IdxT* __restrict__ hist_hi, IdxT* __restrict__ cand_lo,
+    IdxT* __restrict__ cand_hi, int32_t* __restrict__ kv_count, int history_only,
+    int32_t* status) {
   if (*status != 0) return;
-  __shared__ long long s_hmin, s_hmax, s_cmin, s_cmax;
-  __shared__ int s_count, s_bad;
+  __shared__ int s_red[8][6];   // per warp: hmin, hmax, cmin, cmax, count, bad
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int64_t b = blockIdx.x; b < B; b += gridDim.x) {
     const long long s = (long long)off[b], e = (long long)off[b + 1];
     if (!row_ok(s, e, b, B, T)) {
       if (threadIdx.x == 0) set_status(status, JCA_STATUS_BAD_OFFSETS);
       continue;
     }
-    if (threadIdx.x == 0) {
-      s_hmin = LLONG_MAX;
-      s_hmax = -1;
-      s_cmin = LLONG_MAX;
-      s_cmax = -1;
-      s_count = 0;
-      s_bad = 0;
+    const int L = (int)(e - s);   // rows < 2^31 (checked on the host)
+    int c = L;
+    if (FUSED) {
+      const long long cb = (long long)cs[b];
+      if (cb < 0 || cb > L) {
+        if (threadIdx.x == 0) set_status(status, JCA_STATUS_BAD_CAND_START);
+        continue;
+      }
+      c = (int)cb;
     }
-    __syncthreads();
-    long long hmin = LLONG_MAX, hmax = -1, cmin = LLONG_MAX, cmax = -1;
-    int count = 0, bad = 0;
-    for (long long i = threadIdx.x; i < e - s; i += blockDim.x) {
-      const int x = seg[s + i];
+    int hmin = INT_MAX, hmax = -1, cmin = INT_MAX, cmax = -1, count = 0, bad = 0;
+    for (int i = threadIdx.x; i < L; i += blockDim.x) {
+      int x;
+      if (FUSED) {
+        x = i >= c ? -1 : 1;
+        seg[s + i] = (int8_t)x;
+      } else {
+        x = seg[s + i];
+      }
       if (x == 1) {
         hmin = min(hmin, i);
         hmax = max(hmax, i);
         ++count;
       } else if (x == -1) {
-        if (history_only) bad = 1;
+        bad |= history_only;
         cmin = min(cmin, i);
         cmax = max(cmax, i);
       } else if (x != 0) {
         bad = 1;
       }
     }
-    if (hmax >= 0) {
-      atomicMin(&s_hmin, hmin);
-      atomicMax(&s_hmax, hmax);
+    hmin = __reduce_min_sync(0xffffffffu, hmin);
+    hmax = __reduce_max_sync(0xffffffffu, hmax);
+    cmin = __reduce_min_sync(0xffffffffu, cmin);
+    cmax = __reduce_max_sync(0xffffffffu, cmax);
+    count = __reduce_add_sync(0xffffffffu, count);
+    bad = __reduce_or_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      s_red[wid][0] = hmin;
+      s_red[wid][1] = hmax;
+      s_red[wid][2] = cmin;
+      s_red[wid][3] = cmax;
+      s_red[wid][4] = count;
+      s_red[wid][5] = bad;
     }
-    if (cmax >= 0) {
-      atomicMin(&s_cmin, cmin);
-      atomicMax(&s_cmax, cmax);
-    }
-    if (count) atomicAdd(&s_count, count);
-    if (bad) s_bad = 1;
     __syncthreads();
     if (threadIdx.x == 0) {
-      if (s_bad) {
+      for (int w = 1; w < nw; ++w) {
+        hmin = min(hmin, s_red[w][0]);
+        hmax = max(hmax, s_red[w][1]);
+        cmin = min(cmin, s_red[w][2]);
+        cmax = max(cmax, s_red[w][3]);
+        count += s_red[w][4];
+        bad |= s_red[w][5];
+      }
+      if (bad) {
         set_status(status, JCA_STATUS_BAD_SEG_VALUE);
-      } else if (s_hmax >= 0 && s_cmax >= 0 && s_hmax > s_cmin) {
+      } else if (hmax >= 0 && cmax >= 0 && hmax > cmin) {
         set_status(status, JCA_STATUS_BAD_SEG_LAYOUT);
       }
-      const bool has_h = s_hmax >= 0, has_c = s_cmax >= 0;
-      hist_lo[b] = (IdxT)(has_h ? s + s_hmin : s);
-      hist_hi[b] = (IdxT)(has_h ? s + s_hmax + 1 : s);
-      if (cand_lo) cand_lo[b] = (IdxT)(has_c ? s + s_cmin : e);
-      if (cand_hi) cand_hi[b] = (IdxT)(has_c ? s + s_cmax + 1 : e);
-      if (kv_count) kv_count[b] = s_count;
+      const bool has_h = hmax >= 0, has_c = cmax >= 0;
+      hist_lo[b] = (IdxT)(has_h ? s + hmin : s);
+      hist_hi[b] = (IdxT)(has_h ? s + hmax + 1 : s);
+      if (cand_lo) cand_lo[b] = (IdxT)(has_c ? s + cmin : e);
+      if (cand_hi) cand_hi[b] = (IdxT)(has_c ? s + cmax + 1 : e);
+      if (kv_count) kv_count[b] = count;
     }
     __syncthreads();
   }
@@ -256,22 +277,26 @@ __global__ void __launch_bounds__(1024) work_queue_kernel(
     }
     return;
   }
-  for (int64_t b = tid; b < B; b += blockDim.x) {
+  // Pass 2, one warp per user: lane 0 claims the user's run of nq * H slots, the lanes write it.
+  const int nwarps = blockDim.x >> 5;
+  for (int64_t b = wid; b < B; b += nwarps) {
     const long long s = (long long)qoff[b], e = (long long)qoff[b + 1];
     const long long lo = (long long)kvlo[b], hi = (long long)kvhi[b];
     const long long nq = (e - s + kItemRows - 1) / kItemRows;
     if (nq == 0) continue;
     const long long nkv = (hi - lo + kTileN - 1) / kTileN;
     const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
-    const unsigned long long pos = atomicAdd(&s_cursor[key], (unsigned long long)(nq * H));
+    unsigned long long pos = 0;
+    if (lane == 0) pos = atomicAdd(&s_cursor[key], (unsigned long long)(nq * H));
+    pos = __shfl_sync(0xffffffffu, pos, 0);
     const int holes = (kv_count != nullptr && (long long)kv_count[b] != hi - lo) ? 1 : 0;
     const int w = (int)(hi - lo) | (holes << 31);
-    for (int h = 0; h < H; ++h) {
-      for (long long t = 0; t < nq; ++t) {
-        const long long row0 = s + t * kItemRows;
-        const int rows = (int)min((long long)kItemRows, e - row0);
-        items[pos + (unsigned long long)h * nq + t] = make_int4((int)row0, (h << 9) | rows, (int)lo, w);
-      }
+    for (long long i = lane; i < nq * H; i += 32) {
+      const int h = (int)(i / nq);
+      const long long t = i - (long long)h * nq;
+      const long long row0 = s + t * kItemRows;
+      const int rows = (int)min((long long)kItemRows, e - row0);
+      items[pos + (unsigned long long)i] = make_int4((int)row0, (h << 9) | rows, (int)lo, w);
     }
   }
   if (tid == 0) *n_items = (int32_t)s_total;
@@ -328,17 +353,28 @@ cudaError_t launch_segment_ids(const void* offsets, const void* cand_start, cons
 cudaError_t launch_bounds(const int8_t* seg, const void* offsets, int64_t B, int64_t T,
                           int idx_bits, void* hist_lo, void* hist_hi, void* cand_lo,
                           void* cand_hi, int32_t* kv_count, int history_only, int32_t* status,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const void* cand_start, int8_t* seg_out) {
   if (B == 0) return cudaSuccess;
   const int grid = grid_for_rows(B);
-  if (idx_bits == 32)
-    bounds_kernel<int32_t><<<grid, 256, 0, stream>>>(
-        seg, (const int32_t*)offsets, B, T, (int32_t*)hist_lo, (int32_t*)hist_hi,
-        (int32_t*)cand_lo, (int32_t*)cand_hi, kv_count, history_only, status);
-  else
-    bounds_kernel<int64_t><<<grid, 256, 0, stream>>>(
-        seg, (const int64_t*)offsets, B, T, (int64_t*)hist_lo, (int64_t*)hist_hi,
-        (int64_t*)cand_lo, (int64_t*)cand_hi, kv_count, history_only, status);
+  if (idx_bits == 32) {
+    if (cand_start)
+      bounds_kernel<int32_t, true><<<grid, 256, 0, stream>>>(
+          seg_out, (const int32_t*)offsets, (const int32_t*)cand_start, B, T, (int32_t*)hist_lo,
+          (int32_t*)hist_hi, (int32_t*)cand_lo, (int32_t*)cand_hi, kv_count, history_only, status);
+    else
+      bounds_kernel<int32_t, false><<<grid, 256, 0, stream>>>(
+          const_cast<int8_t*>(seg), (const int32_t*)offsets, nullptr, B, T, (int32_t*)hist_lo,
+          (int32_t*)hist_hi, (int32_t*)cand_lo, (int32_t*)cand_hi, kv_count, history_only, status);
+  } else {
+    if (cand_start)
+      bounds_kernel<int64_t, true><<<grid, 256, 0, stream>>>(
+          seg_out, (const int64_t*)offsets, (const int64_t*)cand_start, B, T, (int64_t*)hist_lo,
+          (int64_t*)hist_hi, (int64_t*)cand_lo, (int64_t*)cand_hi, kv_count, history_only, status);
+    else
+      bounds_kernel<int64_t, false><<<grid, 256, 0, stream>>>(
+          const_cast<int8_t*>(seg), (const int64_t*)offsets, nullptr, B, T, (int64_t*)hist_lo,
+          (int64_t*)hist_hi, (int64_t*)cand_lo, (int64_t*)cand_hi, kv_count, history_only, status);
+  }
   return cudaGetLastError();
 }
 

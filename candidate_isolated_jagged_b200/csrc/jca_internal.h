@@ -45,11 +45,14 @@ cudaError_t launch_segment_ids(const void* offsets, const void* cand_start, cons
                                int attend_padded_history, int64_t B, int64_t T, int idx_bits,
                                int8_t* seg, int32_t* status, cudaStream_t stream);
 
-// history_only != 0: segment -1 is invalid (a frozen history may hold only 1 and 0).
+// history_only != 0: segment -1 is invalid (a frozen history may hold only 1 and 0). With
+// cand_start non-null the segment IDs are built from it (every token valid) into seg_out in the
+// same pass, and seg is not read.
 cudaError_t launch_bounds(const int8_t* seg, const void* offsets, int64_t B, int64_t T,
                           int idx_bits, void* hist_lo, void* hist_hi, void* cand_lo,
                           void* cand_hi, int32_t* kv_count, int history_only, int32_t* status,
-                          cudaStream_t stream);
+                          cudaStream_t stream, const void* cand_start = nullptr,
+                          int8_t* seg_out = nullptr);
 
 cudaError_t launch_work_queue(const void* q_offsets, const void* kv_lo, const void* kv_hi,
                               const int32_t* kv_count, int64_t B, int64_t q_rows,
