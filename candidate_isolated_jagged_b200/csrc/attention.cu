@@ -51,12 +51,16 @@ struct AttnArgs {
   void* out;                // [Tq, H, D] bf16 or fp32
   const int4* items;
   const int32_t* n_items;
+  int32_t* queue;           // [2]: next item to claim, CTAs finished
   int32_t* status;
   int H;
   int out_fp32;
   int out_v8;               // out is 32-byte aligned: rows are written with 32-byte stores
   float scale_log2;         // softmax scale * log2(e)
 };
+
+// Depth of the shared ring through which every role receives the claimed work items.
+constexpr int kRing = 4;
 
 template <int D>
 struct Cfg {
@@ -95,10 +99,13 @@ struct Cfg {
   static constexpr int B_DRAIN = B_OFREE + 2;
   static constexpr int B_DIAGFULL = B_DRAIN + 1;           // [slot]: scores written
   static constexpr int B_DIAGEMPTY = B_DIAGFULL + 2;       // [slot]: scores taken
-  static constexpr int NUM_BARS = B_DIAGEMPTY + 2;
+  static constexpr int B_RINGFULL = B_DIAGEMPTY + 2;       // [kRing]: claimed item index written
+  static constexpr int B_RINGEMPTY = B_RINGFULL + kRing;   // [kRing]: index read by every role
+  static constexpr int NUM_BARS = B_RINGEMPTY + kRing;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // Diagonal scores of the candidate rows: two item slots of kItemRows floats.
-  static constexpr int OFF_DIAG = OFF_MISC + 16;
+  static constexpr int OFF_RING = OFF_MISC + 16;           // kRing claimed item indices
+  static constexpr int OFF_DIAG = OFF_RING + 4 * kRing;
   static constexpr int SMEM_USED = OFF_DIAG + 2 * kItemRows * 4;
   static constexpr int SMEM_RAW = SMEM_USED + 1024;                // slack for 1 KB alignment
   // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
@@ -115,6 +122,8 @@ struct Cfg {
 constexpr int kThreads = 384;
 constexpr int kSoftmaxThreads = 256;
 constexpr int kDiagThreads = 64;
+// Readers of the item ring: V producer lane, MMA thread, softmax and diagonal threads.
+constexpr int kRingReaders = 1 + 1 + kSoftmaxThreads + kDiagThreads;
 // Key pairs (of every 16 in a 32-key chunk) whose 2^x is evaluated on the FMA pipe; even.
 #ifndef JCA_EMU_PAIRS
 #define JCA_EMU_PAIRS 0
@@ -138,6 +147,43 @@ __device__ __forceinline__ Item decode_item(int4 v) {
   return w;
 }
 
+// Work items are claimed at run time from a global counter, so that a CTA that finishes early
+// takes the next item (the queue is sorted by cost, largest first). The claiming thread (producer
+// lane 0) writes each claimed index, or -1 once the queue is exhausted, into a shared ring; every
+// other role reads the same sequence from the ring and releases each slot after reading it.
+struct ItemRing {
+  volatile int* slot;   // kRing shared entries
+  uint32_t full;        // address of full barrier 0 (kRing consecutive barriers)
+  uint32_t empty;       // address of empty barrier 0
+  uint32_t k;           // entries taken so far
+};
+
+__device__ __forceinline__ int ring_claim(ItemRing& r, int32_t* head, int n_items,
+                                          volatile int* abort_flag, int32_t* status, bool& ok) {
+  const int s = (int)(r.k % kRing);
+  ok = mbar_wait(r.empty + 8 * s, ((r.k / kRing) & 1) ^ 1, abort_flag, status);
+  if (!ok) return -1;
+  int v = atomicAdd(head, 1);
+  if (v >= n_items) v = -1;
+  r.slot[s] = v;
+  mbar_arrive(r.full + 8 * s);
+  ++r.k;
+  return v;
+}
+
+// Every thread of a consuming role calls this (warps stay converged: `ok` is made warp-uniform
+// by the caller where warp-collective operations follow).
+__device__ __forceinline__ int ring_take(ItemRing& r, volatile int* abort_flag, int32_t* status,
+                                         bool& ok) {
+  const int s = (int)(r.k % kRing);
+  ok = mbar_wait(r.full + 8 * s, (r.k / kRing) & 1, abort_flag, status);
+  if (!ok) return -1;
+  const int v = r.slot[s];
+  mbar_arrive(r.empty + 8 * s);
+  ++r.k;
+  return v;
+}
+
 // ------------------------------------------------------------------------------------------
 // Producer
 // ------------------------------------------------------------------------------------------
@@ -148,12 +194,17 @@ __device__ __forceinline__ Item decode_item(int4 v) {
 template <int D>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               const CUtensorMap* tmV, const AttnArgs& a, uint32_t sbase,
-                              uint32_t bars, int n_items, volatile int* abort_flag, bool loads_v) {
+                              uint32_t bars, int n_items, volatile int* abort_flag, bool loads_v,
+                              ItemRing ring) {
   using C = Cfg<D>;
   uint32_t nq[2] = {0, 0};   // Q loads per query tile
   uint32_t g = 0;            // K (or V) loads
   bool ok = true;
-  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+  for (;;) {
+    // Lane 0 claims the CTA's next item; lane 1 reads the claims from the ring.
+    const int it = loads_v ? ring_take(ring, abort_flag, a.status, ok)
+                           : ring_claim(ring, a.queue, n_items, abort_flag, a.status, ok);
+    if (!ok || it < 0) break;
     const Item w = decode_item(a.items[it]);
     if (w.n_kv == 0) continue;
     if (!loads_v) {
@@ -288,7 +339,7 @@ struct PendingPV {
 
 template <int D>
 __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
-                         int n_items, volatile int* abort_flag) {
+                         volatile int* abort_flag, ItemRing ring) {
   using C = Cfg<D>;
   constexpr uint32_t kIdescQKFull = idesc_bf16_f32(C::BM, C::BN, false, false);
   // QK^T of a trimmed tile: N = keys of the tile rounded up to 16.
@@ -315,7 +366,9 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     pend.valid = 0;
     return true;
   };
-  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+  for (;;) {
+    const int it = ring_take(ring, abort_flag, a.status, ok);
+    if (!ok || it < 0) break;
     const Item w = decode_item(a.items[it]);
     if (w.n_kv == 0) continue;
     const bool has_b = w.nrows > C::BM;
@@ -573,11 +626,14 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int s
 // the epilogue. Slot s is reused for the item after next once all 256 softmax threads have taken
 // the scores out of it.
 template <int D>
-__device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars, int n_items,
-                          volatile int* abort_flag, int t) {
+__device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
+                          volatile int* abort_flag, int t, ItemRing ring) {
   using C = Cfg<D>;
   uint32_t n = 0;
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++n) {
+  bool ok = true;
+  for (;; ++n) {
+    const int it = ring_take(ring, abort_flag, a.status, ok);
+    if (!ok || it < 0) return;
     const Item w = decode_item(a.items[it]);
     const int slot = n & 1;
     if (!mbar_wait(bars + 8 * (C::B_DIAGEMPTY + slot), ((n >> 1) & 1) ^ 1, abort_flag, a.status))
@@ -602,8 +658,8 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars, int n
 
 template <int D>
 __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
-                             const float* sd_buf, int n_items, volatile int* abort_flag, int warp,
-                             int lane) {
+                             const float* sd_buf, volatile int* abort_flag, int warp, int lane,
+                             ItemRing ring) {
   using C = Cfg<D>;
   const int grp = (warp - 2) >> 2;            // query tile A (0) or B (1) of each item
   const int quarter = warp & 3;               // TMEM lane quarter this warp may access
@@ -616,7 +672,10 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
   uint32_t lt = 0, oi = 0;                    // S_w fills and O_w-ready completions seen
   bool ok = true;
   uint32_t n = 0;                             // items walked (diagonal-score slot sequence)
-  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x, ++n) {
+  for (;; ++n) {
+    const int it = ring_take(ring, abort_flag, a.status, ok);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok || it < 0) break;
     const Item w = decode_item(a.items[it]);
     const int slot = n & 1;
     if (grp == 1 && w.nrows <= C::BM) {
@@ -762,7 +821,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using C = Cfg<D>;
-  if (*a.status != 0) return;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -770,8 +828,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bars = sbase + C::OFF_BAR;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* skip = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  // An error recorded earlier on the stream makes the launch a no-op; one thread reads the status
+  // so that the whole CTA takes the same decision.
+  if (threadIdx.x == 0) *skip = *a.status != 0;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * C::QS; ++i) {
       mbar_init(bars + 8 * (C::B_QFULL + i), 1);
@@ -792,6 +854,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (C::B_DIAGEMPTY + i), kSoftmaxThreads);
     }
     mbar_init(bars + 8 * C::B_DRAIN, 1);
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(bars + 8 * (C::B_RINGFULL + i), 1);
+      mbar_init(bars + 8 * (C::B_RINGEMPTY + i), kRingReaders);
+    }
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
@@ -810,18 +876,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_items = *a.n_items;
+  ItemRing ring{reinterpret_cast<volatile int*>(smem + C::OFF_RING), bars + 8 * C::B_RINGFULL,
+                bars + 8 * C::B_RINGEMPTY, 0u};
 
-  if (warp == 0) {
-    if (lane < 2)
-      producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag, lane == 1);
-  } else if (warp == 1) {
-    if (lane == 0) mma_role<D>(a, sbase, bars, tmem, n_items, abort_flag);
-  } else if (warp < 10) {
-    softmax_role<D>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG), n_items,
-                    abort_flag, warp, lane);
-  } else {
-    diag_role<D>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), bars, n_items, abort_flag,
-                 threadIdx.x - 320);
+  if (!*skip) {
+    if (warp == 0) {
+      if (lane < 2)
+        producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag, lane == 1, ring);
+    } else if (warp == 1) {
+      if (lane == 0) mma_role<D>(a, sbase, bars, tmem, abort_flag, ring);
+    } else if (warp < 10) {
+      softmax_role<D>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
+                      abort_flag, warp, lane, ring);
+    } else {
+      diag_role<D>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), bars, abort_flag,
+                   threadIdx.x - 320, ring);
+    }
   }
 
   tc_fence_before();
@@ -829,6 +899,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  // The last CTA to finish resets the run-time queue for the next launch on the stream.
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&a.queue[1], 1) == (int)gridDim.x - 1) {
+      a.queue[0] = 0;
+      a.queue[1] = 0;
+      __threadfence();
+    }
   }
 }
 
@@ -989,7 +1068,8 @@ extern "C" int jagged_cand_attn_plan(const void* offsets, const void* candidate_
     return JCA_ERR_CUDA;
   if (launch_work_queue(offsets, ws + L.hist_lo, ws + L.hist_hi, kv_count, B, T, T, H, idx_bits,
                         reinterpret_cast<int32_t*>(ws + L.items), L.max_items,
-                        reinterpret_cast<int32_t*>(ws + L.n_items), status, st) != cudaSuccess)
+                        reinterpret_cast<int32_t*>(ws + L.n_items), status, st,
+                        reinterpret_cast<int32_t*>(ws + L.queue)) != cudaSuccess)
     return JCA_ERR_CUDA;
   return JCA_OK;
 }
@@ -1021,6 +1101,7 @@ extern "C" int jagged_cand_attn_run(const void* q, const void* k, const void* v,
   a.out = out;
   a.items = reinterpret_cast<const int4*>(ws + L.items);
   a.n_items = reinterpret_cast<const int32_t*>(ws + L.n_items);
+  a.queue = reinterpret_cast<int32_t*>(ws + L.queue);
   a.status = status;
   a.H = H;
   a.out_fp32 = out_fp32 ? 1 : 0;
@@ -1079,7 +1160,8 @@ extern "C" int cand_only_attn_plan(const void* cand_offsets, const void* hist_of
   }
   if (launch_work_queue(cand_offsets, kv_lo, kv_hi, kv_count, B, Nc, Th, H, idx_bits,
                         reinterpret_cast<int32_t*>(ws + L.items), L.max_items,
-                        reinterpret_cast<int32_t*>(ws + L.n_items), status, st) != cudaSuccess)
+                        reinterpret_cast<int32_t*>(ws + L.n_items), status, st,
+                        reinterpret_cast<int32_t*>(ws + L.queue)) != cudaSuccess)
     return JCA_ERR_CUDA;
   return JCA_OK;
 }
@@ -1114,6 +1196,7 @@ extern "C" int cand_only_attn_run(const void* cand_q, const void* own_k, const v
   a.out = out;
   a.items = reinterpret_cast<const int4*>(ws + L.items);
   a.n_items = reinterpret_cast<const int32_t*>(ws + L.n_items);
+  a.queue = reinterpret_cast<int32_t*>(ws + L.queue);
   a.status = status;
   a.H = H;
   a.out_fp32 = out_fp32 ? 1 : 0;

@@ -210,13 +210,18 @@ template <typename IdxT>
 __global__ void __launch_bounds__(1024) work_queue_kernel(
     const IdxT* __restrict__ qoff, const IdxT* __restrict__ kvlo, const IdxT* __restrict__ kvhi,
     const int32_t* __restrict__ kv_count, int64_t B, int64_t q_rows, int64_t kv_rows, int H,
-    int4* __restrict__ items, int64_t max_items, int32_t* n_items, int32_t* status) {
+    int4* __restrict__ items, int64_t max_items, int32_t* n_items, int32_t* status,
+    int32_t* queue_ctl) {
   __shared__ unsigned long long s_cnt[kQueueBuckets];
   __shared__ unsigned long long s_cursor[kQueueBuckets];
   __shared__ unsigned long long s_warp[32];
   __shared__ unsigned long long s_total;
   __shared__ int s_bad;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (queue_ctl != nullptr && tid == 0) {
+    queue_ctl[0] = 0;
+    queue_ctl[1] = 0;
+  }
   if (*status != 0) {
     if (tid == 0) *n_items = 0;
     return;
@@ -329,7 +334,8 @@ WorkspaceLayout workspace_layout(int64_t B, int64_t rows, int H) {
   w.items = p;
   p = align_up(p + 16 * (size_t)w.max_items, 256);
   w.n_items = p;
-  p = align_up(p + 4, 256);
+  w.queue = p + 16;
+  p = align_up(p + 32, 256);
   w.total = p;
   return w;
 }
@@ -382,15 +388,15 @@ cudaError_t launch_work_queue(const void* q_offsets, const void* kv_lo, const vo
                               const int32_t* kv_count, int64_t B, int64_t q_rows,
                               int64_t kv_rows, int H, int idx_bits, int32_t* items,
                               int64_t max_items, int32_t* n_items, int32_t* status,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int32_t* queue_ctl) {
   if (idx_bits == 32)
     work_queue_kernel<int32_t><<<1, kQueueBuckets, 0, stream>>>(
         (const int32_t*)q_offsets, (const int32_t*)kv_lo, (const int32_t*)kv_hi, kv_count, B,
-        q_rows, kv_rows, H, (int4*)items, max_items, n_items, status);
+        q_rows, kv_rows, H, (int4*)items, max_items, n_items, status, queue_ctl);
   else
     work_queue_kernel<int64_t><<<1, kQueueBuckets, 0, stream>>>(
         (const int64_t*)q_offsets, (const int64_t*)kv_lo, (const int64_t*)kv_hi, kv_count, B,
-        q_rows, kv_rows, H, (int4*)items, max_items, n_items, status);
+        q_rows, kv_rows, H, (int4*)items, max_items, n_items, status, queue_ctl);
   return cudaGetLastError();
 }
 

@@ -34,6 +34,8 @@ struct WorkspaceLayout {
   size_t kv_count = 0;   // int32 [B]      segment-1 tokens per user
   size_t items = 0;      // int4  [max_items]
   size_t n_items = 0;    // int32 [1]
+  size_t queue = 0;      // int32 [2]: next item to claim, CTAs finished (the attention kernel's
+                         // run-time queue; zeroed by the plan, reset by the kernel's last CTA)
   size_t total = 0;
   int64_t max_items = 0;
 };
@@ -54,10 +56,11 @@ cudaError_t launch_bounds(const int8_t* seg, const void* offsets, int64_t B, int
                           cudaStream_t stream, const void* cand_start = nullptr,
                           int8_t* seg_out = nullptr);
 
+// queue_ctl non-null: also zero the attention kernel's two run-time queue counters.
 cudaError_t launch_work_queue(const void* q_offsets, const void* kv_lo, const void* kv_hi,
                               const int32_t* kv_count, int64_t B, int64_t q_rows,
                               int64_t kv_rows, int H, int idx_bits, int32_t* items,
                               int64_t max_items, int32_t* n_items, int32_t* status,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int32_t* queue_ctl = nullptr);
 
 }  // namespace jca
