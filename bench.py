@@ -348,6 +348,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     if rank == 0 and world == 1 and not args.no_extras:
         line["cand_only"] = run_cand_only_extras(args, dev, stream, peaks)
+        line["rope"] = run_rope_extras(args, dev, stream, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         users = oracle_sample_users(batch, args.cpu_sample_stride, 3)
         fl, tok, times = time_oracle(batch, users, repeats=1)
@@ -359,6 +360,54 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def run_rope_extras(args, dev, stream, peaks):
+    """Right-anchored RoPE on the 256-user workload's queries and keys: positions, then the
+    rotation of each tensor in place. The rotation reads and writes the tensor once (HBM-bound);
+    reported: kernel time per tensor and algorithmic GB/s against the measured copy bandwidth."""
+    import torch
+    import oracle
+    import synth
+    from candidate_isolated_jagged_b200 import jca
+    b = synth.users256()
+    off_np = oracle.offsets_from_lengths(b.row_lengths)
+    seg = torch.tensor(oracle.segment_ids(off_np, b.cand_start), device=dev)
+    off = torch.tensor(off_np, device=dev)
+    q, k = b.q.to(dev), b.k.to(dev)
+    pos = torch.empty(b.T, dtype=torch.int32, device=dev)
+    st = jca.new_status(dev)
+    for _ in range(3):
+        jca.jca_rope_positions(seg, off, pos, 4096, st, stream=stream)
+        jca.jca_apply_rope(q, q, pos, stream=stream)
+    n = max(10, min(args.steps, 50))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for _ in range(n):
+        jca.jca_rope_positions(seg, off, pos, 4096, st, stream=stream)
+    ev[1].record(stream)
+    for _ in range(n):
+        jca.jca_apply_rope(q, q, pos, stream=stream)
+        jca.jca_apply_rope(k, k, pos, stream=stream)
+    ev[2].record(stream)
+    torch.cuda.synchronize(dev)
+    jca.check_status(st, "rope")
+    pos_ms = ev[0].elapsed_time(ev[1]) / n
+    rot_ms = ev[1].elapsed_time(ev[2]) / (2 * n)
+    byts = 2 * q.numel() * 2   # one bf16 read and one bf16 write per element
+    res = {
+        "workload": "users256 queries and keys (T=%d, H=%d, d=%d), history_end 4096" % (b.T, b.H, b.d),
+        "positions_ms": pos_ms,
+        "rotate_ms_per_tensor": rot_ms,
+        "roofline": {"bound": "hbm", "achieved": byts / rot_ms / 1e6, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": byts / rot_ms / 1e6 / peaks["hbm_gbs"],
+                     "algorithmic_bytes_per_launch": byts},
+        "launches_timed": 3 * n,
+    }
+    del q, k
+    torch.cuda.empty_cache()
+    return res
 
 
 def run_cand_only_extras(args, dev, stream, peaks):

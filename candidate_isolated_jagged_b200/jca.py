@@ -48,6 +48,8 @@ _SIGNATURES = {
                                     c_vp, c_sz, c_vp, c_vp]),
     "cand_only_attn_run": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i64,
                                    c_i64, c_i32, c_i32, c_f32, c_vp, c_sz, c_vp, c_vp]),
+    "jca_rope_positions": (c_i32, [c_vp, c_vp, c_i64, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp]),
+    "jca_apply_rope": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp]),
     "jca_noalloc_scratch_bytes": (c_sz, []),
     "jagged_cand_attn_fwd_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp,
                                              c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp,
@@ -269,6 +271,22 @@ def jagged_cand_attn_fwd_noalloc(q, k, v, out, offsets, candidate_start=None, se
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), _ptr(candidate_start),
         _ptr(seg), B, T, H, d, float(scale), _idx_bits(offsets), _ptr(status), _stream(stream)),
         "jagged_cand_attn_fwd_noalloc")
+
+
+def jca_rope_positions(seg, offsets, positions, history_end: int, status, stream=None) -> int:
+    """Right-anchored positions (int32 [T]) of the tokens of a segment-ID array."""
+    B = offsets.numel() - 1
+    T = seg.numel()
+    return _check(lib().jca_rope_positions(_ptr(seg), _ptr(offsets), B, T, int(history_end),
+                                           _idx_bits(offsets), _ptr(positions), _ptr(status),
+                                           _stream(stream)), "jca_rope_positions")
+
+
+def jca_apply_rope(x, out, positions, base: float = 10000.0, stream=None) -> int:
+    """Rotate the rows of a [T, H, d] bf16 tensor by their positions (out may be x)."""
+    T, H, d = x.shape
+    return _check(lib().jca_apply_rope(_ptr(x), _ptr(out), _ptr(positions), T, H, d, float(base),
+                                       _stream(stream)), "jca_apply_rope")
 
 
 def jca_noalloc_scratch_bytes() -> int:

@@ -257,6 +257,37 @@ int jagged_cand_attn_fwd_noalloc(const void* q, const void* k, const void* v, vo
                                  const int8_t* seg, int64_t B, int64_t T, int H, int d_head,
                                  float scale, int idx_bits, int32_t* status, jca_stream_t stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Right-anchored rotary position embedding (候选隔离注意力掩码, section 位置编码：候选共用一个位置):
+ * the history is right-aligned so that the newest history record of every user sits at
+ * history_end - 1 whatever its length, and every candidate sits at history_end; candidate order
+ * therefore never enters a score. Applied to the queries and keys before jagged_cand_attn_fwd or
+ * cand_only_attn_fwd (scores depend only on position differences, so any constant history_end
+ * gives the same attention output).
+ * ------------------------------------------------------------------------------------------- */
+
+/* Positions of the packed tokens of a segment-ID array. Per user row [offsets[b], offsets[b+1]):
+ * the k-th segment-1 token (prefix and history, in row order) of a row with n of them gets
+ * history_end - n + k; a candidate (segment -1) gets history_end; a padding token (segment 0)
+ * gets history_end - n + (segment-1 tokens before it), a value no score reads.
+ *   seg        device int8 [T]; offsets device [B+1] (idx_bits 32 or 64);
+ *   positions  device int32 [T] (written; values are clamped to the int32 range).
+ * Errors: as jca_bounds_from_segment_ids for the arguments; JCA_STATUS_BAD_OFFSETS in *status for
+ * offsets that are not monotone or do not end at T (then nothing further is written). */
+int jca_rope_positions(const int8_t* seg, const void* offsets, int64_t B, int64_t T,
+                       int64_t history_end, int idx_bits, int32_t* positions, int32_t* status,
+                       jca_stream_t stream);
+
+/* Rotates every row of a token-major [T, H, d_head] bf16 tensor by its token's position: for each
+ * head and each pair (j, j + d_head/2), (a, b) -> (a cos(p t_j) - b sin(p t_j),
+ * a sin(p t_j) + b cos(p t_j)) with t_j = base^(-2j/d_head), computed in fp32 and rounded once to
+ * bf16. out may equal x (in place); both 16-byte aligned, caller-owned device memory.
+ *   positions  device int32 [T], e.g. from jca_rope_positions; base > 1 (10000 in the usual form).
+ * Errors: JCA_ERR_HEAD_DIM, JCA_ERR_SHAPE (T < 0, H < 1, base <= 1), JCA_ERR_NULL, JCA_ERR_ALIGN,
+ * JCA_ERR_CUDA. Nothing is reported through a status word: every input is valid. */
+int jca_apply_rope(const void* x, void* out, const int32_t* positions, int64_t T, int H,
+                   int d_head, float base, jca_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
