@@ -18,4 +18,7 @@ from .workloads import (  # noqa: F401
     custom_batch,
     custom_cand_only,
     users256_history_lengths,
+    StackBatch,
+    custom_stack,
+    stack_users256,
 )

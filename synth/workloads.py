@@ -180,6 +180,50 @@ def custom_cand_only(
     return CandOnlyBatch(name, hl, hvld, cc, cq, ck, cv, hk, hv, int(H), int(d), int(seed))
 
 
+@dataclass
+class StackBatch:
+    """Inputs of a layer stack over a jagged batch.
+
+    ``batch`` gives the row layout only (its small q, k, v are not used by the stack); ``x`` is the
+    bf16 [T, D] input of the first layer (D = H d) and ``weights`` one (Wq, Wk, Wv, Wo) bf16 [D, D]
+    tuple per layer, laid out so that a projection is ``x @ W``.
+    """
+
+    batch: Batch
+    x: torch.Tensor
+    weights: list
+    n_cand_only: int
+    H: int
+    d: int
+
+    @property
+    def D(self) -> int:
+        return int(self.x.shape[1])
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+
+def custom_stack(hist_lengths: Sequence[int], prefix, n_cand, H: int, d: int, n_layers: int,
+                 n_cand_only: int, seed: int = 0, pad_hist_to: Optional[int] = None,
+                 valid_override: Optional[np.ndarray] = None, name: str = "custom_stack"
+                 ) -> StackBatch:
+    """Row layout as ``custom_batch``; then, from a second generator seeded ``seed + 1000``, the
+    input x ~ N(0, 1) and, layer by layer, Wq, Wk, Wv, Wo ~ N(0, 1/D) (fp32, cast to bf16), so that
+    the projections keep the residual stream's scale."""
+    b = custom_batch(hist_lengths, prefix, n_cand, H=1, d=16, seed=seed, pad_hist_to=pad_hist_to,
+                     valid_override=valid_override, name=name)
+    D = H * d
+    gen = torch.Generator().manual_seed(int(seed) + 1000)
+    x = torch.randn(b.T, D, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+    weights = []
+    for _ in range(n_layers):
+        weights.append(tuple((torch.randn(D, D, generator=gen, dtype=torch.float32)
+                              / float(np.sqrt(D))).to(torch.bfloat16) for _ in range(4)))
+    return StackBatch(b, x, weights, int(n_cand_only), int(H), int(d))
+
+
 # ---------------------------------------------------------------------------------------------
 # The five named workloads.
 # ---------------------------------------------------------------------------------------------
@@ -230,6 +274,14 @@ def retrieval() -> CandOnlyBatch:
     40,000 single-token candidates); H=4, d=32 (D = 128), seed 2."""
     return custom_cand_only(np.full(16, 240), np.full(16, 40000), H=4, d=32, seed=2,
                             name="retrieval")
+
+
+def stack_users256() -> StackBatch:
+    """The 256-user rows (as ``users256``) through 8 layers whose last 2 are candidate-only, as in
+    the pages' flagship ranking configuration; H=8, d=128 (D = 1024), seed 0."""
+    n = users256_history_lengths(0)
+    return custom_stack(n, prefix=4, n_cand=64, H=8, d=128, n_layers=8, n_cand_only=2, seed=0,
+                        name="stack_users256")
 
 
 WORKLOADS = {
