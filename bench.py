@@ -349,6 +349,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if rank == 0 and world == 1 and not args.no_extras:
         line["cand_only"] = run_cand_only_extras(args, dev, stream, peaks)
         line["rope"] = run_rope_extras(args, dev, stream, peaks)
+        line["stack"] = run_stack_extras(args, dev, stream, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         users = oracle_sample_users(batch, args.cpu_sample_stride, 3)
         fl, tok, times = time_oracle(batch, users, repeats=1)
@@ -406,6 +407,61 @@ def run_rope_extras(args, dev, stream, peaks):
         "launches_timed": 3 * n,
     }
     del q, k
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_stack_extras(args, dev, stream, peaks):
+    """The layer stack on the 256-user rows: 8 layers (D = 1024, H = 8, d = 128) whose last 2 are
+    candidate-only, with right-anchored RoPE, through jca_stack_fwd; and, for comparison, the same
+    8 layers all run over whole rows (no candidate-only tail). Reported: ms per stack forward,
+    useful TFLOP/s (projection GEMMs + effective attention FLOPs) and tokens/s."""
+    import torch
+    import synth
+    from candidate_isolated_jagged_b200 import jca, metrics
+    sb = synth.stack_users256()
+    b = sb.batch
+    T, D, H = b.T, sb.D, sb.H
+    n1 = b.prefix + b.hist_real
+    Nc, Th = int(b.n_cand.sum()), int(n1.sum())
+    x = sb.x.to(dev)
+    out = torch.empty_like(x)
+    w = torch.stack([torch.stack(list(t)) for t in sb.weights]).to(dev)
+    off = torch.tensor(np.concatenate([[0], np.cumsum(b.row_lengths)]), dtype=torch.int64,
+                       device=dev)
+    cs = torch.tensor(b.cand_start, dtype=torch.int64, device=dev)
+    res = {"workload": ("users256 rows (T=%d, %d candidates, %d history tokens), D=%d, H=%d, "
+                        "8 layers, RoPE history_end 8192" % (T, Nc, Th, D, H))}
+    for name, n_co in (("cand_only_tail_2", sb.n_cand_only), ("all_full", 0)):
+        ws = torch.empty(jca.jca_stack_workspace_bytes(b.B, T, Nc, Th, H, sb.d), dtype=torch.uint8,
+                         device=dev)
+        st = jca.new_status(dev)
+
+        def fwd():
+            jca.jca_stack_fwd(x, out, w, n_co, off, cs, None, Nc=Nc, Th=Th, H=H, history_end=8192,
+                              workspace=ws, status=st, stream=stream)
+
+        for _ in range(3):
+            fwd()
+        n = 10
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        e0.record(stream)
+        for _ in range(n):
+            fwd()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        jca.check_status(st, "stack " + name)
+        ms = e0.elapsed_time(e1) / n
+        fl = metrics.stack_flops(n1, b.n_cand, T, D, H, len(sb.weights), n_co)
+        total = fl["gemm"] + fl["attention"]
+        res[name] = {"ms": ms, "useful_tflops": total / ms / 1e9,
+                     "pct_of_bf16_peak": 100 * total / ms / 1e9 / peaks["bf16_tflops"],
+                     "gemm_tflop": fl["gemm"] / 1e12, "attention_tflop": fl["attention"] / 1e12,
+                     "candidates_per_s": Nc / ms * 1e3, "launches_timed": n}
+        del ws
+    res["speedup_of_tail"] = res["all_full"]["ms"] / res["cand_only_tail_2"]["ms"]
+    del x, out, w
     torch.cuda.empty_cache()
     return res
 

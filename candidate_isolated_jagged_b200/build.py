@@ -22,6 +22,9 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libjca.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# cuBLASLt serves the layer stack's dense projections. Inside a PyTorch process the loader reuses
+# the libcublasLt.so.12 that torch has already loaded; elsewhere the toolkit's copy is found.
+LINK = ["-L/usr/local/cuda/lib64", "-lcublasLt", "-Xlinker", "-rpath=/usr/local/cuda/lib64"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + INCLUDE, "-I" + CSRC]
 
@@ -56,7 +59,7 @@ def build(verbose: bool = False) -> str:
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
     tmp = LIB + ".tmp"
-    cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
+    cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs, *LINK]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stdout}\n{res.stderr}")

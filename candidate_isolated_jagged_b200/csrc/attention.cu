@@ -1250,6 +1250,8 @@ extern "C" const char* jca_status_string(int code) {
     case JCA_STATUS_BAD_SEG_LAYOUT: return "a history token follows a candidate inside a row";
     case JCA_STATUS_BAD_SEG_VALUE: return "segment ID outside the allowed values";
     case JCA_STATUS_QUEUE_OVERFLOW: return "work queue overflow";
+    case JCA_STATUS_BAD_SPLIT:
+      return "history/candidate token counts differ from the totals given to the stack";
     case JCA_STATUS_TIMEOUT: return "an attention pipeline wait timed out";
     default: return "unknown code";
   }

@@ -50,6 +50,10 @@ _SIGNATURES = {
                                    c_i64, c_i32, c_i32, c_f32, c_vp, c_sz, c_vp, c_vp]),
     "jca_rope_positions": (c_i32, [c_vp, c_vp, c_i64, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp]),
     "jca_apply_rope": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp]),
+    "jca_stack_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i64, c_i32, c_i32]),
+    "jca_stack_fwd": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64,
+                              c_i64, c_i32, c_i32, c_f32, c_i64, c_f32, c_i32, c_vp, c_sz, c_vp,
+                              c_vp]),
     "jca_noalloc_scratch_bytes": (c_sz, []),
     "jagged_cand_attn_fwd_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp,
                                              c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp,
@@ -287,6 +291,35 @@ def jca_apply_rope(x, out, positions, base: float = 10000.0, stream=None) -> int
     T, H, d = x.shape
     return _check(lib().jca_apply_rope(_ptr(x), _ptr(out), _ptr(positions), T, H, d, float(base),
                                        _stream(stream)), "jca_apply_rope")
+
+
+def jca_stack_workspace_bytes(B: int, T: int, Nc: int, Th: int, H: int, d_head: int) -> int:
+    return int(lib().jca_stack_workspace_bytes(int(B), int(T), int(Nc), int(Th), int(H),
+                                               int(d_head)))
+
+
+def jca_stack_fwd(x, x_out, weights, n_cand_only: int, offsets, candidate_start=None, seg=None,
+                  Nc: int = 0, Th: int = 0, H: int = 1, scale: float = 0.0,
+                  history_end: Optional[int] = None, rope_base: float = 10000.0,
+                  workspace: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                  stream=None) -> int:
+    """Layer stack with candidate-only tail layers: x [T, D] bf16 -> x_out [T, D] bf16 through
+    weights [n_layers, 4, D, D] bf16 (Wq, Wk, Wv, Wo per layer, x @ W). Nc / Th: total candidate and
+    history tokens. history_end None turns RoPE off."""
+    T, D = x.shape
+    n_layers = weights.shape[0] if weights.dim() == 4 else 0
+    d = D // int(H)
+    B = offsets.numel() - 1
+    if workspace is None:
+        workspace = torch.empty(jca_stack_workspace_bytes(B, T, Nc, Th, H, d), dtype=torch.uint8,
+                                device=x.device)
+    if status is None:
+        status = new_status(x.device)
+    return _check(lib().jca_stack_fwd(
+        _ptr(x), _ptr(x_out), _ptr(weights), int(n_layers), int(n_cand_only), _ptr(offsets),
+        _ptr(candidate_start), _ptr(seg), B, T, int(Nc), int(Th), int(H), d, float(scale),
+        -1 if history_end is None else int(history_end), float(rope_base), _idx_bits(offsets),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)), "jca_stack_fwd")
 
 
 def jca_noalloc_scratch_bytes() -> int:

@@ -66,6 +66,8 @@ enum jca_code {
   JCA_STATUS_BAD_SEG_LAYOUT = 4, /* a segment-1 token follows a candidate inside a row */
   JCA_STATUS_BAD_SEG_VALUE = 5,  /* a segment ID outside {-1, 0, 1} */
   JCA_STATUS_QUEUE_OVERFLOW = 6, /* more work items than the workspace bound (internal) */
+  JCA_STATUS_BAD_SPLIT = 7,      /* jca_stack_fwd: the segment IDs hold a different number of
+                                    history or candidate tokens than the caller's Th / Nc */
   JCA_STATUS_TIMEOUT = 16        /* a pipeline wait in the attention kernel gave up */
 };
 
@@ -287,6 +289,50 @@ int jca_rope_positions(const int8_t* seg, const void* offsets, int64_t B, int64_
  * JCA_ERR_CUDA. Nothing is reported through a status word: every input is valid. */
 int jca_apply_rope(const void* x, void* out, const int32_t* positions, int64_t T, int H,
                    int d_head, float base, jca_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Layer stack with candidate-only tail layers (候选隔离注意力掩码, section 只更新候选的末尾层 and its
+ * flowchart): the first n_layers - n_cand_only layers run over whole rows [prefix | history |
+ * candidates] under the isolation mask; then the states are split into the frozen history
+ * (segment 1, prefix included) and the candidates (segment -1), and each of the last n_cand_only
+ * layers updates only the candidates: their queries attend to the frozen history's keys/values
+ * (projected with that layer's weights) and to their own key/value. Padding rows (segment 0) and
+ * history rows keep the states they had at the split.
+ *
+ * A layer is x <- x + Attn(x Wq, x Wk, x Wv) Wo with square D x D weights, D = H * d_head, no bias
+ * and no normalisation (the pages describe only the attention part of a layer); with
+ * history_end >= 0, right-anchored RoPE (jca_rope_positions / jca_apply_rope, base rope_base) is
+ * applied to the queries and keys of every layer. Projections are bf16 GEMMs with fp32
+ * accumulation (cuBLASLt); every projection, RoPE output, attention output and residual sum is
+ * rounded once to bf16.
+ * ------------------------------------------------------------------------------------------- */
+
+/* Workspace bytes of jca_stack_fwd (0 for invalid sizes). */
+size_t jca_stack_workspace_bytes(int64_t B, int64_t T, int64_t Nc, int64_t Th, int H, int d_head);
+
+/*
+ *   x        [T, D] bf16, read (the first layer's input); x_out [T, D] bf16, written (may equal x).
+ *   weights  [n_layers, 4, D, D] bf16, read: per layer Wq, Wk, Wv, Wo, each row-major [D_in, D_out]
+ *            so that a projection is x @ W.
+ *   n_cand_only  number of candidate-only tail layers, 0 <= n_cand_only <= n_layers.
+ *   offsets [B+1], candidate_start [B] (row-relative) and seg [T] (nullable) as for
+ *            jagged_cand_attn_fwd.
+ *   Nc, Th   total candidate (segment -1) and history (segment 1) tokens of the batch; the host
+ *            needs them to size the tail layers without reading device memory. When they disagree
+ *            with the segment IDs, *status gets JCA_STATUS_BAD_SPLIT and the tail layers do not run.
+ *            Ignored (may be 0) when n_cand_only = 0. Nc + Th <= T.
+ *   scale    softmax scale (<= 0: 1/sqrt(d_head)); history_end < 0 turns RoPE off.
+ *   workspace >= jca_stack_workspace_bytes(B, T, Nc, Th, H, d_head) bytes, 256-byte aligned
+ *            (about (4 T + 2 (Nc + Th)) D bf16 elements plus 32 MiB for the GEMMs).
+ * Errors: the host errors of jagged_cand_attn_fwd; device errors in *status as the builders and
+ * attention kernels report them. After a device error x_out is unspecified (the GEMMs do not read
+ * the status word); the other kernels do nothing further.
+ */
+int jca_stack_fwd(const void* x, void* x_out, const void* weights, int n_layers, int n_cand_only,
+                  const void* offsets, const void* candidate_start, const int8_t* seg, int64_t B,
+                  int64_t T, int64_t Nc, int64_t Th, int H, int d_head, float scale,
+                  int64_t history_end, float rope_base, int idx_bits, void* workspace,
+                  size_t workspace_bytes, int32_t* status, jca_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -210,8 +210,15 @@ def custom_stack(hist_lengths: Sequence[int], prefix, n_cand, H: int, d: int, n_
                  valid_override: Optional[np.ndarray] = None, name: str = "custom_stack"
                  ) -> StackBatch:
     """Row layout as ``custom_batch``; then, from a second generator seeded ``seed + 1000``, the
-    input x ~ N(0, 1) and, layer by layer, Wq, Wk, Wv, Wo ~ N(0, 1/D) (fp32, cast to bf16), so that
-    the projections keep the residual stream's scale."""
+    input x ~ N(0, 1) and, layer by layer, Wq, Wk, Wv ~ N(0, 1/D) and Wo ~ N(0, 1/(D n_layers))
+    (fp32, cast to bf16).
+
+    The pages describe no normalisation inside a layer, so nothing resets the residual stream's
+    scale: with Wo ~ N(0, 1/D) each layer adds roughly its own variance (attention averages value
+    rows whose variance is the stream's), the states grow about 2x in variance per layer, and by
+    the eighth layer the scores are so large that softmax is nearly an argmax, where one-ulp
+    rounding differences pick other keys. Scaling Wo by 1/sqrt(n_layers) bounds the growth by a
+    factor of about e over the whole stack and keeps the scores of order one."""
     b = custom_batch(hist_lengths, prefix, n_cand, H=1, d=16, seed=seed, pad_hist_to=pad_hist_to,
                      valid_override=valid_override, name=name)
     D = H * d
@@ -219,8 +226,10 @@ def custom_stack(hist_lengths: Sequence[int], prefix, n_cand, H: int, d: int, n_
     x = torch.randn(b.T, D, generator=gen, dtype=torch.float32).to(torch.bfloat16)
     weights = []
     for _ in range(n_layers):
-        weights.append(tuple((torch.randn(D, D, generator=gen, dtype=torch.float32)
-                              / float(np.sqrt(D))).to(torch.bfloat16) for _ in range(4)))
+        w = [torch.randn(D, D, generator=gen, dtype=torch.float32) / float(np.sqrt(D))
+             for _ in range(4)]
+        w[3] = w[3] / float(np.sqrt(n_layers))
+        weights.append(tuple(t.to(torch.bfloat16) for t in w))
     return StackBatch(b, x, weights, int(n_cand_only), int(H), int(d))
 
 

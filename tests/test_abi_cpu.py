@@ -26,7 +26,7 @@ def test_header_declares_the_entry_points():
               "jca_build_work_queue", "jca_max_work_items", "jca_workspace_bytes",
               "jagged_cand_attn_fwd", "cand_only_attn_fwd", "jca_status_string",
               "jagged_cand_attn_plan", "jagged_cand_attn_run", "cand_only_attn_plan",
-              "cand_only_attn_run"]:
+              "cand_only_attn_run", "jca_stack_workspace_bytes", "jca_stack_fwd"]:
         assert n in names
 
 
@@ -46,7 +46,7 @@ def test_missing_library_fails_loudly(tmp_path):
 
 def test_status_strings(L):
     assert jca.status_string(0) == "ok"
-    for code in (-1, -2, -3, -4, -5, -6, -7, -8, 1, 2, 3, 4, 5, 6, 16):
+    for code in (-1, -2, -3, -4, -5, -6, -7, -8, -9, 1, 2, 3, 4, 5, 6, 7, 16):
         assert jca.status_string(code) != "unknown code"
     assert jca.status_string(12345) == "unknown code"
 
@@ -101,3 +101,36 @@ def test_host_argument_errors(L):
     cargs_bad = list(cargs)
     cargs_bad[4] = None
     assert L.cand_only_attn_fwd(*cargs_bad) == -1
+
+
+def test_stack_host_argument_errors(L):
+    p = _addr(0x10000)  # never dereferenced: every call below fails its host checks
+    st = _addr(0x20000)
+    ws = _addr(0x40000)
+    assert L.jca_stack_workspace_bytes(3, 20, 9, 8, 2, 16) > 0
+    assert L.jca_stack_workspace_bytes(3, 20, 15, 8, 2, 16) == 0     # Nc + Th > T
+    assert L.jca_stack_workspace_bytes(3, 20, 9, 8, 2, 24) == 0      # head dim
+    names = ["x", "x_out", "w", "n_layers", "n_cand_only", "off", "cs", "seg", "B", "T", "Nc", "Th",
+             "H", "d", "scale", "history_end", "base", "idx_bits", "ws", "ws_bytes", "status",
+             "stream"]
+    args = [p, p, p, 3, 1, p, p, None, 3, 20, 9, 8, 2, 16, 0.0, -1, 10000.0, 32, ws, 1 << 30, st,
+            None]
+
+    def call(**kw):
+        a = list(args)
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return L.jca_stack_fwd(*a)
+
+    assert call(idx_bits=16) == -5
+    assert call(d=24) == -3
+    assert call(n_cand_only=4) == -2         # more tail layers than layers
+    assert call(n_layers=-1) == -2
+    assert call(Nc=15) == -2                 # Nc + Th > T
+    assert call(history_end=5, base=1.0) == -2
+    assert call(x=None) == -1
+    assert call(w=None) == -1
+    assert call(cs=None) == -1               # neither candidate_start nor seg
+    assert call(x_out=_addr(0x10004)) == -4
+    assert call(ws=_addr(0x40010)) == -4
+    assert call(ws_bytes=4096) == -6
