@@ -350,6 +350,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         line["cand_only"] = run_cand_only_extras(args, dev, stream, peaks)
         line["rope"] = run_rope_extras(args, dev, stream, peaks)
         line["stack"] = run_stack_extras(args, dev, stream, peaks)
+        line["backward"] = run_backward_extras(args, dev, stream, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         users = oracle_sample_users(batch, args.cpu_sample_stride, 3)
         fl, tok, times = time_oracle(batch, users, repeats=1)
@@ -407,6 +408,72 @@ def run_rope_extras(args, dev, stream, peaks):
         "launches_timed": 3 * n,
     }
     del q, k
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_backward_extras(args, dev, stream, peaks):
+    """The training path on the 256-user workload: the forward with its log-sum-exp, then the
+    backward pass (plan, key-tile queue, row statistics, the dK/dV kernel and the dQ kernel), each
+    timed with CUDA events over repeated calls. Effective backward FLOPs follow the usual
+    flash-attention count, 2.5x the forward's (five d-deep products per allowed pair: the score,
+    dP, dV, dK and dQ); the kernels here recompute the score and dP once more (seven products)."""
+    import torch
+    import synth
+    from candidate_isolated_jagged_b200 import jca, metrics
+    b = synth.users256()
+    B, T, H, d = b.B, b.T, b.H, b.d
+    pairs = metrics.allowed_pairs_from_counts(b.prefix + b.hist_real, b.n_cand)
+    fwd_flops = metrics.effective_flops(pairs, H, d)
+    q, k, v = (t.to(dev) for t in (b.q, b.k, b.v))
+    dout = synth.upstream_grad(b.q.shape, 15).to(dev)
+    off = torch.tensor(np.concatenate([[0], np.cumsum(b.row_lengths)]), dtype=torch.int64,
+                       device=dev)
+    cs = torch.tensor(b.cand_start, dtype=torch.int64, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(T, H, dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    wsf = torch.empty(jca.jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=dev)
+    wsb = torch.empty(jca.jca_bwd_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=dev)
+    st = jca.new_status(dev)
+
+    def fwd():
+        jca.jagged_cand_attn_fwd_lse(q, k, v, out, lse, off, cs, None, workspace=wsf, status=st,
+                                     stream=stream)
+
+    def bwd():
+        jca.jagged_cand_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, off, cs, None,
+                                 workspace=wsb, status=st, stream=stream)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    n = 20
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for _ in range(n):
+        fwd()
+    ev[1].record(stream)
+    for _ in range(n):
+        bwd()
+    ev[2].record(stream)
+    torch.cuda.synchronize(dev)
+    jca.check_status(st, "backward")
+    f_ms = ev[0].elapsed_time(ev[1]) / n
+    b_ms = ev[1].elapsed_time(ev[2]) / n
+    bwd_flops = 2.5 * fwd_flops
+    res = {
+        "workload": "users256 (T=%d, H=%d, d=%d), dO ~ N(0,1) seed 15, bf16 gradients" % (T, H, d),
+        "fwd_lse_ms": f_ms, "fwd_lse_effective_tflops": fwd_flops / f_ms / 1e9,
+        "bwd_ms": b_ms, "bwd_effective_tflops": bwd_flops / b_ms / 1e9,
+        "bwd_pct_of_bf16_peak": 100 * bwd_flops / b_ms / 1e9 / peaks["bf16_tflops"],
+        "bwd_executed_tflops": 3.5 * fwd_flops / b_ms / 1e9,
+        "train_step_attention_ms": f_ms + b_ms,
+        "launches_per_bwd": 6,
+        "launches_timed": 2 * n,
+    }
+    del q, k, v, dout, out, lse, dq, dk, dv, wsf, wsb
     torch.cuda.empty_cache()
     return res
 

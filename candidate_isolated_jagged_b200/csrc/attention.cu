@@ -57,6 +57,7 @@ struct AttnArgs {
   int out_fp32;
   int out_v8;               // out is 32-byte aligned: rows are written with 32-byte stores
   float scale_log2;         // softmax scale * log2(e)
+  float* lse = nullptr;     // [Tq, H] natural-log softmax denominators, or null (not written)
 };
 
 // Depth of the shared ring through which every role receives the claimed work items.
@@ -572,6 +573,12 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int s
   }
   // Padding queries (segment 0) see no key and output 0.
   const float inv = (seg != 0 && l > 0.f) ? 1.f / l : 0.f;
+  if (a.lse != nullptr && row_ok) {
+    // log of the row's softmax denominator: l is relative to the reference max (log2 units),
+    // which the diagonal merge moved to max(m, sd) for a candidate; -inf for a padding row.
+    const float ref = cand ? fmaxf(m, sd) : m;
+    a.lse[base / D] = seg == 0 ? -INFINITY : (ref + log2f(l)) * 0.69314718055994531f;
+  }
   const float scale_o = alpha * inv, scale_v = beta * inv;
   constexpr int CW = D < 32 ? D : 32;            // columns per TMEM load
   constexpr int PER = (D / CW) >= 2 ? 2 : 1;     // loads per TMEM wait
@@ -1074,11 +1081,12 @@ extern "C" int jagged_cand_attn_plan(const void* offsets, const void* candidate_
   return JCA_OK;
 }
 
-extern "C" int jagged_cand_attn_run(const void* q, const void* k, const void* v, void* out,
-                                    int out_fp32, const int8_t* seg, int64_t B, int64_t T, int H,
-                                    int d_head, float scale, void* workspace,
-                                    size_t workspace_bytes, int32_t* status,
-                                    jca_stream_t stream) {
+namespace jca {
+namespace {
+
+int run_full(const void* q, const void* k, const void* v, void* out, int out_fp32, float* lse,
+             const int8_t* seg, int64_t B, int64_t T, int H, int d_head, float scale,
+             void* workspace, size_t workspace_bytes, int32_t* status, jca_stream_t stream) {
   int rc = check_sizes(32, d_head, B, T, T, H);
   if (rc) return rc;
   if (!status) return JCA_ERR_NULL;
@@ -1106,7 +1114,40 @@ extern "C" int jagged_cand_attn_run(const void* q, const void* k, const void* v,
   a.H = H;
   a.out_fp32 = out_fp32 ? 1 : 0;
   a.scale_log2 = scale * 1.4426950408889634f;
+  a.lse = lse;
   return launch_attention(d_head, a, q, T, k, v, T, reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace jca
+
+extern "C" int jagged_cand_attn_run(const void* q, const void* k, const void* v, void* out,
+                                    int out_fp32, const int8_t* seg, int64_t B, int64_t T, int H,
+                                    int d_head, float scale, void* workspace,
+                                    size_t workspace_bytes, int32_t* status,
+                                    jca_stream_t stream) {
+  return run_full(q, k, v, out, out_fp32, nullptr, seg, B, T, H, d_head, scale, workspace,
+                  workspace_bytes, status, stream);
+}
+
+extern "C" int jagged_cand_attn_fwd_lse(const void* q, const void* k, const void* v, void* out,
+                                        int out_fp32, float* lse, const void* offsets,
+                                        const void* candidate_start, const int8_t* seg, int64_t B,
+                                        int64_t T, int H, int d_head, float scale, int idx_bits,
+                                        void* workspace, size_t workspace_bytes, int32_t* status,
+                                        jca_stream_t stream) {
+  int rc = check_sizes(idx_bits, d_head, B, T, T, H);
+  if (rc) return rc;
+  if (!status || !offsets || (T > 0 && (!q || !k || !v || !out || !lse))) return JCA_ERR_NULL;
+  if (B > 0 && !seg && !candidate_start) return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+                !aligned(lse, 4)))
+    return JCA_ERR_ALIGN;
+  rc = jagged_cand_attn_plan(offsets, candidate_start, seg, B, T, H, d_head, idx_bits, workspace,
+                             workspace_bytes, status, stream);
+  if (rc) return rc;
+  return run_full(q, k, v, out, out_fp32, lse, seg, B, T, H, d_head, scale, workspace,
+                  workspace_bytes, status, stream);
 }
 
 extern "C" int jagged_cand_attn_fwd(const void* q, const void* k, const void* v, void* out,

@@ -1,0 +1,946 @@
+// Backward pass of jagged candidate-isolated attention on sm_100a (tcgen05 + TMEM + TMA).
+//
+// What it computes: the gradients of the forward's masked softmax attention (候选隔离注意力掩码,
+// sections 段 ID：掩码的表达方式 and 掩码长什么样), trained on the same packed layout the forward
+// serves (section 训练时的序列打包). Per user and head, with P the forward's probabilities,
+//   dV = P^T dO,   dP = dO V^T,   dS = P * (dP - D) with D = rowsum(dO * O),
+//   dQ = scale dS K,   dK = scale dS^T Q.
+// P is rebuilt tile by tile from the forward's log-sum-exp, so no [L, L] matrix exists anywhere.
+// The mask splits the work in three parts with no overlap and no atomics:
+//   * keys with segment 1 (prefix + history) are seen by every non-padding query of their user:
+//     a key-outer kernel (mode dKV) takes one 128-key tile of a user's history interval and walks
+//     all of the user's query tiles, accumulating dV = P^T dO and dK = dS^T Q in TMEM;
+//   * every query reads only the segment-1 keys plus, for a candidate, itself: a query-outer
+//     kernel (mode dQ) takes one 128-row query tile and walks the history key tiles,
+//     accumulating dQ = dS K in TMEM;
+//   * a candidate's own key and value are seen by that candidate alone, so their gradients (and
+//     the candidate's diagonal share of dQ) are scalar work done in the dQ kernel's epilogue on
+//     CUDA cores, like the forward's diagonal term.
+// Both modes share one kernel body. With O1/O2 the two "outer" tiles loaded once per unit and
+// I1/I2 the two "inner" tiles streamed through a ring, every inner step issues
+//   S = O1 I1^T and dP = O2 I2^T (SS MMAs, M = N = 128, K = d, fp32 in TMEM),
+// the compute warps (one TMEM lane = one outer row per thread) turn them into bf16 dS (and, for
+// dKV, bf16 P) written back over S / dP, and the MMA thread issues the TS MMAs that read them
+// from TMEM as the A operand:
+//   mode dQ  (O1 = Q, O2 = dO, I1 = K, I2 = V):   acc0 += dS I1
+//   mode dKV (O1 = K, O2 = V, I1 = Q, I2 = dO):   acc0 (dV) += P^T I2,  acc1 (dK) += dS^T I1.
+// TMEM columns: S | dP | acc0 | acc1 (128 each, 512 allocated).
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "jca_device.cuh"
+#include "jca_internal.h"
+
+namespace jca {
+namespace {
+
+using bf16 = __nv_bfloat16;
+
+constexpr int kModeDQ = 0;
+constexpr int kModeDKV = 1;
+constexpr int kBwdThreads = 192;     // warp 0 producer, warp 1 MMA, warps 2..5 compute
+constexpr int kBwdCompute = 128;
+constexpr int kBwdStages = 2;        // inner ring depth
+
+struct BwdArgs {
+  const bf16* q;
+  const bf16* k;
+  const bf16* v;
+  const bf16* dout;
+  void* dq;
+  void* dk;
+  void* dv;
+  const int8_t* seg;       // [T]
+  const float* lse2;       // [H][T]: log2-units log-sum-exp of each row; +inf = row sees no key
+  const float* dsum;       // [H][T]: rowsum(dO * O)
+  const int4* items;
+  const int32_t* n_items;
+  int32_t* status;
+  int64_t T;
+  int H;
+  int grad_fp32;
+  float scale;
+  float scale_log2;
+};
+
+template <int D>
+struct BCfg {
+  static constexpr int BM = kTileM;
+  static constexpr int ROW_BYTES = D * 2;
+  static constexpr int SW = ROW_BYTES >= 128 ? 128 : ROW_BYTES;
+  static constexpr int NBLK = ROW_BYTES / SW;
+  static constexpr int BOX_X = SW / 2;
+  static constexpr int TILE_BYTES = BM * ROW_BYTES;
+  static constexpr int BLK_BYTES = BM * SW;
+  static constexpr uint32_t LAYOUT = SW == 128 ? 2u : (SW == 64 ? 4u : 6u);
+  static constexpr int KSTEPS_QK = D / 16;
+  static constexpr int KSTEPS_PER_BLK = SW / 32;
+  static constexpr int OFF_OUT = 0;                                   // 2 tiles
+  static constexpr int OFF_IN = 2 * TILE_BYTES;                       // kBwdStages x 2 tiles
+  static constexpr int OFF_BAR = OFF_IN + kBwdStages * 2 * TILE_BYTES;
+  static constexpr int B_OUTFULL = 0;
+  static constexpr int B_OUTEMPTY = 1;
+  static constexpr int B_INFULL = 2;                                  // [kBwdStages]
+  static constexpr int B_INEMPTY = B_INFULL + kBwdStages;             // [kBwdStages]
+  static constexpr int B_SPFULL = B_INEMPTY + kBwdStages;             // S and dP written
+  static constexpr int B_DSFULL = B_SPFULL + 1;                       // dS (and P) written back
+  static constexpr int B_ACCFULL = B_DSFULL + 1;                      // unit's last TS MMA done
+  static constexpr int B_ACCFREE = B_ACCFULL + 1;                     // accumulators read
+  static constexpr int B_COLS = B_ACCFREE + 1;                        // [2] column stats (dKV)
+  static constexpr int B_DRAIN = B_COLS + 2;
+  static constexpr int NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_COLS = OFF_MISC + 16;                      // [2][2][128] floats
+  static constexpr int SMEM_USED = OFF_COLS + 2 * 2 * BM * 4;
+  static constexpr int SMEM_RAW = SMEM_USED + 1024;
+  // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
+  static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+  static constexpr uint32_t TMEM_S = 0, TMEM_P = 128, TMEM_A0 = 256, TMEM_A1 = 384,
+                            TMEM_COLS = 512;
+  static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
+};
+
+// One unit of work: `orows` outer rows starting at `orow0` for head h, against the inner rows
+// [in_lo, in_lo + in_len) walked in tiles of 128.
+struct Unit {
+  int orow0, orows, h, in_lo, in_len, holes, n_in;
+};
+
+// Units of an item. dQ items are the forward's work items (up to 256 query rows: two units);
+// dKV items hold one key tile.
+template <int MODE>
+__device__ __forceinline__ int unit_count(int4 v) {
+  if (MODE == kModeDKV) return 1;
+  return ((v.y & 511) + kTileM - 1) / kTileM;
+}
+
+template <int MODE>
+__device__ __forceinline__ Unit decode_unit(int4 v, int t) {
+  Unit u;
+  u.h = v.y >> 9;
+  const int rows = v.y & 511;
+  u.orow0 = v.x + t * kTileM;
+  u.orows = min(kTileM, rows - t * kTileM);
+  u.in_lo = v.z;
+  if (MODE == kModeDQ) {
+    u.in_len = v.w & 0x7fffffff;
+    u.holes = (int)((unsigned)v.w >> 31);
+  } else {
+    u.in_len = v.w;
+    u.holes = 0;
+  }
+  u.n_in = (u.in_len + kTileN - 1) / kTileN;
+  return u;
+}
+
+// ------------------------------------------------------------------------------------------
+// Producer: outer tiles once per unit, inner tile pairs through a kBwdStages ring.
+// ------------------------------------------------------------------------------------------
+template <int D, int MODE>
+__device__ void bwd_producer(const CUtensorMap* tmO1, const CUtensorMap* tmO2,
+                             const CUtensorMap* tmI1, const CUtensorMap* tmI2, const BwdArgs& a,
+                             uint32_t sbase, uint32_t bars, int n_items,
+                             volatile int* abort_flag) {
+  using C = BCfg<D>;
+  uint32_t u_count = 0, g = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+    const int4 raw = a.items[it];
+    const int nu = unit_count<MODE>(raw);
+    for (int t = 0; ok && t < nu; ++t) {
+      const Unit u = decode_unit<MODE>(raw, t);
+      if (u.n_in == 0) continue;
+      ok = mbar_wait(bars + 8 * C::B_OUTEMPTY, (u_count & 1) ^ 1, abort_flag, a.status);
+      if (!ok) break;
+      mbar_arrive_expect_tx(bars + 8 * C::B_OUTFULL, 2 * C::TILE_BYTES);
+      ++u_count;
+#pragma unroll
+      for (int c = 0; c < C::NBLK; ++c) {
+        tma_load_3d(sbase + C::OFF_OUT + c * C::BLK_BYTES, tmO1, bars + 8 * C::B_OUTFULL,
+                    c * C::BOX_X, u.h, u.orow0);
+        tma_load_3d(sbase + C::OFF_OUT + C::TILE_BYTES + c * C::BLK_BYTES, tmO2,
+                    bars + 8 * C::B_OUTFULL, c * C::BOX_X, u.h, u.orow0);
+      }
+      for (int i = 0; i < u.n_in; ++i, ++g) {
+        const int s = (int)(g % kBwdStages);
+        ok = mbar_wait(bars + 8 * (C::B_INEMPTY + s), ((g / kBwdStages) & 1) ^ 1, abort_flag,
+                       a.status);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bars + 8 * (C::B_INFULL + s), 2 * C::TILE_BYTES);
+        const uint32_t dst = sbase + C::OFF_IN + s * 2 * C::TILE_BYTES;
+        const int row = u.in_lo + i * kTileN;
+#pragma unroll
+        for (int c = 0; c < C::NBLK; ++c) {
+          tma_load_3d(dst + c * C::BLK_BYTES, tmI1, bars + 8 * (C::B_INFULL + s), c * C::BOX_X,
+                      u.h, row);
+          tma_load_3d(dst + C::TILE_BYTES + c * C::BLK_BYTES, tmI2, bars + 8 * (C::B_INFULL + s),
+                      c * C::BOX_X, u.h, row);
+        }
+      }
+    }
+  }
+  if (!ok) {
+    // Aborting: let the copies this thread started land before the CTA exits.
+    if (u_count > 0) mbar_wait_drain(bars + 8 * C::B_OUTFULL, (u_count - 1) & 1);
+    for (uint32_t n = g > (uint32_t)kBwdStages ? g - kBwdStages : 0; n < g; ++n)
+      mbar_wait_drain(bars + 8 * (C::B_INFULL + (int)(n % kBwdStages)), (n / kBwdStages) & 1);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// MMA issuer
+// ------------------------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                           uint32_t idesc) {
+  using C = BCfg<D>;
+#pragma unroll
+  for (int kk = 0; kk < C::KSTEPS_QK; ++kk) {
+    const uint32_t off =
+        ((kk / C::KSTEPS_PER_BLK) * C::BLK_BYTES + (kk % C::KSTEPS_PER_BLK) * 32) >> 4;
+    tc_mma(d_tmem, a + off, b + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// acc (+)= A[tmem, bf16 pairs, M = 128 lanes x K = 16 ksteps] * B[smem, MN-major, K rows x N = D].
+template <int D>
+__device__ __forceinline__ void bwd_mma_ts(uint32_t acc, uint32_t a_tmem, uint64_t b, int ksteps,
+                                           bool overwrite) {
+  using C = BCfg<D>;
+  constexpr uint32_t kIdesc = idesc_bf16_f32(C::BM, D, false, true);
+  constexpr uint32_t kStep = (16 * C::SW) >> 4;
+  for (int kk = 0; kk < ksteps; ++kk)
+    tc_mma_ts(acc, a_tmem + (uint32_t)kk * 8u, b + (uint64_t)(kk * kStep), kIdesc,
+              (overwrite && kk == 0) ? 0u : 1u);
+}
+
+template <int D, int MODE>
+__device__ void bwd_mma(const BwdArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                        int n_items, volatile int* abort_flag) {
+  using C = BCfg<D>;
+  constexpr uint32_t kIdescFull = idesc_bf16_f32(C::BM, kTileN, false, false);
+  constexpr uint32_t kIdesc0 = kIdescFull & ~(0x3Fu << 17);
+  const uint64_t o1 = smem_desc(sbase + C::OFF_OUT, 16, 8 * C::SW, C::LAYOUT);
+  const uint64_t o2 = o1 + (uint64_t)(C::TILE_BYTES >> 4);
+  const uint64_t in_k = smem_desc(sbase + C::OFF_IN, 16, 8 * C::SW, C::LAYOUT);
+  const uint64_t in_mn = smem_desc(sbase + C::OFF_IN, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
+  uint32_t u_count = 0, g = 0, ds_seen = 0, acc_units = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+    const int4 raw = a.items[it];
+    const int nu = unit_count<MODE>(raw);
+    for (int t = 0; ok && t < nu; ++t) {
+      const Unit u = decode_unit<MODE>(raw, t);
+      if (u.n_in == 0) continue;
+      ok = mbar_wait(bars + 8 * C::B_OUTFULL, u_count & 1, abort_flag, a.status);
+      if (!ok) break;
+      ++u_count;
+      tc_fence_after();
+      for (int i = 0; i < u.n_in; ++i, ++g) {
+        const int s = (int)(g % kBwdStages);
+        ok = mbar_wait(bars + 8 * (C::B_INFULL + s), (g / kBwdStages) & 1, abort_flag, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        const int valid = min(kTileN, u.in_len - i * kTileN);
+        const uint32_t idesc =
+            valid == kTileN ? kIdescFull
+                            : (kIdesc0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17));
+        const uint64_t i1 = in_k + (uint64_t)((s * 2 * C::TILE_BYTES) >> 4);
+        const uint64_t i2 = i1 + (uint64_t)(C::TILE_BYTES >> 4);
+        bwd_mma_ss<D>(tmem + C::TMEM_S, o1, i1, idesc);
+        bwd_mma_ss<D>(tmem + C::TMEM_P, o2, i2, idesc);
+        tc_commit(bars + 8 * C::B_SPFULL);
+        ok = mbar_wait(bars + 8 * C::B_DSFULL, ds_seen & 1, abort_flag, a.status);
+        if (!ok) break;
+        ++ds_seen;
+        if (i == 0 && acc_units > 0) {
+          ok = mbar_wait(bars + 8 * C::B_ACCFREE, (acc_units - 1) & 1, abort_flag, a.status);
+          if (!ok) break;
+        }
+        tc_fence_after();
+        const int ksteps = (valid + 15) >> 4;
+        const uint64_t m1 = in_mn + (uint64_t)((s * 2 * C::TILE_BYTES) >> 4);
+        const uint64_t m2 = m1 + (uint64_t)(C::TILE_BYTES >> 4);
+        if (MODE == kModeDQ) {
+          bwd_mma_ts<D>(tmem + C::TMEM_A0, tmem + C::TMEM_P, m1, ksteps, i == 0);
+        } else {
+          bwd_mma_ts<D>(tmem + C::TMEM_A0, tmem + C::TMEM_S, m2, ksteps, i == 0);
+          bwd_mma_ts<D>(tmem + C::TMEM_A1, tmem + C::TMEM_P, m1, ksteps, i == 0);
+        }
+        tc_commit(bars + 8 * (C::B_INEMPTY + s));
+      }
+      if (!ok) break;
+      tc_commit(bars + 8 * C::B_OUTEMPTY);
+      tc_commit(bars + 8 * C::B_ACCFULL);
+      ++acc_units;
+    }
+  }
+  if (!ok) {
+    tc_commit(bars + 8 * C::B_DRAIN);
+    mbar_wait_drain(bars + 8 * C::B_DRAIN, 0);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Compute warps
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ void store_row8(void* base, int fp32, size_t idx, const float* o) {
+  if (fp32) {
+    float* p = reinterpret_cast<float*>(base) + idx;
+    reinterpret_cast<float4*>(p)[0] = make_float4(o[0], o[1], o[2], o[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(o[4], o[5], o[6], o[7]);
+  } else {
+    reinterpret_cast<uint4*>(reinterpret_cast<bf16*>(base) + idx)[0] =
+        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                   pack_bf16x2(o[6], o[7]));
+  }
+}
+
+// Dot product of two bf16 rows of D elements.
+template <int D>
+__device__ __forceinline__ float row_dot(const bf16* x, const bf16* y) {
+  const uint4* xp = reinterpret_cast<const uint4*>(x);
+  const uint4* yp = reinterpret_cast<const uint4*>(y);
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < D / 8; ++c) {
+    const uint4 xv = ld_global_nc_v4(xp + c), yv = ld_global_nc_v4(yp + c);
+    acc0 = fmaf(bf16_lo(xv.x), bf16_lo(yv.x), acc0);
+    acc1 = fmaf(bf16_hi(xv.x), bf16_hi(yv.x), acc1);
+    acc0 = fmaf(bf16_lo(xv.y), bf16_lo(yv.y), acc0);
+    acc1 = fmaf(bf16_hi(xv.y), bf16_hi(yv.y), acc1);
+    acc0 = fmaf(bf16_lo(xv.z), bf16_lo(yv.z), acc0);
+    acc1 = fmaf(bf16_hi(xv.z), bf16_hi(yv.z), acc1);
+    acc0 = fmaf(bf16_lo(xv.w), bf16_lo(yv.w), acc0);
+    acc1 = fmaf(bf16_hi(xv.w), bf16_hi(yv.w), acc1);
+  }
+  return acc0 + acc1;
+}
+
+__device__ __forceinline__ void unpack8(uint4 w, float* o) {
+  o[0] = bf16_lo(w.x); o[1] = bf16_hi(w.x); o[2] = bf16_lo(w.y); o[3] = bf16_hi(w.y);
+  o[4] = bf16_lo(w.z); o[5] = bf16_hi(w.z); o[6] = bf16_lo(w.w); o[7] = bf16_hi(w.w);
+}
+
+template <int D, int MODE>
+__device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, float* cols,
+                            int n_items, volatile int* abort_flag, int warp, int lane) {
+  using C = BCfg<D>;
+  const int quarter = warp & 3;
+  const int r = quarter * 32 + lane;            // outer row of this thread inside its tile
+  const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+  const uint32_t t_s = t_lane + C::TMEM_S, t_p = t_lane + C::TMEM_P;
+  const uint32_t t_a0 = t_lane + C::TMEM_A0, t_a1 = t_lane + C::TMEM_A1;
+  const float sl2 = a.scale_log2;
+  const int64_t T = a.T;
+  uint32_t sp_seen = 0, acc_seen = 0, cols_n = 0;
+  bool ok = true;
+  for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
+    const int4 raw = a.items[it];
+    const int nu = unit_count<MODE>(raw);
+    for (int t = 0; ok && t < nu; ++t) {
+      const Unit u = decode_unit<MODE>(raw, t);
+      const bool row_ok = r < u.orows;
+      const int64_t row = (int64_t)u.orow0 + (row_ok ? r : 0);
+      const int seg = row_ok ? (int)a.seg[row] : 0;
+      const size_t base = ((size_t)row * (size_t)a.H + (size_t)u.h) * D;
+      const size_t stat = (size_t)u.h * (size_t)T + (size_t)row;
+      // dQ: this row's statistics; dKV: whether this key row is a segment-1 key.
+      const float lse2 = (MODE == kModeDQ && row_ok) ? a.lse2[stat] : INFINITY;
+      const float dsum = (MODE == kModeDQ && row_ok) ? a.dsum[stat] : 0.f;
+      const bool kvalid = MODE == kModeDKV && row_ok && seg == 1;
+      for (int i = 0; i < u.n_in; ++i) {
+        const int valid = min(kTileN, u.in_len - i * kTileN);
+        const int nchunks = (valid + 31) >> 5;
+        float* cl = cols + (cols_n & 1) * 2 * kTileN;   // dKV: this inner tile's column stats
+        if (MODE == kModeDKV) {
+          // Column statistics of the query tile (+inf / 0 past the user's rows, so that those
+          // columns get P = 0), shared through shared memory: thread r fills column r.
+          const int64_t qrow = (int64_t)u.in_lo + (int64_t)i * kTileN + r;
+          const size_t qs = (size_t)u.h * (size_t)T + (size_t)qrow;
+          cl[r] = r < valid ? a.lse2[qs] : INFINITY;
+          cl[kTileN + r] = r < valid ? a.dsum[qs] : 0.f;
+          mbar_arrive(bars + 8 * (C::B_COLS + (cols_n & 1)));
+          ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_COLS + (cols_n & 1)),
+                                                 (cols_n >> 1) & 1, abort_flag, a.status));
+          ++cols_n;
+          if (!ok) break;
+        }
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bars + 8 * C::B_SPFULL, sp_seen & 1, abort_flag, a.status));
+        if (!ok) break;
+        ++sp_seen;
+        tc_fence_after();
+        uint32_t bits[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+        if (MODE == kModeDQ && (valid < kTileN || u.holes)) {
+          // Key columns past the interval or on padding holes are masked (one ballot per 32).
+          const int8_t* kseg = u.holes ? a.seg + (u.in_lo + i * kTileN) : nullptr;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int c = 32 * k + lane;
+            bool keep = c < valid;
+            if (keep && kseg != nullptr) keep = kseg[c] == 1;
+            bits[k] = __ballot_sync(0xffffffffu, keep);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          if (c >= nchunks) break;
+          uint32_t sv[32], dp[32];
+          tmem_ld_x32(t_s + 32 * c, sv);
+          tmem_ld_x32(t_p + 32 * c, dp);
+          tmem_wait_ld();
+          reg_fence16(sv);
+          reg_fence16(sv + 16);
+          reg_fence16(dp);
+          reg_fence16(dp + 16);
+          uint32_t pk_ds[16], pk_p[16];
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            float p0, p1, d0, d1;
+            if (MODE == kModeDQ) {
+              const bool k0 = (bits[c] >> j) & 1u, k1 = (bits[c] >> (j + 1)) & 1u;
+              p0 = k0 ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -lse2)) : 0.f;
+              p1 = k1 ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -lse2)) : 0.f;
+              d0 = dsum;
+              d1 = dsum;
+            } else {
+              const float l0 = cl[32 * c + j], l1 = cl[32 * c + j + 1];
+              d0 = cl[kTileN + 32 * c + j];
+              d1 = cl[kTileN + 32 * c + j + 1];
+              p0 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -l0)) : 0.f;
+              p1 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -l1)) : 0.f;
+            }
+            const float ds0 = p0 * (__uint_as_float(dp[j]) - d0);
+            const float ds1 = p1 * (__uint_as_float(dp[j + 1]) - d1);
+            pk_ds[j / 2] = pack_bf16x2(ds0, ds1);
+            pk_p[j / 2] = pack_bf16x2(p0, p1);
+          }
+          tmem_st_x16(t_p + 16 * c, pk_ds);
+          if (MODE == kModeDKV) tmem_st_x16(t_s + 16 * c, pk_p);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bars + 8 * C::B_DSFULL);
+      }
+      if (!ok) break;
+
+      // ---- epilogue ----
+      const bool has_acc = u.n_in > 0;
+      if (has_acc) {
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bars + 8 * C::B_ACCFULL, acc_seen & 1, abort_flag, a.status));
+        if (!ok) break;
+        ++acc_seen;
+        tc_fence_after();
+      }
+      constexpr int CW = D < 32 ? D : 32;
+      if (MODE == kModeDKV) {
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += CW) {
+          uint32_t dvv[CW], dkv[CW];
+          if constexpr (CW == 32) {
+            tmem_ld_x32(t_a0 + c0, dvv);
+            tmem_ld_x32(t_a1 + c0, dkv);
+          } else {
+            tmem_ld_x16(t_a0 + c0, dvv);
+            tmem_ld_x16(t_a1 + c0, dkv);
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < CW; x += 16) {
+            reg_fence16(dvv + x);
+            reg_fence16(dkv + x);
+          }
+          if (c0 + CW >= D) {
+            tc_fence_before();
+            mbar_arrive(bars + 8 * C::B_ACCFREE);
+          }
+          if (!kvalid) continue;
+#pragma unroll
+          for (int x = 0; x < CW; x += 8) {
+            float ov[8], ok8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              ov[e] = __uint_as_float(dvv[x + e]);
+              ok8[e] = __uint_as_float(dkv[x + e]) * a.scale;
+            }
+            store_row8(a.dv, a.grad_fp32, base + c0 + x, ov);
+            store_row8(a.dk, a.grad_fp32, base + c0 + x, ok8);
+          }
+        }
+      } else {
+        // Diagonal term of a candidate row: its score against its own key, P_ii from the
+        // forward's log-sum-exp, dS_ii = P_ii (dO_i . v_i - D_i).
+        float pd = 0.f, dsd = 0.f;
+        if (row_ok && seg == -1) {
+          const float sd = row_dot<D>(a.q + base, a.k + base) * sl2;
+          pd = fast_exp2(sd - lse2);
+          dsd = pd * (row_dot<D>(a.dout + base, a.v + base) - dsum);
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += CW) {
+          uint32_t acc[CW];
+          if (has_acc) {
+            if constexpr (CW == 32) tmem_ld_x32(t_a0 + c0, acc);
+            else tmem_ld_x16(t_a0 + c0, acc);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < CW; x += 16) reg_fence16(acc + x);
+            if (c0 + CW >= D) {
+              tc_fence_before();
+              mbar_arrive(bars + 8 * C::B_ACCFREE);
+            }
+          } else {
+#pragma unroll
+            for (int x = 0; x < CW; ++x) acc[x] = 0u;
+          }
+          if (!row_ok) continue;
+#pragma unroll
+          for (int x = 0; x < CW; x += 8) {
+            float kv8[8], o[8];
+            unpack8(ld_global_nc_v4(a.k + base + c0 + x), kv8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              o[e] = a.scale * fmaf(dsd, kv8[e], __uint_as_float(acc[x + e]));
+            store_row8(a.dq, a.grad_fp32, base + c0 + x, o);
+            if (seg != 1) {
+              // Candidate rows: their key and value are seen by themselves only. Padding rows:
+              // pd = dsd = 0, so their gradients are written as 0.
+              float qv8[8], dov8[8], dk8[8], dv8[8];
+              unpack8(ld_global_nc_v4(a.q + base + c0 + x), qv8);
+              unpack8(ld_global_nc_v4(a.dout + base + c0 + x), dov8);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                dk8[e] = a.scale * dsd * qv8[e];
+                dv8[e] = pd * dov8[e];
+              }
+              store_row8(a.dk, a.grad_fp32, base + c0 + x, dk8);
+              store_row8(a.dv, a.grad_fp32, base + c0 + x, dv8);
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Kernel
+// ------------------------------------------------------------------------------------------
+template <int D, int MODE>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    jagged_attn_bwd_kernel(const __grid_constant__ CUtensorMap tmO1,
+                           const __grid_constant__ CUtensorMap tmO2,
+                           const __grid_constant__ CUtensorMap tmI1,
+                           const __grid_constant__ CUtensorMap tmI2, const BwdArgs a) {
+  using C = BCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  const uint32_t bars = sbase + C::OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* skip = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    *skip = *a.status != 0;
+    mbar_init(bars + 8 * C::B_OUTFULL, 1);
+    mbar_init(bars + 8 * C::B_OUTEMPTY, 1);
+    for (int i = 0; i < kBwdStages; ++i) {
+      mbar_init(bars + 8 * (C::B_INFULL + i), 1);
+      mbar_init(bars + 8 * (C::B_INEMPTY + i), 1);
+    }
+    mbar_init(bars + 8 * C::B_SPFULL, 1);
+    mbar_init(bars + 8 * C::B_DSFULL, kBwdCompute);
+    mbar_init(bars + 8 * C::B_ACCFULL, 1);
+    mbar_init(bars + 8 * C::B_ACCFREE, kBwdCompute);
+    mbar_init(bars + 8 * (C::B_COLS + 0), kBwdCompute);
+    mbar_init(bars + 8 * (C::B_COLS + 1), kBwdCompute);
+    mbar_init(bars + 8 * C::B_DRAIN, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmO1);
+    tma_prefetch_map(&tmO2);
+    tma_prefetch_map(&tmI1);
+    tma_prefetch_map(&tmI2);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int n_items = *a.n_items;
+  if (!*skip) {
+    if (warp == 0) {
+      if (lane == 0)
+        bwd_producer<D, MODE>(&tmO1, &tmO2, &tmI1, &tmI2, a, sbase, bars, n_items, abort_flag);
+    } else if (warp == 1) {
+      if (lane == 0) bwd_mma<D, MODE>(a, sbase, bars, tmem, n_items, abort_flag);
+    } else {
+      bwd_compute<D, MODE>(a, bars, tmem, reinterpret_cast<float*>(smem + C::OFF_COLS), n_items,
+                           abort_flag, warp, lane);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Per-row statistics: lse2 = lse * log2(e) (+inf for a row with no key) and D = rowsum(dO * O),
+// both transposed to [H][T] so that a tile's 128 consecutive rows of one head are contiguous.
+// ------------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ out, int out_fp32,
+                                                       const bf16* __restrict__ dout,
+                                                       const float* __restrict__ lse, int64_t T,
+                                                       int H, float* __restrict__ lse2,
+                                                       float* __restrict__ dsum,
+                                                       const int32_t* status) {
+  if (*status != 0) return;
+  const int64_t n = T * H;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < n;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = idx / H;
+    const int h = (int)(idx - row * H);
+    const size_t base = (size_t)idx * D;
+    const uint4* dp = reinterpret_cast<const uint4*>(dout + base);
+    float acc = 0.f;
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c) {
+      float g[8], o[8];
+      unpack8(ld_global_nc_v4(dp + c), g);
+      if (out_fp32) {
+        const float4* op = reinterpret_cast<const float4*>(static_cast<const float*>(out) + base);
+        const float4 a0 = op[2 * c], a1 = op[2 * c + 1];
+        o[0] = a0.x; o[1] = a0.y; o[2] = a0.z; o[3] = a0.w;
+        o[4] = a1.x; o[5] = a1.y; o[6] = a1.z; o[7] = a1.w;
+      } else {
+        unpack8(ld_global_nc_v4(reinterpret_cast<const uint4*>(static_cast<const bf16*>(out) +
+                                                               base) + c), o);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc = fmaf(g[e], o[e], acc);
+    }
+    const float l = lse[idx];
+    lse2[(size_t)h * T + row] = l == -INFINITY ? INFINITY : l * 1.4426950408889634f;
+    dsum[(size_t)h * T + row] = acc;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Work queue of the dKV kernel: one item per (user, head, 128-key tile of the history interval),
+// sorted by the number of the user's 128-row query tiles, largest first (counting sort in one
+// block, as the forward's queue). Item = {first key row, (h << 9) | key rows, row start, row
+// length}.
+// ------------------------------------------------------------------------------------------
+template <typename IdxT>
+__global__ void __launch_bounds__(1024) dkv_queue_kernel(const IdxT* __restrict__ off,
+                                                         const IdxT* __restrict__ hlo,
+                                                         const IdxT* __restrict__ hhi, int64_t B,
+                                                         int H, int4* __restrict__ items,
+                                                         int64_t max_items, int32_t* n_items,
+                                                         int32_t* status) {
+  __shared__ unsigned long long s_cnt[kQueueBuckets];
+  __shared__ unsigned long long s_cursor[kQueueBuckets];
+  __shared__ unsigned long long s_warp[32];
+  __shared__ unsigned long long s_total;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (*status != 0) {
+    if (tid == 0) *n_items = 0;
+    return;
+  }
+  for (int i = tid; i < kQueueBuckets; i += blockDim.x) s_cnt[i] = 0;
+  __syncthreads();
+  for (int64_t b = tid; b < B; b += blockDim.x) {
+    const long long nk = ((long long)hhi[b] - (long long)hlo[b] + kTileN - 1) / kTileN;
+    const long long nq = ((long long)off[b + 1] - (long long)off[b] + kTileM - 1) / kTileM;
+    const int key = (int)min(nq, (long long)(kQueueBuckets - 1));
+    if (nk) atomicAdd(&s_cnt[key], (unsigned long long)(nk * H));
+  }
+  __syncthreads();
+  static_assert(kQueueBuckets == 1024, "scan assumes one bucket per thread");
+  const int kb = kQueueBuckets - 1 - tid;
+  const unsigned long long val = s_cnt[kb];
+  unsigned long long v = val;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    unsigned long long w = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const unsigned long long incl = v + (wid > 0 ? s_warp[wid - 1] : 0ull);
+  s_cursor[kb] = incl - val;
+  if (tid == kQueueBuckets - 1) s_total = incl;
+  __syncthreads();
+  if (s_total > (unsigned long long)max_items) {
+    if (tid == 0) {
+      atomicCAS(status, 0, (int32_t)JCA_STATUS_QUEUE_OVERFLOW);
+      *n_items = 0;
+    }
+    return;
+  }
+  const int nwarps = blockDim.x >> 5;
+  for (int64_t b = wid; b < B; b += nwarps) {
+    const long long lo = (long long)hlo[b], hi = (long long)hhi[b];
+    const long long s = (long long)off[b], e = (long long)off[b + 1];
+    const long long nk = (hi - lo + kTileN - 1) / kTileN;
+    if (nk == 0) continue;
+    const long long nq = (e - s + kTileM - 1) / kTileM;
+    const int key = (int)min(nq, (long long)(kQueueBuckets - 1));
+    unsigned long long pos = 0;
+    if (lane == 0) pos = atomicAdd(&s_cursor[key], (unsigned long long)(nk * H));
+    pos = __shfl_sync(0xffffffffu, pos, 0);
+    for (long long i = lane; i < nk * H; i += 32) {
+      const int h = (int)(i / nk);
+      const long long t = i - (long long)h * nk;
+      const long long k0 = lo + t * kTileN;
+      const int rows = (int)min((long long)kTileN, hi - k0);
+      items[pos + (unsigned long long)i] = make_int4((int)k0, (h << 9) | rows, (int)s, (int)(e - s));
+    }
+  }
+  if (tid == 0) *n_items = (int32_t)s_total;
+}
+
+// ------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn bwd_encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D map over a token-major [rows, H, D] bf16 tensor; box = {swizzle span, 1 head, 128 rows}.
+template <int D>
+bool bwd_map(CUtensorMap* map, const void* base, int64_t rows, int H) {
+  using C = BCfg<D>;
+  EncodeTiledFn enc = bwd_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)C::BOX_X, 1u, (cuuint32_t)C::BM};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle sw = C::SW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : C::SW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_32B;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int kMaxDevices = 64;
+struct BwdDevice {
+  int sms = 0;
+  bool sm100 = false;
+  bool attr_set[4][2] = {};
+};
+BwdDevice g_bwd_dev[kMaxDevices];
+std::mutex g_bwd_mu;
+
+int d_slot(int d) { return d == 16 ? 0 : d == 32 ? 1 : d == 64 ? 2 : 3; }
+
+template <int D, int MODE>
+int launch_bwd_mode(const BwdArgs& a, const void* o1, const void* o2, const void* i1,
+                    const void* i2, int64_t T, cudaStream_t stream) {
+  using C = BCfg<D>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return JCA_ERR_CUDA;
+  BwdDevice* info = &g_bwd_dev[dev];
+  {
+    std::lock_guard<std::mutex> lock(g_bwd_mu);
+    if (info->sms == 0) {
+      int major = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return JCA_ERR_CUDA;
+      info->sm100 = major == 10;
+      info->sms = sms;
+    }
+    if (!info->sm100) return JCA_ERR_DEVICE;
+    if (!info->attr_set[d_slot(D)][MODE]) {
+      if (cudaFuncSetAttribute(jagged_attn_bwd_kernel<D, MODE>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_ALLOC) != cudaSuccess)
+        return JCA_ERR_CUDA;
+      info->attr_set[d_slot(D)][MODE] = true;
+    }
+  }
+  CUtensorMap m1, m2, m3, m4;
+  if (!bwd_map<D>(&m1, o1, T, a.H) || !bwd_map<D>(&m2, o2, T, a.H) ||
+      !bwd_map<D>(&m3, i1, T, a.H) || !bwd_map<D>(&m4, i2, T, a.H))
+    return JCA_ERR_CUDA;
+  jagged_attn_bwd_kernel<D, MODE><<<info->sms, kBwdThreads, C::SMEM_ALLOC, stream>>>(m1, m2, m3,
+                                                                                      m4, a);
+  return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+}
+
+// Workspace of the backward pass: the forward's plan (segment IDs, bounds, dQ work queue), then
+// the dKV queue and the transposed row statistics.
+struct BwdLayout {
+  size_t plan = 0, dkv_items = 0, dkv_n = 0, lse2 = 0, dsum = 0, total = 0;
+  int64_t dkv_max = 0;
+};
+
+BwdLayout bwd_layout(int64_t B, int64_t T, int H) {
+  BwdLayout L;
+  size_t o = align_up(workspace_layout(B, T, H).total, 256);
+  L.plan = 0;
+  L.dkv_max = (T / kTileN + B + 1) * (int64_t)H;
+  L.dkv_items = o;
+  o = align_up(o + 16 * (size_t)L.dkv_max, 256);
+  L.dkv_n = o;
+  o = align_up(o + 16, 256);
+  L.lse2 = o;
+  o = align_up(o + 4 * (size_t)T * H, 256);
+  L.dsum = o;
+  o = align_up(o + 4 * (size_t)T * H, 256);
+  L.total = o;
+  return L;
+}
+
+template <int D>
+int launch_backward(const BwdArgs& base_args, const void* out, int out_fp32, const float* lse,
+                    int64_t T, void* ws, const WorkspaceLayout& W, const BwdLayout& L,
+                    cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
+  const int64_t n = T * base_args.H;
+  const int64_t want = (n + 255) / 256;
+  const int grid = (int)(want < 148 * 16 ? (want > 0 ? want : 1) : 148 * 16);
+  bwd_prep_kernel<D><<<grid, 256, 0, st>>>(out, out_fp32, base_args.dout, lse, T, base_args.H,
+                                           reinterpret_cast<float*>(w + L.lse2),
+                                           reinterpret_cast<float*>(w + L.dsum),
+                                           base_args.status);
+  if (cudaGetLastError() != cudaSuccess) return JCA_ERR_CUDA;
+  BwdArgs a = base_args;
+  a.lse2 = reinterpret_cast<const float*>(w + L.lse2);
+  a.dsum = reinterpret_cast<const float*>(w + L.dsum);
+  // Keys of segment 1: dK, dV.
+  a.items = reinterpret_cast<const int4*>(w + L.dkv_items);
+  a.n_items = reinterpret_cast<const int32_t*>(w + L.dkv_n);
+  int rc = launch_bwd_mode<D, kModeDKV>(a, a.k, a.v, a.q, a.dout, T, st);
+  if (rc) return rc;
+  // Every query: dQ, plus dK, dV of the other rows (candidates' diagonal terms; padding zeros).
+  a.items = reinterpret_cast<const int4*>(w + W.items);
+  a.n_items = reinterpret_cast<const int32_t*>(w + W.n_items);
+  return launch_bwd_mode<D, kModeDQ>(a, a.q, a.dout, a.k, a.v, T, st);
+}
+
+}  // namespace
+}  // namespace jca
+
+using namespace jca;
+
+extern "C" size_t jca_bwd_workspace_bytes(int64_t B, int64_t T, int H, int d_head) {
+  if (B < 0 || T < 0 || H < 1 || !head_dim_ok(d_head)) return 0;
+  return bwd_layout(B, T, H).total;
+}
+
+extern "C" int jagged_cand_attn_bwd(const void* q, const void* k, const void* v, const void* out,
+                                    int out_fp32, const void* dout, const float* lse, void* dq,
+                                    void* dk, void* dv, int grad_fp32, const void* offsets,
+                                    const void* candidate_start, const int8_t* seg, int64_t B,
+                                    int64_t T, int H, int d_head, float scale, int idx_bits,
+                                    void* workspace, size_t workspace_bytes, int32_t* status,
+                                    jca_stream_t stream) {
+  if (idx_bits != 32 && idx_bits != 64) return JCA_ERR_IDX_BITS;
+  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
+  if (B < 0 || T < 0 || H < 1 || H >= 65536 || T >= (int64_t)INT_MAX || B >= (int64_t)INT_MAX ||
+      (B == 0 && T != 0))
+    return JCA_ERR_SHAPE;
+  if (!status || !offsets || !workspace) return JCA_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv))
+    return JCA_ERR_NULL;
+  if (B > 0 && !seg && !candidate_start) return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+                !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+                !aligned(lse, 4)))
+    return JCA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+  const BwdLayout L = bwd_layout(B, T, H);
+  if (workspace_bytes < L.total) return JCA_ERR_WORKSPACE;
+  if (T == 0) return JCA_OK;
+  const WorkspaceLayout W = workspace_layout(B, T, H);
+  int rc = jagged_cand_attn_plan(offsets, candidate_start, seg, B, T, H, d_head, idx_bits,
+                                 workspace, W.total, status, stream);
+  if (rc) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  if (idx_bits == 32)
+    dkv_queue_kernel<int32_t><<<1, kQueueBuckets, 0, st>>>(
+        (const int32_t*)offsets, (const int32_t*)(w + W.hist_lo), (const int32_t*)(w + W.hist_hi),
+        B, H, reinterpret_cast<int4*>(w + L.dkv_items), L.dkv_max,
+        reinterpret_cast<int32_t*>(w + L.dkv_n), status);
+  else
+    dkv_queue_kernel<int64_t><<<1, kQueueBuckets, 0, st>>>(
+        (const int64_t*)offsets, (const int64_t*)(w + W.hist_lo), (const int64_t*)(w + W.hist_hi),
+        B, H, reinterpret_cast<int4*>(w + L.dkv_items), L.dkv_max,
+        reinterpret_cast<int32_t*>(w + L.dkv_n), status);
+  if (cudaGetLastError() != cudaSuccess) return JCA_ERR_CUDA;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
+  BwdArgs a;
+  a.q = static_cast<const bf16*>(q);
+  a.k = static_cast<const bf16*>(k);
+  a.v = static_cast<const bf16*>(v);
+  a.dout = static_cast<const bf16*>(dout);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.seg = seg ? seg : reinterpret_cast<const int8_t*>(w + W.seg);
+  a.lse2 = nullptr;
+  a.dsum = nullptr;
+  a.items = nullptr;
+  a.n_items = nullptr;
+  a.status = status;
+  a.T = T;
+  a.H = H;
+  a.grad_fp32 = grad_fp32 ? 1 : 0;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  switch (d_head) {
+    case 16: return launch_backward<16>(a, out, out_fp32, lse, T, workspace, W, L, st);
+    case 32: return launch_backward<32>(a, out, out_fp32, lse, T, workspace, W, L, st);
+    case 64: return launch_backward<64>(a, out, out_fp32, lse, T, workspace, W, L, st);
+    default: return launch_backward<128>(a, out, out_fp32, lse, T, workspace, W, L, st);
+  }
+}

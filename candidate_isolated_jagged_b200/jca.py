@@ -50,6 +50,13 @@ _SIGNATURES = {
                                    c_i64, c_i32, c_i32, c_f32, c_vp, c_sz, c_vp, c_vp]),
     "jca_rope_positions": (c_i32, [c_vp, c_vp, c_i64, c_i64, c_i64, c_i32, c_vp, c_vp, c_vp]),
     "jca_apply_rope": (c_i32, [c_vp, c_vp, c_vp, c_i64, c_i32, c_i32, c_f32, c_vp]),
+    "jagged_cand_attn_fwd_lse": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp,
+                                         c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp, c_sz,
+                                         c_vp, c_vp]),
+    "jca_bwd_workspace_bytes": (c_sz, [c_i64, c_i64, c_i32, c_i32]),
+    "jagged_cand_attn_bwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
+                                     c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_f32,
+                                     c_i32, c_vp, c_sz, c_vp, c_vp]),
     "jca_stack_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i64, c_i32, c_i32]),
     "jca_stack_fwd": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64,
                               c_i64, c_i32, c_i32, c_f32, c_i64, c_f32, c_i32, c_vp, c_sz, c_vp,
@@ -291,6 +298,51 @@ def jca_apply_rope(x, out, positions, base: float = 10000.0, stream=None) -> int
     T, H, d = x.shape
     return _check(lib().jca_apply_rope(_ptr(x), _ptr(out), _ptr(positions), T, H, d, float(base),
                                        _stream(stream)), "jca_apply_rope")
+
+
+def jagged_cand_attn_fwd_lse(q, k, v, out, lse, offsets, candidate_start=None, seg=None,
+                             scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                             status: Optional[torch.Tensor] = None, stream=None) -> int:
+    """jagged_cand_attn_fwd that also writes lse [T, H] fp32 (log of each row's softmax
+    denominator; -inf for padding rows)."""
+    T, H, d = q.shape
+    B = offsets.numel() - 1
+    if workspace is None:
+        workspace = torch.empty(jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=q.device)
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().jagged_cand_attn_fwd_lse(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(lse), _ptr(offsets),
+        _ptr(candidate_start), _ptr(seg), B, T, H, d, float(scale), _idx_bits(offsets),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
+        "jagged_cand_attn_fwd_lse")
+
+
+def jca_bwd_workspace_bytes(B: int, T: int, H: int, d_head: int) -> int:
+    return int(lib().jca_bwd_workspace_bytes(int(B), int(T), int(H), int(d_head)))
+
+
+def jagged_cand_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, offsets, candidate_start=None,
+                         seg=None, scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                         status: Optional[torch.Tensor] = None, stream=None) -> int:
+    """Gradients dq, dk, dv ([T, H, d], bf16 or fp32 as the tensors given) of the jagged
+    candidate-isolated attention for the upstream gradient dout."""
+    T, H, d = q.shape
+    B = offsets.numel() - 1
+    if workspace is None:
+        workspace = torch.empty(jca_bwd_workspace_bytes(B, T, H, d), dtype=torch.uint8,
+                                device=q.device)
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    grad_fp32 = 1 if dq.dtype == torch.float32 else 0
+    assert dk.dtype == dq.dtype and dv.dtype == dq.dtype
+    return _check(lib().jagged_cand_attn_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+        _ptr(dv), grad_fp32, _ptr(offsets), _ptr(candidate_start), _ptr(seg), B, T, H, d,
+        float(scale), _idx_bits(offsets), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream)), "jagged_cand_attn_bwd")
 
 
 def jca_stack_workspace_bytes(B: int, T: int, Nc: int, Th: int, H: int, d_head: int) -> int:

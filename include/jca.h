@@ -291,6 +291,46 @@ int jca_apply_rope(const void* x, void* out, const int32_t* positions, int64_t T
                    int d_head, float base, jca_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Training: the forward with its log-sum-exp, and the backward pass. The pages train on the same
+ * packed layout they serve (候选隔离注意力掩码, section 训练时的序列打包: several users' sequences
+ * in one packed matrix, split at cu_seqlens = the offsets here), under the same mask.
+ * ------------------------------------------------------------------------------------------- */
+
+/* jagged_cand_attn_fwd that also writes lse [T, H] fp32 (4-byte aligned): per row and head, the
+ * natural log of the row's softmax denominator, log sum_j exp(scale q.k_j) over the keys the mask
+ * lets it see (its own key included for a candidate); -inf for a padding row. The backward pass
+ * rebuilds the probabilities from it. Other arguments and errors as jagged_cand_attn_fwd. */
+int jagged_cand_attn_fwd_lse(const void* q, const void* k, const void* v, void* out, int out_fp32,
+                             float* lse, const void* offsets, const void* candidate_start,
+                             const int8_t* seg, int64_t B, int64_t T, int H, int d_head,
+                             float scale, int idx_bits, void* workspace, size_t workspace_bytes,
+                             int32_t* status, jca_stream_t stream);
+
+/* Workspace bytes of jagged_cand_attn_bwd (0 for invalid sizes). */
+size_t jca_bwd_workspace_bytes(int64_t B, int64_t T, int H, int d_head);
+
+/*
+ * Gradients of jagged_cand_attn_fwd for the upstream gradient dout: per user and head, with P the
+ * forward's probabilities, dV = P^T dO, dS = P * (dO V^T - rowsum(dO * O)), dQ = scale dS K,
+ * dK = scale dS^T Q. Rows of padding get zero gradients; a candidate's own key and value receive
+ * gradient from that candidate only.
+ *   q, k, v, dout [T, H, d_head] bf16, read; out [T, H, d_head] bf16 or fp32 (out_fp32), the
+ *   forward's output, read; lse [T, H] fp32 from jagged_cand_attn_fwd_lse, read.
+ *   dq, dk, dv [T, H, d_head] bf16 or fp32 (grad_fp32), written (every row).
+ *   offsets, candidate_start, seg, B, T, H, d_head, scale, idx_bits: as for the forward (the same
+ *   values the forward was called with).
+ *   workspace >= jca_bwd_workspace_bytes(B, T, H, d_head) bytes, 256-byte aligned.
+ * Device errors: as jagged_cand_attn_fwd (the layout is validated again), plus
+ * JCA_STATUS_QUEUE_OVERFLOW (internal) and JCA_STATUS_TIMEOUT.
+ */
+int jagged_cand_attn_bwd(const void* q, const void* k, const void* v, const void* out, int out_fp32,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                         int grad_fp32, const void* offsets, const void* candidate_start,
+                         const int8_t* seg, int64_t B, int64_t T, int H, int d_head, float scale,
+                         int idx_bits, void* workspace, size_t workspace_bytes, int32_t* status,
+                         jca_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Layer stack with candidate-only tail layers (候选隔离注意力掩码, section 只更新候选的末尾层 and its
  * flowchart): the first n_layers - n_cand_only layers run over whole rows [prefix | history |
  * candidates] under the isolation mask; then the states are split into the frozen history

@@ -20,5 +20,6 @@ from .workloads import (  # noqa: F401
     users256_history_lengths,
     StackBatch,
     custom_stack,
+    upstream_grad,
     stack_users256,
 )

@@ -304,3 +304,10 @@ WORKLOADS = {
 
 def make_workload(name: str):
     return WORKLOADS[name]()
+
+
+def upstream_grad(shape, seed: int) -> torch.Tensor:
+    """A seeded upstream gradient dO for the backward pass: fp32 N(0, 1) from
+    ``torch.Generator().manual_seed(seed)``, cast to bf16."""
+    gen = torch.Generator().manual_seed(int(seed))
+    return torch.randn(*shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)

@@ -134,3 +134,35 @@ def test_stack_host_argument_errors(L):
     assert call(x_out=_addr(0x10004)) == -4
     assert call(ws=_addr(0x40010)) == -4
     assert call(ws_bytes=4096) == -6
+
+
+def test_training_host_argument_errors(L):
+    p = _addr(0x10000)  # never dereferenced: every call below fails its host checks
+    st = _addr(0x20000)
+    ws = _addr(0x40000)
+    assert L.jca_bwd_workspace_bytes(3, 20, 2, 16) >= L.jca_workspace_bytes(3, 20, 2, 16)
+    assert L.jca_bwd_workspace_bytes(3, 20, 2, 24) == 0
+    fargs = [p, p, p, p, 0, p, p, p, None, 3, 20, 2, 16, 0.0, 32, ws, 1 << 20, st, None]
+    assert L.jagged_cand_attn_fwd_lse(*fargs[:5], None, *fargs[6:]) == -1      # lse missing
+    assert L.jagged_cand_attn_fwd_lse(*fargs[:5], _addr(0x10002), *fargs[6:]) == -4
+    names = ["q", "k", "v", "out", "out_fp32", "dout", "lse", "dq", "dk", "dv", "grad_fp32",
+             "off", "cs", "seg", "B", "T", "H", "d", "scale", "idx_bits", "ws", "ws_bytes",
+             "status", "stream"]
+    args = [p, p, p, p, 0, p, p, p, p, p, 1, p, p, None, 3, 20, 2, 16, 0.0, 32, ws, 1 << 20, st,
+            None]
+
+    def call(**kw):
+        a = list(args)
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return L.jagged_cand_attn_bwd(*a)
+
+    assert call(idx_bits=8) == -5
+    assert call(d=48) == -3
+    assert call(H=0) == -2
+    assert call(dout=None) == -1
+    assert call(lse=None) == -1
+    assert call(cs=None) == -1
+    assert call(dk=_addr(0x10008)) == -4
+    assert call(ws=_addr(0x40010)) == -4
+    assert call(ws_bytes=64) == -6
