@@ -24,7 +24,9 @@
 // from TMEM as the A operand:
 //   mode dQ  (O1 = Q, O2 = dO, I1 = K, I2 = V):   acc0 += dS I1
 //   mode dKV (O1 = K, O2 = V, I1 = Q, I2 = dO):   acc0 (dV) += P^T I2,  acc1 (dK) += dS^T I1.
-// TMEM columns: S | dP | acc0 | acc1 (128 each, 512 allocated).
+// Each 128-row inner tile is consumed as two 64-row half steps, so that S and dP fit twice in
+// TMEM: while the compute warps work on half step t, the tensor core computes S and dP of t + 1.
+// TMEM columns: S0 | dP0 | S1 | dP1 (64 each) | acc0 | acc1 (128 each); 512 allocated.
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -47,6 +49,7 @@ constexpr int kModeDKV = 1;
 constexpr int kBwdThreads = 192;     // warp 0 producer, warp 1 MMA, warps 2..5 compute
 constexpr int kBwdCompute = 128;
 constexpr int kBwdStages = 2;        // inner ring depth
+constexpr int kHalf = 64;            // inner rows per half step
 
 struct BwdArgs {
   const bf16* q;
@@ -88,9 +91,12 @@ struct BCfg {
   static constexpr int B_OUTEMPTY = 1;
   static constexpr int B_INFULL = 2;                                  // [kBwdStages]
   static constexpr int B_INEMPTY = B_INFULL + kBwdStages;             // [kBwdStages]
-  static constexpr int B_SPFULL = B_INEMPTY + kBwdStages;             // S and dP written
-  static constexpr int B_DSFULL = B_SPFULL + 1;                       // dS (and P) written back
-  static constexpr int B_ACCFULL = B_DSFULL + 1;                      // unit's last TS MMA done
+  static constexpr int B_SPFULL = B_INEMPTY + kBwdStages;             // [2] S and dP written
+  // [2] dS (and P) of the half step in buffer b written back. One barrier per buffer: with
+  // S/dP of step t + 1 already computed, a warp may finish step t + 1 before another warp
+  // finishes step t, and its arrival must not count toward step t.
+  static constexpr int B_DSFULL = B_SPFULL + 2;
+  static constexpr int B_ACCFULL = B_DSFULL + 2;                      // unit's last TS MMA done
   static constexpr int B_ACCFREE = B_ACCFULL + 1;                     // accumulators read
   static constexpr int B_COLS = B_ACCFREE + 1;                        // [2] column stats (dKV)
   static constexpr int B_DRAIN = B_COLS + 2;
@@ -101,8 +107,9 @@ struct BCfg {
   static constexpr int SMEM_RAW = SMEM_USED + 1024;
   // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
   static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
-  static constexpr uint32_t TMEM_S = 0, TMEM_P = 128, TMEM_A0 = 256, TMEM_A1 = 384,
-                            TMEM_COLS = 512;
+  // Half-step buffer b: S at 128 b, dP at 128 b + 64.
+  static constexpr uint32_t TMEM_S = 0, TMEM_P = 64, TMEM_BUF = 128, TMEM_A0 = 256,
+                            TMEM_A1 = 384, TMEM_COLS = 512;
   static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
 };
 
@@ -220,18 +227,76 @@ __device__ __forceinline__ void bwd_mma_ts(uint32_t acc, uint32_t a_tmem, uint64
               (overwrite && kk == 0) ? 0u : 1u);
 }
 
+// Half steps of a unit: inner tile i is split into rows [0, 64) and [64, 128) of the tile; the
+// second half exists only when the tile holds more than 64 valid rows.
+struct HalfStep {
+  int i, hh, valid;   // inner tile, half (0 / 1), valid rows of the half (1..64)
+};
+
+__device__ __forceinline__ bool next_half(const Unit& u, HalfStep& h) {
+  const int tile_valid = min(kTileN, u.in_len - h.i * kTileN);
+  if (h.hh == 0 && tile_valid > kHalf) {
+    h.hh = 1;
+  } else {
+    if (h.i + 1 >= u.n_in) return false;
+    ++h.i;
+    h.hh = 0;
+  }
+  h.valid = min(kHalf, min(kTileN, u.in_len - h.i * kTileN) - h.hh * kHalf);
+  return true;
+}
+
 template <int D, int MODE>
 __device__ void bwd_mma(const BwdArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
                         int n_items, volatile int* abort_flag) {
   using C = BCfg<D>;
-  constexpr uint32_t kIdescFull = idesc_bf16_f32(C::BM, kTileN, false, false);
-  constexpr uint32_t kIdesc0 = kIdescFull & ~(0x3Fu << 17);
+  constexpr uint32_t kIdescHalf = idesc_bf16_f32(C::BM, kHalf, false, false);
+  constexpr uint32_t kIdesc0 = kIdescHalf & ~(0x3Fu << 17);
+  constexpr uint32_t kHalfRows = (kHalf * C::SW) >> 4;   // descriptor offset of row 64
   const uint64_t o1 = smem_desc(sbase + C::OFF_OUT, 16, 8 * C::SW, C::LAYOUT);
   const uint64_t o2 = o1 + (uint64_t)(C::TILE_BYTES >> 4);
   const uint64_t in_k = smem_desc(sbase + C::OFF_IN, 16, 8 * C::SW, C::LAYOUT);
   const uint64_t in_mn = smem_desc(sbase + C::OFF_IN, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
-  uint32_t u_count = 0, g = 0, ds_seen = 0, acc_units = 0;
+  uint32_t u_count = 0, g = 0, steps = 0, ts_steps = 0, acc_units = 0;
   bool ok = true;
+  // S = O1 I1^T and dP = O2 I2^T of one half step, into TMEM buffer (step & 1).
+  auto issue_sp = [&](const HalfStep& h, uint32_t stage) {
+    const uint32_t idesc =
+        h.valid == kHalf ? kIdescHalf
+                         : (kIdesc0 | ((uint32_t)(((h.valid + 15) & ~15) >> 3) << 17));
+    const uint64_t i1 = in_k + (uint64_t)((stage * 2 * C::TILE_BYTES) >> 4) +
+                        (uint64_t)(h.hh * kHalfRows);
+    const uint64_t i2 = i1 + (uint64_t)(C::TILE_BYTES >> 4);
+    const uint32_t buf = (steps & 1) * C::TMEM_BUF;
+    bwd_mma_ss<D>(tmem + buf + C::TMEM_S, o1, i1, idesc);
+    bwd_mma_ss<D>(tmem + buf + C::TMEM_P, o2, i2, idesc);
+    tc_commit(bars + 8 * (C::B_SPFULL + (int)(steps & 1)));
+    ++steps;
+  };
+  // The TS MMAs of a half step, once the compute warps wrote its dS (and P).
+  auto issue_ts = [&](const HalfStep& h, uint32_t stage, bool first, bool last_half) -> bool {
+    if (!mbar_wait(bars + 8 * (C::B_DSFULL + (int)(ts_steps & 1)), (ts_steps >> 1) & 1,
+                   abort_flag, a.status))
+      return false;
+    const uint32_t buf = (ts_steps & 1) * C::TMEM_BUF;
+    ++ts_steps;
+    if (first && acc_units > 0 &&
+        !mbar_wait(bars + 8 * C::B_ACCFREE, (acc_units - 1) & 1, abort_flag, a.status))
+      return false;
+    tc_fence_after();
+    const int ksteps = (h.valid + 15) >> 4;
+    const uint64_t m1 = in_mn + (uint64_t)((stage * 2 * C::TILE_BYTES) >> 4) +
+                        (uint64_t)(h.hh * kHalfRows);
+    const uint64_t m2 = m1 + (uint64_t)(C::TILE_BYTES >> 4);
+    if (MODE == kModeDQ) {
+      bwd_mma_ts<D>(tmem + C::TMEM_A0, tmem + buf + C::TMEM_P, m1, ksteps, first);
+    } else {
+      bwd_mma_ts<D>(tmem + C::TMEM_A0, tmem + buf + C::TMEM_S, m2, ksteps, first);
+      bwd_mma_ts<D>(tmem + C::TMEM_A1, tmem + buf + C::TMEM_P, m1, ksteps, first);
+    }
+    if (last_half) tc_commit(bars + 8 * (C::B_INEMPTY + (int)stage));
+    return true;
+  };
   for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
     const int4 raw = a.items[it];
     const int nu = unit_count<MODE>(raw);
@@ -241,41 +306,39 @@ __device__ void bwd_mma(const BwdArgs& a, uint32_t sbase, uint32_t bars, uint32_
       ok = mbar_wait(bars + 8 * C::B_OUTFULL, u_count & 1, abort_flag, a.status);
       if (!ok) break;
       ++u_count;
+      // One half step of lookahead: S/dP of step t + 1 are issued before the TS MMAs of step t.
+      HalfStep cur{0, 0, min(kHalf, min(kTileN, u.in_len))};
+      uint32_t cur_stage = g % kBwdStages;
+      ok = mbar_wait(bars + 8 * (C::B_INFULL + (int)cur_stage), (g / kBwdStages) & 1, abort_flag,
+                     a.status);
+      if (!ok) break;
       tc_fence_after();
-      for (int i = 0; i < u.n_in; ++i, ++g) {
-        const int s = (int)(g % kBwdStages);
-        ok = mbar_wait(bars + 8 * (C::B_INFULL + s), (g / kBwdStages) & 1, abort_flag, a.status);
-        if (!ok) break;
-        tc_fence_after();
-        const int valid = min(kTileN, u.in_len - i * kTileN);
-        const uint32_t idesc =
-            valid == kTileN ? kIdescFull
-                            : (kIdesc0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17));
-        const uint64_t i1 = in_k + (uint64_t)((s * 2 * C::TILE_BYTES) >> 4);
-        const uint64_t i2 = i1 + (uint64_t)(C::TILE_BYTES >> 4);
-        bwd_mma_ss<D>(tmem + C::TMEM_S, o1, i1, idesc);
-        bwd_mma_ss<D>(tmem + C::TMEM_P, o2, i2, idesc);
-        tc_commit(bars + 8 * C::B_SPFULL);
-        ok = mbar_wait(bars + 8 * C::B_DSFULL, ds_seen & 1, abort_flag, a.status);
-        if (!ok) break;
-        ++ds_seen;
-        if (i == 0 && acc_units > 0) {
-          ok = mbar_wait(bars + 8 * C::B_ACCFREE, (acc_units - 1) & 1, abort_flag, a.status);
+      issue_sp(cur, cur_stage);
+      bool first = true;
+      for (;;) {
+        HalfStep nxt = cur;
+        const bool more = next_half(u, nxt);
+        uint32_t nxt_stage = cur_stage;
+        if (more && nxt.hh == 0) {
+          ++g;
+          nxt_stage = g % kBwdStages;
+          ok = mbar_wait(bars + 8 * (C::B_INFULL + (int)nxt_stage), (g / kBwdStages) & 1,
+                         abort_flag, a.status);
           if (!ok) break;
+          tc_fence_after();
         }
-        tc_fence_after();
-        const int ksteps = (valid + 15) >> 4;
-        const uint64_t m1 = in_mn + (uint64_t)((s * 2 * C::TILE_BYTES) >> 4);
-        const uint64_t m2 = m1 + (uint64_t)(C::TILE_BYTES >> 4);
-        if (MODE == kModeDQ) {
-          bwd_mma_ts<D>(tmem + C::TMEM_A0, tmem + C::TMEM_P, m1, ksteps, i == 0);
-        } else {
-          bwd_mma_ts<D>(tmem + C::TMEM_A0, tmem + C::TMEM_S, m2, ksteps, i == 0);
-          bwd_mma_ts<D>(tmem + C::TMEM_A1, tmem + C::TMEM_P, m1, ksteps, i == 0);
-        }
-        tc_commit(bars + 8 * (C::B_INEMPTY + s));
+        if (more) issue_sp(nxt, nxt_stage);
+        // The current half closes its inner tile unless the next step is the tile's second half.
+        const bool last_half = !(more && nxt.hh == 1);
+        ok = issue_ts(cur, cur_stage, first, last_half);
+        if (!ok) break;
+        first = false;
+        if (!more) break;
+        cur = nxt;
+        cur_stage = nxt_stage;
       }
       if (!ok) break;
+      ++g;
       tc_commit(bars + 8 * C::B_OUTEMPTY);
       tc_commit(bars + 8 * C::B_ACCFULL);
       ++acc_units;
@@ -357,7 +420,6 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
       const bool kvalid = MODE == kModeDKV && row_ok && seg == 1;
       for (int i = 0; i < u.n_in; ++i) {
         const int valid = min(kTileN, u.in_len - i * kTileN);
-        const int nchunks = (valid + 31) >> 5;
         float* cl = cols + (cols_n & 1) * 2 * kTileN;   // dKV: this inner tile's column stats
         if (MODE == kModeDKV) {
           // Column statistics of the query tile (+inf / 0 past the user's rows, so that those
@@ -372,62 +434,73 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
           ++cols_n;
           if (!ok) break;
         }
-        ok = __all_sync(0xffffffffu,
-                        mbar_wait(bars + 8 * C::B_SPFULL, sp_seen & 1, abort_flag, a.status));
-        if (!ok) break;
-        ++sp_seen;
-        tc_fence_after();
-        uint32_t bits[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-        if (MODE == kModeDQ && (valid < kTileN || u.holes)) {
-          // Key columns past the interval or on padding holes are masked (one ballot per 32).
-          const int8_t* kseg = u.holes ? a.seg + (u.in_lo + i * kTileN) : nullptr;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int hvalid = min(kHalf, valid - hh * kHalf);
+          if (hvalid <= 0) break;
+          const int nchunks = (hvalid + 31) >> 5;
+          const int b = (int)(sp_seen & 1);
+          ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_SPFULL + b),
+                                                 (sp_seen >> 1) & 1, abort_flag, a.status));
+          if (!ok) break;
+          ++sp_seen;
+          tc_fence_after();
+          const uint32_t ts = t_s + b * C::TMEM_BUF, tp = t_p + b * C::TMEM_BUF;
+          uint32_t bits[2] = {0xffffffffu, 0xffffffffu};
+          if (MODE == kModeDQ && (hvalid < kHalf || u.holes)) {
+            // Key columns past the interval or on padding holes are masked (one ballot per 32).
+            const int8_t* kseg =
+                u.holes ? a.seg + (u.in_lo + i * kTileN + hh * kHalf) : nullptr;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int c = 32 * k + lane;
-            bool keep = c < valid;
-            if (keep && kseg != nullptr) keep = kseg[c] == 1;
-            bits[k] = __ballot_sync(0xffffffffu, keep);
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          if (c >= nchunks) break;
-          uint32_t sv[32], dp[32];
-          tmem_ld_x32(t_s + 32 * c, sv);
-          tmem_ld_x32(t_p + 32 * c, dp);
-          tmem_wait_ld();
-          reg_fence16(sv);
-          reg_fence16(sv + 16);
-          reg_fence16(dp);
-          reg_fence16(dp + 16);
-          uint32_t pk_ds[16], pk_p[16];
-#pragma unroll
-          for (int j = 0; j < 32; j += 2) {
-            float p0, p1, d0, d1;
-            if (MODE == kModeDQ) {
-              const bool k0 = (bits[c] >> j) & 1u, k1 = (bits[c] >> (j + 1)) & 1u;
-              p0 = k0 ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -lse2)) : 0.f;
-              p1 = k1 ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -lse2)) : 0.f;
-              d0 = dsum;
-              d1 = dsum;
-            } else {
-              const float l0 = cl[32 * c + j], l1 = cl[32 * c + j + 1];
-              d0 = cl[kTileN + 32 * c + j];
-              d1 = cl[kTileN + 32 * c + j + 1];
-              p0 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -l0)) : 0.f;
-              p1 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -l1)) : 0.f;
+            for (int k = 0; k < 2; ++k) {
+              const int c = 32 * k + lane;
+              bool keep = c < hvalid;
+              if (keep && kseg != nullptr) keep = kseg[c] == 1;
+              bits[k] = __ballot_sync(0xffffffffu, keep);
             }
-            const float ds0 = p0 * (__uint_as_float(dp[j]) - d0);
-            const float ds1 = p1 * (__uint_as_float(dp[j + 1]) - d1);
-            pk_ds[j / 2] = pack_bf16x2(ds0, ds1);
-            pk_p[j / 2] = pack_bf16x2(p0, p1);
           }
-          tmem_st_x16(t_p + 16 * c, pk_ds);
-          if (MODE == kModeDKV) tmem_st_x16(t_s + 16 * c, pk_p);
+          const float* clh = cl + hh * kHalf;
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (c >= nchunks) break;
+            uint32_t sv[32], dp[32];
+            tmem_ld_x32(ts + 32 * c, sv);
+            tmem_ld_x32(tp + 32 * c, dp);
+            tmem_wait_ld();
+            reg_fence16(sv);
+            reg_fence16(sv + 16);
+            reg_fence16(dp);
+            reg_fence16(dp + 16);
+            uint32_t pk_ds[16], pk_p[16];
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              float p0, p1, d0, d1;
+              if (MODE == kModeDQ) {
+                const bool k0 = (bits[c] >> j) & 1u, k1 = (bits[c] >> (j + 1)) & 1u;
+                p0 = k0 ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -lse2)) : 0.f;
+                p1 = k1 ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -lse2)) : 0.f;
+                d0 = dsum;
+                d1 = dsum;
+              } else {
+                const float2 l2 = *reinterpret_cast<const float2*>(clh + 32 * c + j);
+                const float2 dd = *reinterpret_cast<const float2*>(clh + kTileN + 32 * c + j);
+                d0 = dd.x;
+                d1 = dd.y;
+                p0 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -l2.x)) : 0.f;
+                p1 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -l2.y)) : 0.f;
+              }
+              const float ds0 = p0 * (__uint_as_float(dp[j]) - d0);
+              const float ds1 = p1 * (__uint_as_float(dp[j + 1]) - d1);
+              pk_ds[j / 2] = pack_bf16x2(ds0, ds1);
+              pk_p[j / 2] = pack_bf16x2(p0, p1);
+            }
+            tmem_st_x16(tp + 16 * c, pk_ds);
+            if (MODE == kModeDKV) tmem_st_x16(ts + 16 * c, pk_p);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bars + 8 * (C::B_DSFULL + b));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bars + 8 * C::B_DSFULL);
+        if (!ok) break;
       }
       if (!ok) break;
 
@@ -552,19 +625,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     *skip = *a.status != 0;
-    mbar_init(bars + 8 * C::B_OUTFULL, 1);
-    mbar_init(bars + 8 * C::B_OUTEMPTY, 1);
-    for (int i = 0; i < kBwdStages; ++i) {
-      mbar_init(bars + 8 * (C::B_INFULL + i), 1);
-      mbar_init(bars + 8 * (C::B_INEMPTY + i), 1);
+    // Every barrier slot is initialised: the ones the compute warps arrive on count 128
+    // arrivals, all others (TMA transactions, MMA commits) one.
+    for (int i = 0; i < C::NUM_BARS; ++i) {
+      const bool by_compute = i == C::B_DSFULL || i == C::B_DSFULL + 1 || i == C::B_ACCFREE ||
+                              i == C::B_COLS || i == C::B_COLS + 1;
+      mbar_init(bars + 8 * i, by_compute ? kBwdCompute : 1);
     }
-    mbar_init(bars + 8 * C::B_SPFULL, 1);
-    mbar_init(bars + 8 * C::B_DSFULL, kBwdCompute);
-    mbar_init(bars + 8 * C::B_ACCFULL, 1);
-    mbar_init(bars + 8 * C::B_ACCFREE, kBwdCompute);
-    mbar_init(bars + 8 * (C::B_COLS + 0), kBwdCompute);
-    mbar_init(bars + 8 * (C::B_COLS + 1), kBwdCompute);
-    mbar_init(bars + 8 * C::B_DRAIN, 1);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
