@@ -46,8 +46,8 @@ using bf16 = __nv_bfloat16;
 
 constexpr int kModeDQ = 0;
 constexpr int kModeDKV = 1;
-constexpr int kBwdThreads = 192;     // warp 0 producer, warp 1 MMA, warps 2..5 compute
-constexpr int kBwdCompute = 128;
+constexpr int kBwdThreads = 320;     // warp 0 producer, warp 1 MMA, warps 2..9 compute
+constexpr int kBwdCompute = 256;
 constexpr int kBwdStages = 2;        // inner ring depth
 constexpr int kHalf = 64;            // inner rows per half step
 
@@ -216,6 +216,8 @@ __device__ __forceinline__ void bwd_mma_ss(uint32_t d_tmem, uint64_t a, uint64_t
 }
 
 // acc (+)= A[tmem, bf16 pairs, M = 128 lanes x K = 16 ksteps] * B[smem, MN-major, K rows x N = D].
+// The A pairs of a half step sit in two 16-column runs, columns [0, 16) for inner rows 0..31 and
+// [32, 48) for rows 32..63 (one run per compute warp of a lane quarter).
 template <int D>
 __device__ __forceinline__ void bwd_mma_ts(uint32_t acc, uint32_t a_tmem, uint64_t b, int ksteps,
                                            bool overwrite) {
@@ -223,8 +225,8 @@ __device__ __forceinline__ void bwd_mma_ts(uint32_t acc, uint32_t a_tmem, uint64
   constexpr uint32_t kIdesc = idesc_bf16_f32(C::BM, D, false, true);
   constexpr uint32_t kStep = (16 * C::SW) >> 4;
   for (int kk = 0; kk < ksteps; ++kk)
-    tc_mma_ts(acc, a_tmem + (uint32_t)kk * 8u, b + (uint64_t)(kk * kStep), kIdesc,
-              (overwrite && kk == 0) ? 0u : 1u);
+    tc_mma_ts(acc, a_tmem + (uint32_t)(kk >> 1) * 32u + (uint32_t)(kk & 1) * 8u,
+              b + (uint64_t)(kk * kStep), kIdesc, (overwrite && kk == 0) ? 0u : 1u);
 }
 
 // Half steps of a unit: inner tile i is split into rows [0, 64) and [64, 128) of the tile; the
@@ -391,16 +393,47 @@ __device__ __forceinline__ void unpack8(uint4 w, float* o) {
   o[4] = bf16_lo(w.z); o[5] = bf16_hi(w.z); o[6] = bf16_lo(w.w); o[7] = bf16_hi(w.w);
 }
 
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t t, uint32_t* r) {
+  if constexpr (N == 8) {
+    tmem_ld_x8(t, r);
+  } else if constexpr (N == 16) {
+    tmem_ld_x16(t, r);
+  } else {
+    tmem_ld_x32(t, r);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void reg_fence_n(uint32_t* r) {
+  if constexpr (N == 8) {
+    reg_fence8(r);
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; i += 16) reg_fence16(r + i);
+  }
+}
+
+// Compute warps 2..9: warp w serves TMEM lane quarter w % 4 (one outer row per thread) and column
+// half ch = (w - 2) / 4, i.e. 32 of the 64 inner columns of every half step and half of the D
+// columns of the accumulators in the epilogue.
 template <int D, int MODE>
 __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, float* cols,
                             int n_items, volatile int* abort_flag, int warp, int lane) {
   using C = BCfg<D>;
   const int quarter = warp & 3;
+  const int ch = (warp - 2) >> 2;
   const int r = quarter * 32 + lane;            // outer row of this thread inside its tile
   const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-  const uint32_t t_s = t_lane + C::TMEM_S, t_p = t_lane + C::TMEM_P;
-  const uint32_t t_a0 = t_lane + C::TMEM_A0, t_a1 = t_lane + C::TMEM_A1;
+  const uint32_t t_s = t_lane + C::TMEM_S + 32 * ch, t_p = t_lane + C::TMEM_P + 32 * ch;
+  // The bf16 pairs of a chunk go to the first 16 columns of the chunk itself, so that a warp
+  // never writes columns the other warp of its lane quarter still has to read.
+  const uint32_t t_ps = t_s, t_ds = t_p;
+  constexpr int HD = D / 2;                     // accumulator columns of this warp
+  constexpr int CW = HD < 32 ? HD : 32;
+  const uint32_t t_a0 = t_lane + C::TMEM_A0 + ch * HD, t_a1 = t_lane + C::TMEM_A1 + ch * HD;
   const float sl2 = a.scale_log2;
+  const float2 sl2v = make_float2(sl2, sl2);
   const int64_t T = a.T;
   uint32_t sp_seen = 0, acc_seen = 0, cols_n = 0;
   bool ok = true;
@@ -414,21 +447,37 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
       const int seg = row_ok ? (int)a.seg[row] : 0;
       const size_t base = ((size_t)row * (size_t)a.H + (size_t)u.h) * D;
       const size_t stat = (size_t)u.h * (size_t)T + (size_t)row;
-      // dQ: this row's statistics; dKV: whether this key row is a segment-1 key.
+      // dQ: this row's statistics (padding rows: lse2 = +inf, so P = 0). dKV: a key row that is
+      // not a segment-1 key only pollutes its own accumulator row, which is never stored.
       const float lse2 = (MODE == kModeDQ && row_ok) ? a.lse2[stat] : INFINITY;
       const float dsum = (MODE == kModeDQ && row_ok) ? a.dsum[stat] : 0.f;
-      const bool kvalid = MODE == kModeDKV && row_ok && seg == 1;
+      const float2 nlv = make_float2(-lse2, -lse2), ndv = make_float2(-dsum, -dsum);
+      // dQ: the diagonal term of a candidate row (its score against its own key, P_ii from the
+      // forward's log-sum-exp, dS_ii = P_ii (dO_i . v_i - D_i)), computed while the unit's first
+      // tiles load, so that the epilogue can release the accumulator at once.
+      float pd = 0.f, dsd = 0.f;
+      if (MODE == kModeDQ && row_ok && seg == -1) {
+        const float sd = row_dot<D>(a.q + base, a.k + base) * sl2;
+        pd = fast_exp2(sd - lse2);
+        dsd = pd * (row_dot<D>(a.dout + base, a.v + base) - dsum);
+      }
+      // dKV: column statistics of the query tiles (lse2 = +inf, D = 0 past the user's rows, so
+      // that those columns get P = 0), stored negated in shared memory (warps of column half 0
+      // fill -lse2, half 1 -D). The value for tile i + 1 is fetched while tile i is computed.
+      auto col_stat = [&](int i) -> float {
+        const int v = min(kTileN, u.in_len - i * kTileN);
+        if (r >= v) return ch == 0 ? -INFINITY : 0.f;
+        const size_t qs = (size_t)u.h * (size_t)T + (size_t)((int64_t)u.in_lo + i * kTileN + r);
+        return ch == 0 ? -a.lse2[qs] : -a.dsum[qs];
+      };
+      float next_stat = (MODE == kModeDKV && u.n_in > 0) ? col_stat(0) : 0.f;
       for (int i = 0; i < u.n_in; ++i) {
         const int valid = min(kTileN, u.in_len - i * kTileN);
-        float* cl = cols + (cols_n & 1) * 2 * kTileN;   // dKV: this inner tile's column stats
+        float* cl = cols + (cols_n & 1) * 2 * kTileN;   // dKV: -lse2 | -dsum of the 128 columns
         if (MODE == kModeDKV) {
-          // Column statistics of the query tile (+inf / 0 past the user's rows, so that those
-          // columns get P = 0), shared through shared memory: thread r fills column r.
-          const int64_t qrow = (int64_t)u.in_lo + (int64_t)i * kTileN + r;
-          const size_t qs = (size_t)u.h * (size_t)T + (size_t)qrow;
-          cl[r] = r < valid ? a.lse2[qs] : INFINITY;
-          cl[kTileN + r] = r < valid ? a.dsum[qs] : 0.f;
+          cl[ch * kTileN + r] = next_stat;
           mbar_arrive(bars + 8 * (C::B_COLS + (cols_n & 1)));
+          if (i + 1 < u.n_in) next_stat = col_stat(i + 1);
           ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_COLS + (cols_n & 1)),
                                                  (cols_n >> 1) & 1, abort_flag, a.status));
           ++cols_n;
@@ -437,66 +486,57 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
         for (int hh = 0; hh < 2; ++hh) {
           const int hvalid = min(kHalf, valid - hh * kHalf);
           if (hvalid <= 0) break;
-          const int nchunks = (hvalid + 31) >> 5;
           const int b = (int)(sp_seen & 1);
           ok = __all_sync(0xffffffffu, mbar_wait(bars + 8 * (C::B_SPFULL + b),
                                                  (sp_seen >> 1) & 1, abort_flag, a.status));
           if (!ok) break;
           ++sp_seen;
           tc_fence_after();
-          const uint32_t ts = t_s + b * C::TMEM_BUF, tp = t_p + b * C::TMEM_BUF;
-          uint32_t bits[2] = {0xffffffffu, 0xffffffffu};
-          if (MODE == kModeDQ && (hvalid < kHalf || u.holes)) {
-            // Key columns past the interval or on padding holes are masked (one ballot per 32).
-            const int8_t* kseg =
-                u.holes ? a.seg + (u.in_lo + i * kTileN + hh * kHalf) : nullptr;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              const int c = 32 * k + lane;
-              bool keep = c < hvalid;
-              if (keep && kseg != nullptr) keep = kseg[c] == 1;
-              bits[k] = __ballot_sync(0xffffffffu, keep);
-            }
-          }
-          const float* clh = cl + hh * kHalf;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            if (c >= nchunks) break;
+          const int cvalid = hvalid - 32 * ch;          // valid columns of this warp's chunk
+          if (cvalid > 0) {
+            const uint32_t buf = b * C::TMEM_BUF;
             uint32_t sv[32], dp[32];
-            tmem_ld_x32(ts + 32 * c, sv);
-            tmem_ld_x32(tp + 32 * c, dp);
+            tmem_ld_x32(t_s + buf, sv);
+            tmem_ld_x32(t_p + buf, dp);
+            uint32_t bits = 0xffffffffu;
+            if (MODE == kModeDQ && (cvalid < 32 || u.holes)) {
+              // Key columns past the interval or on padding holes are masked.
+              const int c = 32 * ch + lane;
+              bool keep = lane < cvalid;
+              if (keep && u.holes) keep = a.seg[u.in_lo + i * kTileN + hh * kHalf + c] == 1;
+              bits = __ballot_sync(0xffffffffu, keep);
+            }
             tmem_wait_ld();
             reg_fence16(sv);
             reg_fence16(sv + 16);
             reg_fence16(dp);
             reg_fence16(dp + 16);
+            if (MODE == kModeDQ && bits != 0xffffffffu) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sv[j] = ((bits >> j) & 1u) ? sv[j] : 0xff800000u;
+            }
+            const float* cln = cl + hh * kHalf + 32 * ch;
             uint32_t pk_ds[16], pk_p[16];
 #pragma unroll
             for (int j = 0; j < 32; j += 2) {
-              float p0, p1, d0, d1;
-              if (MODE == kModeDQ) {
-                const bool k0 = (bits[c] >> j) & 1u, k1 = (bits[c] >> (j + 1)) & 1u;
-                p0 = k0 ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -lse2)) : 0.f;
-                p1 = k1 ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -lse2)) : 0.f;
-                d0 = dsum;
-                d1 = dsum;
-              } else {
-                const float2 l2 = *reinterpret_cast<const float2*>(clh + 32 * c + j);
-                const float2 dd = *reinterpret_cast<const float2*>(clh + kTileN + 32 * c + j);
-                d0 = dd.x;
-                d1 = dd.y;
-                p0 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j]), sl2, -l2.x)) : 0.f;
-                p1 = kvalid ? fast_exp2(fmaf(__uint_as_float(sv[j + 1]), sl2, -l2.y)) : 0.f;
+              float2 nl = nlv, nd = ndv;
+              if (MODE == kModeDKV) {
+                nl = *reinterpret_cast<const float2*>(cln + j);
+                nd = *reinterpret_cast<const float2*>(cln + kTileN + j);
               }
-              const float ds0 = p0 * (__uint_as_float(dp[j]) - d0);
-              const float ds1 = p1 * (__uint_as_float(dp[j + 1]) - d1);
-              pk_ds[j / 2] = pack_bf16x2(ds0, ds1);
-              pk_p[j / 2] = pack_bf16x2(p0, p1);
+              const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[j]),
+                                                      __uint_as_float(sv[j + 1])), sl2v, nl);
+              const float2 pp = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              const float2 dd = __fadd2_rn(make_float2(__uint_as_float(dp[j]),
+                                                       __uint_as_float(dp[j + 1])), nd);
+              const float2 ds = __fmul2_rn(pp, dd);
+              pk_ds[j / 2] = pack_bf16x2(ds.x, ds.y);
+              if (MODE == kModeDKV) pk_p[j / 2] = pack_bf16x2(pp.x, pp.y);
             }
-            tmem_st_x16(tp + 16 * c, pk_ds);
-            if (MODE == kModeDKV) tmem_st_x16(ts + 16 * c, pk_p);
+            tmem_st_x16(t_ds + buf, pk_ds);
+            if (MODE == kModeDKV) tmem_st_x16(t_ps + buf, pk_p);
+            tmem_wait_st();
           }
-          tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bars + 8 * (C::B_DSFULL + b));
         }
@@ -504,7 +544,7 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
       }
       if (!ok) break;
 
-      // ---- epilogue ----
+      // ---- epilogue: this warp's half of the D accumulator columns ----
       const bool has_acc = u.n_in > 0;
       if (has_acc) {
         ok = __all_sync(0xffffffffu,
@@ -513,25 +553,18 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
         ++acc_seen;
         tc_fence_after();
       }
-      constexpr int CW = D < 32 ? D : 32;
+      const size_t cbase = base + (size_t)(ch * HD);
       if (MODE == kModeDKV) {
+        const bool kvalid = row_ok && seg == 1;
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += CW) {
+        for (int c0 = 0; c0 < HD; c0 += CW) {
           uint32_t dvv[CW], dkv[CW];
-          if constexpr (CW == 32) {
-            tmem_ld_x32(t_a0 + c0, dvv);
-            tmem_ld_x32(t_a1 + c0, dkv);
-          } else {
-            tmem_ld_x16(t_a0 + c0, dvv);
-            tmem_ld_x16(t_a1 + c0, dkv);
-          }
+          tmem_ld_n<CW>(t_a0 + c0, dvv);
+          tmem_ld_n<CW>(t_a1 + c0, dkv);
           tmem_wait_ld();
-#pragma unroll
-          for (int x = 0; x < CW; x += 16) {
-            reg_fence16(dvv + x);
-            reg_fence16(dkv + x);
-          }
-          if (c0 + CW >= D) {
+          reg_fence_n<CW>(dvv);
+          reg_fence_n<CW>(dkv);
+          if (c0 + CW >= HD) {
             tc_fence_before();
             mbar_arrive(bars + 8 * C::B_ACCFREE);
           }
@@ -544,29 +577,19 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
               ov[e] = __uint_as_float(dvv[x + e]);
               ok8[e] = __uint_as_float(dkv[x + e]) * a.scale;
             }
-            store_row8(a.dv, a.grad_fp32, base + c0 + x, ov);
-            store_row8(a.dk, a.grad_fp32, base + c0 + x, ok8);
+            store_row8(a.dv, a.grad_fp32, cbase + c0 + x, ov);
+            store_row8(a.dk, a.grad_fp32, cbase + c0 + x, ok8);
           }
         }
       } else {
-        // Diagonal term of a candidate row: its score against its own key, P_ii from the
-        // forward's log-sum-exp, dS_ii = P_ii (dO_i . v_i - D_i).
-        float pd = 0.f, dsd = 0.f;
-        if (row_ok && seg == -1) {
-          const float sd = row_dot<D>(a.q + base, a.k + base) * sl2;
-          pd = fast_exp2(sd - lse2);
-          dsd = pd * (row_dot<D>(a.dout + base, a.v + base) - dsum);
-        }
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += CW) {
+        for (int c0 = 0; c0 < HD; c0 += CW) {
           uint32_t acc[CW];
           if (has_acc) {
-            if constexpr (CW == 32) tmem_ld_x32(t_a0 + c0, acc);
-            else tmem_ld_x16(t_a0 + c0, acc);
+            tmem_ld_n<CW>(t_a0 + c0, acc);
             tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < CW; x += 16) reg_fence16(acc + x);
-            if (c0 + CW >= D) {
+            reg_fence_n<CW>(acc);
+            if (c0 + CW >= HD) {
               tc_fence_before();
               mbar_arrive(bars + 8 * C::B_ACCFREE);
             }
@@ -578,24 +601,24 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
 #pragma unroll
           for (int x = 0; x < CW; x += 8) {
             float kv8[8], o[8];
-            unpack8(ld_global_nc_v4(a.k + base + c0 + x), kv8);
+            unpack8(ld_global_nc_v4(a.k + cbase + c0 + x), kv8);
 #pragma unroll
             for (int e = 0; e < 8; ++e)
               o[e] = a.scale * fmaf(dsd, kv8[e], __uint_as_float(acc[x + e]));
-            store_row8(a.dq, a.grad_fp32, base + c0 + x, o);
+            store_row8(a.dq, a.grad_fp32, cbase + c0 + x, o);
             if (seg != 1) {
               // Candidate rows: their key and value are seen by themselves only. Padding rows:
               // pd = dsd = 0, so their gradients are written as 0.
               float qv8[8], dov8[8], dk8[8], dv8[8];
-              unpack8(ld_global_nc_v4(a.q + base + c0 + x), qv8);
-              unpack8(ld_global_nc_v4(a.dout + base + c0 + x), dov8);
+              unpack8(ld_global_nc_v4(a.q + cbase + c0 + x), qv8);
+              unpack8(ld_global_nc_v4(a.dout + cbase + c0 + x), dov8);
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 dk8[e] = a.scale * dsd * qv8[e];
                 dv8[e] = pd * dov8[e];
               }
-              store_row8(a.dk, a.grad_fp32, base + c0 + x, dk8);
-              store_row8(a.dv, a.grad_fp32, base + c0 + x, dv8);
+              store_row8(a.dk, a.grad_fp32, cbase + c0 + x, dk8);
+              store_row8(a.dv, a.grad_fp32, cbase + c0 + x, dv8);
             }
           }
         }
@@ -625,8 +648,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     *skip = *a.status != 0;
-    // Every barrier slot is initialised: the ones the compute warps arrive on count 128
-    // arrivals, all others (TMA transactions, MMA commits) one.
+    // Every barrier slot is initialised: the ones the compute warps arrive on count one arrival
+    // per compute thread, all others (TMA transactions, MMA commits) one.
     for (int i = 0; i < C::NUM_BARS; ++i) {
       const bool by_compute = i == C::B_DSFULL || i == C::B_DSFULL + 1 || i == C::B_ACCFREE ||
                               i == C::B_COLS || i == C::B_COLS + 1;
