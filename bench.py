@@ -421,7 +421,12 @@ def run_backward_extras(args, dev, stream, peaks):
     import torch
     import synth
     from candidate_isolated_jagged_b200 import jca, metrics
-    b = synth.users256()
+    n_users = getattr(args, "users", 256)
+    if n_users >= 256:
+        b = synth.users256()
+    else:   # the first n_users users of the same workload (smaller profiling captures)
+        b = synth.custom_batch(synth.users256_history_lengths(0)[:n_users], prefix=4, n_cand=64,
+                               H=8, d=128, seed=0, name="users256_head")
     B, T, H, d = b.B, b.T, b.H, b.d
     pairs = metrics.allowed_pairs_from_counts(b.prefix + b.hist_real, b.n_cand)
     fwd_flops = metrics.effective_flops(pairs, H, d)
@@ -445,10 +450,10 @@ def run_backward_extras(args, dev, stream, peaks):
         jca.jagged_cand_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, off, cs, None,
                                  workspace=wsb, status=st, stream=stream)
 
-    for _ in range(3):
+    for _ in range(max(3, args.warmup)):
         fwd()
         bwd()
-    n = 20
+    n = max(1, min(args.steps, 20))
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
     torch.cuda.synchronize(dev)
     ev[0].record(stream)
@@ -464,7 +469,8 @@ def run_backward_extras(args, dev, stream, peaks):
     b_ms = ev[1].elapsed_time(ev[2]) / n
     bwd_flops = 2.5 * fwd_flops
     res = {
-        "workload": "users256 (T=%d, H=%d, d=%d), dO ~ N(0,1) seed 15, bf16 gradients" % (T, H, d),
+        "workload": "%s (%d users, T=%d, H=%d, d=%d), dO ~ N(0,1) seed 15, bf16 gradients" % (
+            b.name, B, T, H, d),
         "fwd_lse_ms": f_ms, "fwd_lse_effective_tflops": fwd_flops / f_ms / 1e9,
         "bwd_ms": b_ms, "bwd_effective_tflops": bwd_flops / b_ms / 1e9,
         "bwd_pct_of_bf16_peak": 100 * bwd_flops / b_ms / 1e9 / peaks["bf16_tflops"],
@@ -590,6 +596,10 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the candidate-only workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-stride", type=int, default=4)
+    ap.add_argument("--only", choices=["cand_only", "rope", "stack", "backward"], default=None,
+                    help="run one extra section alone on one GPU and print its result (profiling)")
+    ap.add_argument("--users", type=int, default=256,
+                    help="--only backward: use the first N users of the 256-user workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -599,6 +609,15 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank)
+    if args.only is not None:
+        import torch
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        fn = {"cand_only": run_cand_only_extras, "rope": run_rope_extras,
+              "stack": run_stack_extras, "backward": run_backward_extras}[args.only]
+        print(json.dumps({args.only: fn(args, dev, torch.cuda.current_stream(dev), load_peaks())}),
+              flush=True)
+        return 0
     if world > 1:
         import datetime
         import torch
