@@ -351,6 +351,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         line["rope"] = run_rope_extras(args, dev, stream, peaks)
         line["stack"] = run_stack_extras(args, dev, stream, peaks)
         line["backward"] = run_backward_extras(args, dev, stream, peaks)
+        line["causal"] = run_causal_extras(args, dev, stream, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         users = oracle_sample_users(batch, args.cpu_sample_stride, 3)
         fl, tok, times = time_oracle(batch, users, repeats=1)
@@ -408,6 +409,46 @@ def run_rope_extras(args, dev, stream, peaks):
         "launches_timed": 3 * n,
     }
     del q, k
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_causal_extras(args, dev, stream, peaks):
+    """The per-user causal variant on the 256-user row lengths (4 prefix + history + 64
+    candidates per user as one causal sequence each), H = 8, d = 128: queue builder plus attention
+    kernel per call, timed with CUDA events; effective FLOPs = 4 d H per allowed pair,
+    L (L + 1) / 2 pairs per user."""
+    import torch
+    import synth
+    from candidate_isolated_jagged_b200 import jca, metrics
+    n = synth.users256_history_lengths(0)
+    b = synth.custom_batch(n + 68, prefix=0, n_cand=0, H=8, d=128, seed=0, name="users256_causal")
+    B, T, H, d = b.B, b.T, b.H, b.d
+    lengths = b.row_lengths.astype(np.int64)
+    pairs = int((lengths * (lengths + 1) // 2).sum())
+    flops = metrics.effective_flops(pairs, H, d)
+    q, k, v = (t.to(dev) for t in (b.q, b.k, b.v))
+    off = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int64, device=dev)
+    out = torch.empty_like(q)
+    ws = torch.empty(jca.jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=dev)
+    st = jca.new_status(dev)
+    for _ in range(max(3, args.warmup)):
+        jca.jagged_causal_attn_fwd(q, k, v, out, off, workspace=ws, status=st, stream=stream)
+    n_it = max(10, min(args.steps, 100))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(n_it):
+        jca.jagged_causal_attn_fwd(q, k, v, out, off, workspace=ws, status=st, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    jca.check_status(st, "causal")
+    ms = e0.elapsed_time(e1) / n_it
+    res = {"workload": "users256 row lengths as causal sequences (T=%d, H=%d, d=%d)" % (T, H, d),
+           "ms": ms, "effective_tflops": flops / ms / 1e9,
+           "pct_of_bf16_peak": 100 * flops / ms / 1e9 / peaks["bf16_tflops"],
+           "allowed_pairs": pairs, "launches_per_call": 2, "launches_timed": 2 * n_it}
+    del q, k, v, out, ws
     torch.cuda.empty_cache()
     return res
 
@@ -596,7 +637,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the candidate-only workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-stride", type=int, default=4)
-    ap.add_argument("--only", choices=["cand_only", "rope", "stack", "backward"], default=None,
+    ap.add_argument("--only", choices=["cand_only", "rope", "stack", "backward", "causal"],
+                    default=None,
                     help="run one extra section alone on one GPU and print its result (profiling)")
     ap.add_argument("--users", type=int, default=256,
                     help="--only backward: use the first N users of the 256-user workload")
@@ -614,7 +656,8 @@ def main():
         dev = torch.device("cuda", local_rank)
         torch.cuda.set_device(dev)
         fn = {"cand_only": run_cand_only_extras, "rope": run_rope_extras,
-              "stack": run_stack_extras, "backward": run_backward_extras}[args.only]
+              "stack": run_stack_extras, "backward": run_backward_extras,
+              "causal": run_causal_extras}[args.only]
         print(json.dumps({args.only: fn(args, dev, torch.cuda.current_stream(dev), load_peaks())}),
               flush=True)
         return 0

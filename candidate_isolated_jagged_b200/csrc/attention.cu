@@ -58,6 +58,8 @@ struct AttnArgs {
   int out_v8;               // out is 32-byte aligned: rows are written with 32-byte stores
   float scale_log2;         // softmax scale * log2(e)
   float* lse = nullptr;     // [Tq, H] natural-log softmax denominators, or null (not written)
+  int causal = 0;           // per-user causal variant: row i sees the keys j <= i of its user,
+                            // no candidate or padding rows (items come from the causal queue)
 };
 
 // Depth of the shared ring through which every role receives the claimed work items.
@@ -649,7 +651,7 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
       float sd = -INFINITY;
       if (rr < w.nrows) {
         const int row = w.q_row0 + rr;
-        if (!a.q_seg || a.q_seg[row] == -1) {
+        if (!a.causal && (!a.q_seg || a.q_seg[row] == -1)) {
           const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
 #pragma unroll
           for (int c = 0; c < D * 2; c += 128)
@@ -696,14 +698,19 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
     const bool row_ok = row_in_item < w.nrows;
     const int row = w.q_row0 + (row_ok ? row_in_item : 0);
     const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
-    const int seg = row_ok ? (a.q_seg ? (int)a.q_seg[row] : -1) : 0;
+    const int seg = row_ok ? (a.causal ? 1 : (a.q_seg ? (int)a.q_seg[row] : -1)) : 0;
     float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
     for (int j = 0; j < w.n_kv; ++j, ++lt) {
       const int valid = min(C::BN, w.kv_len - j * C::BN);
       const int nchunks = (valid + 31) >> 5;
       // Edge tiles (the trimmed last tile, or any tile of a user with padding holes) are masked
       // column by column; interior tiles take the unmasked path.
-      const bool edge = valid < C::BN || w.holes;
+      // Causal variant: columns past the diagonal of this group's rows are masked; key and query
+      // tiles both start at the user's first row, so the offset is a multiple of the tile size
+      // (a whole tile of this group's rows sees the whole key tile, or none of it, or the lower
+      // triangle of it).
+      const int diag_off = a.causal ? (w.q_row0 + grp * C::BM) - (w.kv_lo + j * C::BN) : C::BN;
+      const bool edge = valid < C::BN || w.holes || diag_off < C::BN - 1;
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bars + 8 * (C::B_SFULL + grp), lt & 1, abort_flag, a.status));
       if (!ok) break;
@@ -733,7 +740,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
         }
 #pragma unroll
         for (int c = 0; c < 128; ++c)
-          x[c] = ((bits[c >> 5] >> (c & 31)) & 1u) ? x[c] : 0xff800000u;   // -inf
+          x[c] = (((bits[c >> 5] >> (c & 31)) & 1u) && c <= r + diag_off) ? x[c] : 0xff800000u;
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
@@ -1168,6 +1175,46 @@ extern "C" int jagged_cand_attn_fwd(const void* q, const void* k, const void* v,
   if (rc) return rc;
   return jagged_cand_attn_run(q, k, v, out, out_fp32, seg, B, T, H, d_head, scale, workspace,
                               workspace_bytes, status, stream);
+}
+
+extern "C" int jagged_causal_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                      int out_fp32, const void* offsets, int64_t B, int64_t T,
+                                      int H, int d_head, float scale, int idx_bits,
+                                      void* workspace, size_t workspace_bytes, int32_t* status,
+                                      jca_stream_t stream) {
+  int rc = check_sizes(idx_bits, d_head, B, T, T, H);
+  if (rc) return rc;
+  if (!status || !offsets) return JCA_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !out)) return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)))
+    return JCA_ERR_ALIGN;
+  rc = check_workspace(workspace, workspace_bytes, B, T, H);
+  if (rc) return rc;
+  const WorkspaceLayout L = workspace_layout(B, T, H);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  if (launch_causal_queue(offsets, B, T, H, idx_bits, reinterpret_cast<int32_t*>(ws + L.items),
+                          L.max_items, reinterpret_cast<int32_t*>(ws + L.n_items), status, st,
+                          reinterpret_cast<int32_t*>(ws + L.queue)) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  if (T == 0) return JCA_OK;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
+  AttnArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.dk = static_cast<const __nv_bfloat16*>(k);
+  a.dv = static_cast<const __nv_bfloat16*>(v);
+  a.q_seg = nullptr;
+  a.kv_seg = nullptr;
+  a.out = out;
+  a.items = reinterpret_cast<const int4*>(ws + L.items);
+  a.n_items = reinterpret_cast<const int32_t*>(ws + L.n_items);
+  a.queue = reinterpret_cast<int32_t*>(ws + L.queue);
+  a.status = status;
+  a.H = H;
+  a.out_fp32 = out_fp32 ? 1 : 0;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.causal = 1;
+  return launch_attention(d_head, a, q, T, k, v, T, st);
 }
 
 extern "C" int cand_only_attn_plan(const void* cand_offsets, const void* hist_offsets,

@@ -307,6 +307,102 @@ __global__ void __launch_bounds__(1024) work_queue_kernel(
   if (tid == 0) *n_items = (int32_t)s_total;
 }
 
+// ---------------------------------------------------------------------------------------------
+// Work queue of the per-user causal variant: one item per (user, head, 256-row query block); the
+// keys of a block are the user's rows up to the block's last row, so the cost (128-key tiles)
+// grows with the block's position. Same counting sort as above, keyed per item.
+// ---------------------------------------------------------------------------------------------
+template <typename IdxT>
+__global__ void __launch_bounds__(1024) causal_queue_kernel(
+    const IdxT* __restrict__ off, int64_t B, int64_t rows, int H, int4* __restrict__ items,
+    int64_t max_items, int32_t* n_items, int32_t* status, int32_t* queue_ctl) {
+  __shared__ unsigned long long s_cnt[kQueueBuckets];
+  __shared__ unsigned long long s_cursor[kQueueBuckets];
+  __shared__ unsigned long long s_warp[32];
+  __shared__ unsigned long long s_total;
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) {
+    queue_ctl[0] = 0;
+    queue_ctl[1] = 0;
+  }
+  if (*status != 0) {
+    if (tid == 0) *n_items = 0;
+    return;
+  }
+  for (int i = tid; i < kQueueBuckets; i += blockDim.x) s_cnt[i] = 0;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  auto key_of = [](long long kv_len) {
+    return (int)min((kv_len + kTileN - 1) / kTileN, (long long)(kQueueBuckets - 1));
+  };
+  for (int64_t b = tid; b < B; b += blockDim.x) {
+    const long long s = (long long)off[b], e = (long long)off[b + 1];
+    if (!row_ok(s, e, b, B, rows)) {
+      s_bad = 1;
+      continue;
+    }
+    for (long long r0 = s; r0 < e; r0 += kItemRows)
+      atomicAdd(&s_cnt[key_of(min(r0 + kItemRows, e) - s)], (unsigned long long)H);
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      set_status(status, JCA_STATUS_BAD_OFFSETS);
+      *n_items = 0;
+    }
+    return;
+  }
+  static_assert(kQueueBuckets == 1024, "scan assumes one bucket per thread");
+  const int kb = kQueueBuckets - 1 - tid;
+  const unsigned long long val = s_cnt[kb];
+  unsigned long long v = val;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) s_warp[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    unsigned long long w = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const unsigned long long incl = v + (wid > 0 ? s_warp[wid - 1] : 0ull);
+  s_cursor[kb] = incl - val;
+  if (tid == kQueueBuckets - 1) s_total = incl;
+  __syncthreads();
+  if (s_total > (unsigned long long)max_items) {
+    if (tid == 0) {
+      set_status(status, JCA_STATUS_QUEUE_OVERFLOW);
+      *n_items = 0;
+    }
+    return;
+  }
+  // One warp per user: per query block, lane 0 claims H slots, the lanes write them (one per head).
+  const int nwarps = blockDim.x >> 5;
+  for (int64_t b = wid; b < B; b += nwarps) {
+    const long long s = (long long)off[b], e = (long long)off[b + 1];
+    for (long long r0 = s; r0 < e; r0 += kItemRows) {
+      const long long kv_len = min(r0 + kItemRows, e) - s;
+      unsigned long long pos = 0;
+      if (lane == 0) pos = atomicAdd(&s_cursor[key_of(kv_len)], (unsigned long long)H);
+      pos = __shfl_sync(0xffffffffu, pos, 0);
+      const int nrows = (int)(min(r0 + kItemRows, e) - r0);
+      for (int h = lane; h < H; h += 32)
+        items[pos + (unsigned long long)h] =
+            make_int4((int)r0, (h << 9) | nrows, (int)s, (int)kv_len);
+    }
+  }
+  if (tid == 0) *n_items = (int32_t)s_total;
+}
+
 inline int grid_for_rows(int64_t B) { return (int)(B < (1 << 20) ? B : (1 << 20)); }
 
 }  // namespace
@@ -381,6 +477,18 @@ cudaError_t launch_bounds(const int8_t* seg, const void* offsets, int64_t B, int
           const_cast<int8_t*>(seg), (const int64_t*)offsets, nullptr, B, T, (int64_t*)hist_lo,
           (int64_t*)hist_hi, (int64_t*)cand_lo, (int64_t*)cand_hi, kv_count, history_only, status);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_causal_queue(const void* offsets, int64_t B, int64_t rows, int H,
+                                int idx_bits, int32_t* items, int64_t max_items, int32_t* n_items,
+                                int32_t* status, cudaStream_t stream, int32_t* queue_ctl) {
+  if (idx_bits == 32)
+    causal_queue_kernel<int32_t><<<1, kQueueBuckets, 0, stream>>>(
+        (const int32_t*)offsets, B, rows, H, (int4*)items, max_items, n_items, status, queue_ctl);
+  else
+    causal_queue_kernel<int64_t><<<1, kQueueBuckets, 0, stream>>>(
+        (const int64_t*)offsets, B, rows, H, (int4*)items, max_items, n_items, status, queue_ctl);
   return cudaGetLastError();
 }
 

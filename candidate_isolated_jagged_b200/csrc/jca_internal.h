@@ -63,4 +63,9 @@ cudaError_t launch_work_queue(const void* q_offsets, const void* kv_lo, const vo
                               int64_t max_items, int32_t* n_items, int32_t* status,
                               cudaStream_t stream, int32_t* queue_ctl = nullptr);
 
+// Work queue of the per-user causal variant (also zeroes the two run-time queue counters).
+cudaError_t launch_causal_queue(const void* offsets, int64_t B, int64_t rows, int H,
+                                int idx_bits, int32_t* items, int64_t max_items, int32_t* n_items,
+                                int32_t* status, cudaStream_t stream, int32_t* queue_ctl);
+
 }  // namespace jca

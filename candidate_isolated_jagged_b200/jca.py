@@ -54,6 +54,8 @@ _SIGNATURES = {
                                          c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp, c_sz,
                                          c_vp, c_vp]),
     "jca_bwd_workspace_bytes": (c_sz, [c_i64, c_i64, c_i32, c_i32]),
+    "jagged_causal_attn_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i64, c_i64, c_i32,
+                                       c_i32, c_f32, c_i32, c_vp, c_sz, c_vp, c_vp]),
     "jagged_cand_attn_bwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_f32,
                                      c_i32, c_vp, c_sz, c_vp, c_vp]),
@@ -317,6 +319,23 @@ def jagged_cand_attn_fwd_lse(q, k, v, out, lse, offsets, candidate_start=None, s
         _ptr(candidate_start), _ptr(seg), B, T, H, d, float(scale), _idx_bits(offsets),
         _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
         "jagged_cand_attn_fwd_lse")
+
+
+def jagged_causal_attn_fwd(q, k, v, out, offsets, scale: float = 0.0,
+                           workspace: Optional[torch.Tensor] = None,
+                           status: Optional[torch.Tensor] = None, stream=None) -> int:
+    """Per-user causal attention over packed sequences (row i sees rows j <= i of its user)."""
+    T, H, d = q.shape
+    B = offsets.numel() - 1
+    if workspace is None:
+        workspace = torch.empty(jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=q.device)
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().jagged_causal_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), B, T, H, d, float(scale),
+        _idx_bits(offsets), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
+        "jagged_causal_attn_fwd")
 
 
 def jca_bwd_workspace_bytes(B: int, T: int, H: int, d_head: int) -> int:

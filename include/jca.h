@@ -291,6 +291,20 @@ int jca_apply_rope(const void* x, void* out, const int32_t* positions, int64_t T
                    int d_head, float base, jca_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Variant: per-user causal attention on the packed layout (prior art on the pages: the early
+ * demo ranker's lower-triangular mask, noted in the FAQ of 候选隔离注意力掩码, and the
+ * block-diagonal causal varlen attention of the contest repository). Row i of user b attends to
+ * rows j <= i of user b; no segment IDs (every row is real).
+ *   q, k, v [T, H, d_head] bf16, read; out [T, H, d_head] bf16 or fp32 (out_fp32), written.
+ *   offsets [B+1] (idx_bits type), read. workspace >= jca_workspace_bytes(B, T, H, d_head).
+ * Device errors: bad offsets -> JCA_STATUS_BAD_OFFSETS (nothing written); JCA_STATUS_TIMEOUT.
+ * ------------------------------------------------------------------------------------------- */
+int jagged_causal_attn_fwd(const void* q, const void* k, const void* v, void* out, int out_fp32,
+                           const void* offsets, int64_t B, int64_t T, int H, int d_head,
+                           float scale, int idx_bits, void* workspace, size_t workspace_bytes,
+                           int32_t* status, jca_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Training: the forward with its log-sum-exp, and the backward pass. The pages train on the same
  * packed layout they serve (候选隔离注意力掩码, section 训练时的序列打包: several users' sequences
  * in one packed matrix, split at cu_seqlens = the offsets here), under the same mask.

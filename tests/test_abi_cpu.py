@@ -26,7 +26,9 @@ def test_header_declares_the_entry_points():
               "jca_build_work_queue", "jca_max_work_items", "jca_workspace_bytes",
               "jagged_cand_attn_fwd", "cand_only_attn_fwd", "jca_status_string",
               "jagged_cand_attn_plan", "jagged_cand_attn_run", "cand_only_attn_plan",
-              "cand_only_attn_run", "jca_stack_workspace_bytes", "jca_stack_fwd"]:
+              "cand_only_attn_run", "jca_stack_workspace_bytes", "jca_stack_fwd",
+              "jagged_cand_attn_fwd_lse", "jca_bwd_workspace_bytes", "jagged_cand_attn_bwd",
+              "jagged_causal_attn_fwd"]:
         assert n in names
 
 
@@ -166,3 +168,16 @@ def test_training_host_argument_errors(L):
     assert call(dk=_addr(0x10008)) == -4
     assert call(ws=_addr(0x40010)) == -4
     assert call(ws_bytes=64) == -6
+
+
+def test_causal_host_argument_errors(L):
+    p = _addr(0x10000)  # never dereferenced: every call below fails its host checks
+    st = _addr(0x20000)
+    ws = _addr(0x40000)
+    args = [p, p, p, p, 0, p, 3, 20, 2, 16, 0.0, 32, ws, 1 << 20, st, None]
+    assert L.jagged_causal_attn_fwd(*args[:11], 8, *args[12:]) == -5         # idx_bits
+    assert L.jagged_causal_attn_fwd(*args[:9], 48, *args[10:]) == -3          # head dim
+    assert L.jagged_causal_attn_fwd(None, *args[1:]) == -1
+    assert L.jagged_causal_attn_fwd(*args[:5], None, *args[6:]) == -1         # offsets
+    assert L.jagged_causal_attn_fwd(*args[:3], _addr(0x10002), *args[4:]) == -4
+    assert L.jagged_causal_attn_fwd(*args[:13], 16, *args[14:]) == -6         # workspace
