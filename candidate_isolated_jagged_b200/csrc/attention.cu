@@ -59,7 +59,8 @@ struct AttnArgs {
   float scale_log2;         // softmax scale * log2(e)
   float* lse = nullptr;     // [Tq, H] natural-log softmax denominators, or null (not written)
   int causal = 0;           // per-user causal variant: row i sees the keys j <= i of its user,
-                            // no candidate or padding rows (items come from the causal queue)
+                            // no candidate or padding rows (items come from the causal queue);
+                            // selects the CAUSAL instantiation of the kernel
 };
 
 // Depth of the shared ring through which every role receives the claimed work items.
@@ -634,7 +635,7 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int s
 // a two-slot shared array; it also starts moving each candidate row's own value towards L2 for
 // the epilogue. Slot s is reused for the item after next once all 256 softmax threads have taken
 // the scores out of it.
-template <int D>
+template <int D, bool CAUSAL>
 __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
                           volatile int* abort_flag, int t, ItemRing ring) {
   using C = Cfg<D>;
@@ -651,7 +652,7 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
       float sd = -INFINITY;
       if (rr < w.nrows) {
         const int row = w.q_row0 + rr;
-        if (!a.causal && (!a.q_seg || a.q_seg[row] == -1)) {
+        if (!CAUSAL && (!a.q_seg || a.q_seg[row] == -1)) {
           const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
 #pragma unroll
           for (int c = 0; c < D * 2; c += 128)
@@ -665,7 +666,7 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
   }
 }
 
-template <int D>
+template <int D, bool CAUSAL>
 __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
                              const float* sd_buf, volatile int* abort_flag, int warp, int lane,
                              ItemRing ring) {
@@ -698,7 +699,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
     const bool row_ok = row_in_item < w.nrows;
     const int row = w.q_row0 + (row_ok ? row_in_item : 0);
     const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
-    const int seg = row_ok ? (a.causal ? 1 : (a.q_seg ? (int)a.q_seg[row] : -1)) : 0;
+    const int seg = row_ok ? (CAUSAL ? 1 : (a.q_seg ? (int)a.q_seg[row] : -1)) : 0;
     float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
     for (int j = 0; j < w.n_kv; ++j, ++lt) {
       const int valid = min(C::BN, w.kv_len - j * C::BN);
@@ -709,8 +710,8 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       // tiles both start at the user's first row, so the offset is a multiple of the tile size
       // (a whole tile of this group's rows sees the whole key tile, or none of it, or the lower
       // triangle of it).
-      const int diag_off = a.causal ? (w.q_row0 + grp * C::BM) - (w.kv_lo + j * C::BN) : C::BN;
-      const bool edge = valid < C::BN || w.holes || diag_off < C::BN - 1;
+      const int diag_off = CAUSAL ? (w.q_row0 + grp * C::BM) - (w.kv_lo + j * C::BN) : C::BN;
+      const bool edge = valid < C::BN || w.holes || (CAUSAL && diag_off < C::BN - 1);
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bars + 8 * (C::B_SFULL + grp), lt & 1, abort_flag, a.status));
       if (!ok) break;
@@ -738,9 +739,15 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
           if (keep && kseg != nullptr) keep = kseg[c] == 1;
           bits[k] = __ballot_sync(0xffffffffu, keep);
         }
+        if (CAUSAL) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          x[c] = (((bits[c >> 5] >> (c & 31)) & 1u) && c <= r + diag_off) ? x[c] : 0xff800000u;
+          for (int c = 0; c < 128; ++c)
+            x[c] = (((bits[c >> 5] >> (c & 31)) & 1u) && c <= r + diag_off) ? x[c] : 0xff800000u;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            x[c] = ((bits[c >> 5] >> (c & 31)) & 1u) ? x[c] : 0xff800000u;   // -inf
+        }
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
@@ -829,7 +836,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
 // ------------------------------------------------------------------------------------------
 // Kernel
 // ------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
     jagged_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -900,10 +907,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       if (lane == 0) mma_role<D>(a, sbase, bars, tmem, abort_flag, ring);
     } else if (warp < 10) {
-      softmax_role<D>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
+      softmax_role<D, CAUSAL>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
                       abort_flag, warp, lane, ring);
     } else {
-      diag_role<D>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), bars, abort_flag,
+      diag_role<D, CAUSAL>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), bars, abort_flag,
                    threadIdx.x - 320, ring);
     }
   }
@@ -995,7 +1002,11 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
     }
     if (!info->sm100) return JCA_ERR_DEVICE;
     if (!info->attr_set[d_index(D)]) {
-      if (cudaFuncSetAttribute(jagged_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      if (cudaFuncSetAttribute(jagged_attn_kernel<D, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_ALLOC) != cudaSuccess ||
+          cudaFuncSetAttribute(jagged_attn_kernel<D, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess)
         return JCA_ERR_CUDA;
       info->attr_set[d_index(D)] = true;
@@ -1007,7 +1018,11 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
     return JCA_ERR_CUDA;
   AttnArgs args = a;
   args.out_v8 = aligned(a.out, 32) ? 1 : 0;
-  jagged_attn_kernel<D><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, args);
+  if (a.causal)
+    jagged_attn_kernel<D, true><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, args);
+  else
+    jagged_attn_kernel<D, false><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV,
+                                                                                  args);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }
 
