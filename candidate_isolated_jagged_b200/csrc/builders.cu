@@ -282,26 +282,26 @@ __global__ void __launch_bounds__(1024) work_queue_kernel(
     }
     return;
   }
-  // Pass 2, one warp per user: lane 0 claims the user's run of nq * H slots, the lanes write it.
-  const int nwarps = blockDim.x >> 5;
-  for (int64_t b = wid; b < B; b += nwarps) {
+  // Pass 2, one thread per user (all users at once, so that the loads of a user's offsets and
+  // bounds are not serialised behind other users'): the thread claims the user's run of nq * H
+  // slots and writes it.
+  for (int64_t b = tid; b < B; b += blockDim.x) {
     const long long s = (long long)qoff[b], e = (long long)qoff[b + 1];
     const long long lo = (long long)kvlo[b], hi = (long long)kvhi[b];
     const long long nq = (e - s + kItemRows - 1) / kItemRows;
     if (nq == 0) continue;
     const long long nkv = (hi - lo + kTileN - 1) / kTileN;
     const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
-    unsigned long long pos = 0;
-    if (lane == 0) pos = atomicAdd(&s_cursor[key], (unsigned long long)(nq * H));
-    pos = __shfl_sync(0xffffffffu, pos, 0);
+    const unsigned long long pos = atomicAdd(&s_cursor[key], (unsigned long long)(nq * H));
     const int holes = (kv_count != nullptr && (long long)kv_count[b] != hi - lo) ? 1 : 0;
     const int w = (int)(hi - lo) | (holes << 31);
-    for (long long i = lane; i < nq * H; i += 32) {
-      const int h = (int)(i / nq);
-      const long long t = i - (long long)h * nq;
-      const long long row0 = s + t * kItemRows;
-      const int rows = (int)min((long long)kItemRows, e - row0);
-      items[pos + (unsigned long long)i] = make_int4((int)row0, (h << 9) | rows, (int)lo, w);
+    for (int h = 0; h < H; ++h) {
+      for (long long t = 0; t < nq; ++t) {
+        const long long row0 = s + t * kItemRows;
+        const int rows = (int)min((long long)kItemRows, e - row0);
+        items[pos + (unsigned long long)(h * nq + t)] =
+            make_int4((int)row0, (h << 9) | rows, (int)lo, w);
+      }
     }
   }
   if (tid == 0) *n_items = (int32_t)s_total;
