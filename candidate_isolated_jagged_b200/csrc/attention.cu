@@ -57,7 +57,8 @@ struct AttnArgs {
   int out_fp32;
   int out_v8;               // out is 32-byte aligned: rows are written with 32-byte stores
   float scale_log2;         // softmax scale * log2(e)
-  float* lse = nullptr;     // [Tq, H] natural-log softmax denominators, or null (not written)
+  float* lse = nullptr;     // [Tq, H] natural-log softmax denominators, or null (not written);
+                            // non-null selects the LSE instantiation of the kernel
   int causal = 0;           // per-user causal variant: row i sees the keys j <= i of its user,
                             // no candidate or padding rows (items come from the causal queue);
                             // selects the CAUSAL instantiation of the kernel
@@ -562,7 +563,7 @@ __device__ __forceinline__ void store16_bf16(const AttnArgs& a, size_t idx, cons
 // value vv were fetched before O_w was complete, so that after it completes only the TMEM reads,
 // the merge, the normalisation and the stores remain: read O_w, release it to the MMA warp, merge
 // the diagonal term of a candidate row, normalise and store.
-template <int D>
+template <int D, bool LSE>
 __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int seg, size_t base,
                                            uint32_t t_o, bool has_o, float m, float l, float sd,
                                            const uint4 (&vv)[D / 8], uint32_t o_free_bar) {
@@ -576,7 +577,7 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int s
   }
   // Padding queries (segment 0) see no key and output 0.
   const float inv = (seg != 0 && l > 0.f) ? 1.f / l : 0.f;
-  if (a.lse != nullptr && row_ok) {
+  if (LSE && row_ok) {
     // log of the row's softmax denominator: l is relative to the reference max (log2 units),
     // which the diagonal merge moved to max(m, sd) for a candidate; -inf for a padding row.
     const float ref = cand ? fmaxf(m, sd) : m;
@@ -666,7 +667,7 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
   }
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool LSE>
 __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
                              const float* sd_buf, volatile int* abort_flag, int warp, int lane,
                              ItemRing ring) {
@@ -829,14 +830,15 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       tc_fence_after();
       ++oi;
     }
-    finish_row<D>(a, row_ok, seg, base, t_o, w.n_kv > 0, m, l, sd, vv, bars + 8 * (C::B_OFREE + grp));
+    finish_row<D, LSE>(a, row_ok, seg, base, t_o, w.n_kv > 0, m, l, sd, vv,
+                       bars + 8 * (C::B_OFREE + grp));
   }
 }
 
 // ------------------------------------------------------------------------------------------
 // Kernel
 // ------------------------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool LSE>
 __global__ void __launch_bounds__(kThreads, 1)
     jagged_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
@@ -907,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
       if (lane == 0) mma_role<D>(a, sbase, bars, tmem, abort_flag, ring);
     } else if (warp < 10) {
-      softmax_role<D, CAUSAL>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
+      softmax_role<D, CAUSAL, LSE>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
                       abort_flag, warp, lane, ring);
     } else {
       diag_role<D, CAUSAL>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), bars, abort_flag,
@@ -1002,10 +1004,13 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
     }
     if (!info->sm100) return JCA_ERR_DEVICE;
     if (!info->attr_set[d_index(D)]) {
-      if (cudaFuncSetAttribute(jagged_attn_kernel<D, false>,
+      if (cudaFuncSetAttribute(jagged_attn_kernel<D, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess ||
-          cudaFuncSetAttribute(jagged_attn_kernel<D, true>,
+          cudaFuncSetAttribute(jagged_attn_kernel<D, true, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_ALLOC) != cudaSuccess ||
+          cudaFuncSetAttribute(jagged_attn_kernel<D, false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess)
         return JCA_ERR_CUDA;
@@ -1018,11 +1023,17 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
     return JCA_ERR_CUDA;
   AttnArgs args = a;
   args.out_v8 = aligned(a.out, 32) ? 1 : 0;
+  // Instantiations: the main path, the causal variant, and the training forward (log-sum-exp
+  // output); each mode is compile-time so that the main path carries none of the others' code.
   if (a.causal)
-    jagged_attn_kernel<D, true><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, args);
+    jagged_attn_kernel<D, true, false><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
+                                                                                        tmV, args);
+  else if (a.lse != nullptr)
+    jagged_attn_kernel<D, false, true><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
+                                                                                        tmV, args);
   else
-    jagged_attn_kernel<D, false><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV,
-                                                                                  args);
+    jagged_attn_kernel<D, false, false><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
+                                                                                         tmV, args);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }
 
