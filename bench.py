@@ -281,37 +281,65 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     value = weak_scaling_value(flops, world, args.steps, elapsed_ms) / 1e12
 
     # ---- end to end through the public API: host inputs in, host output back ----
+    # Every step copies its inputs from pinned host memory and reads its output back. The copies
+    # run on their own streams and the device tensors are double-buffered, so that step i + 1's
+    # inputs cross PCIe while step i computes and step i - 1's output comes back (the link is
+    # full duplex); the timed region spans the first input copy to the last output copy.
     e2e_steps = max(1, min(args.steps, args.e2e_steps))
     pin = lambda t: t.pin_memory()  # noqa: E731
     q_h, k_h, v_h = pin(batch.q), pin(batch.k), pin(batch.v)
     len_h = pin(torch.tensor(batch.row_lengths, dtype=torch.int64))
     cs_h = pin(torch.tensor(batch.cand_start, dtype=torch.int64))
-    out_h = torch.empty(T, H, d, dtype=torch.bfloat16).pin_memory()
+    out_hs = [torch.empty(T, H, d, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h, len_h, cs_h))
-    d2h = out_h.numel() * out_h.element_size()
+    d2h = out_hs[0].numel() * out_hs[0].element_size()
+    bufs = [dict(q=q, k=k, v=v, lengths=lengths, cs=cand_start, off=offsets, out=out, ws=ws)]
+    bufs.append(dict(q=torch.empty_like(q), k=torch.empty_like(k), v=torch.empty_like(v),
+                     lengths=torch.empty_like(lengths), cs=torch.empty_like(cand_start),
+                     off=torch.empty_like(offsets), out=torch.empty_like(out),
+                     ws=torch.empty_like(ws)))
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def e2e_step():
-        q.copy_(q_h, non_blocking=True)
-        k.copy_(k_h, non_blocking=True)
-        v.copy_(v_h, non_blocking=True)
-        lengths.copy_(len_h, non_blocking=True)
-        cand_start.copy_(cs_h, non_blocking=True)
-        step()
-        out_h.copy_(out, non_blocking=True)
+    def e2e_run(n_steps):
+        ev_in = [torch.cuda.Event() for _ in range(n_steps)]
+        ev_c = [torch.cuda.Event() for _ in range(n_steps)]
+        ev_out = [torch.cuda.Event() for _ in range(n_steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(s_in)
+        for i in range(n_steps):
+            b = bufs[i & 1]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_c[i - 2])       # step i - 2 has finished reading b
+                for dst, src in ((b["q"], q_h), (b["k"], k_h), (b["v"], v_h),
+                                 (b["lengths"], len_h), (b["cs"], cs_h)):
+                    dst.copy_(src, non_blocking=True)
+                ev_in[i].record(s_in)
+            stream.wait_event(ev_in[i])
+            if i >= 2:
+                stream.wait_event(ev_out[i - 2])       # b's previous output has been read back
+            jca.jca_offsets_from_lengths(b["lengths"], b["off"], status, stream)
+            jca.jagged_cand_attn_plan(b["off"], b["cs"], None, T, H, d, b["ws"], status, stream)
+            jca.jagged_cand_attn_run(b["q"], b["k"], b["v"], b["out"], None, B, b["ws"], status,
+                                     stream=stream)
+            ev_c[i].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[i])
+                out_hs[i & 1].copy_(b["out"], non_blocking=True)
+                ev_out[i].record(s_out)
+        s_in.wait_stream(s_out)
+        s_in.wait_stream(stream)
+        t1.record(s_in)
+        torch.cuda.synchronize(dev)
+        return t0.elapsed_time(t1)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_run(2)
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    e2e_ms = max_over_ranks([e0.elapsed_time(e1)], dist, dev)[0]
+    e2e_ms = max_over_ranks([e2e_run(e2e_steps)], dist, dev)[0]
     jca.check_status(status, "end-to-end")
+    assert torch.equal(out_hs[(e2e_steps - 1) & 1], out.cpu()), "end-to-end output differs"
     e2e_value = weak_scaling_value(flops, world, e2e_steps, e2e_ms) / 1e12
 
     achieved = flops / (kernel_ms / 1e3) / 1e12
@@ -344,7 +372,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(),
     }
-    del q_h, k_h, v_h, out_h
+    del q_h, k_h, v_h, out_hs, bufs
 
     if rank == 0 and world == 1 and not args.no_extras:
         line["cand_only"] = run_cand_only_extras(args, dev, stream, peaks)
