@@ -54,11 +54,16 @@ def load_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of the attention kernel's source with comments and blank space removed, so that only a
+    change of the code (not of its comments) invalidates a recorded capture."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "candidate_isolated_jagged_b200", "csrc")
     for name in ("attention.cu", "jca_device.cuh"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

@@ -9,24 +9,28 @@
 // (history x candidate and candidate x other-candidate pairs are skipped wholesale), and the
 // candidate's self term is merged into the online softmax as a diagonal epilogue on CUDA cores.
 //
-// Kernel structure (one persistent CTA per SM, 10 warps). A work item is a block of up to 256 query
+// Kernel structure (one persistent CTA per SM, 12 warps). A work item is a block of up to 256 query
 // rows of one (user, head): two 128-row query tiles A and B that share every K/V tile load.
-//   warp 0      two TMA producer threads: lane 0 loads the item's Q tiles and the K tiles, lane 1
-//               loads the V tiles (2-stage rings each).
-//   warp 1      TMEM allocator and single-thread MMA issuer.
-//   warps 2..9  two softmax warpgroups, one per query tile, one query row per thread (TMEM lane =
-//               row). Each group owns an S buffer in TMEM (P is written back over S as bf16 pairs
-//               and read from there by the PV MMA), an fp32 O accumulator and its rows' running
-//               max / sum, and finalises its own rows (diagonal term, 1/l, store).
-// TMEM columns: S_A | S_B | O_A | O_B (128 each). MMA order per key tile j:
+//   warp 0       two TMA producer threads: lane 0 claims the CTA's items and loads their Q tiles
+//                and the K tiles, lane 1 loads the V tiles (rings of stages).
+//   warp 1       TMEM allocator and single-thread MMA issuer.
+//   warps 2..9   two softmax warpgroups, one per query tile, one query row per thread (TMEM lane =
+//                row). Each group owns an S buffer in TMEM (P is written back over S as bf16 pairs
+//                and read from there by the PV MMA), an fp32 O accumulator and its rows' running
+//                max / sum, and finalises its own rows (diagonal term, 1/l, store).
+//   warps 10..11 diagonal scores of candidate rows, one item ahead of the softmax warps.
+// TMEM columns: S_A | S_B | O_A | O_B (128 each). MMA order per key tile j, one stream over all the
+// CTA's items:
 //   QK_A(j), PV_B(j-1), QK_B(j), PV_A(j)
 // so each group's chain (softmax -> PV -> next QK) is short and the tensor core works for one
 // group while the other runs its softmax. An MMA that overwrites S_w is issued after the PV that
 // reads the P stored there, and MMAs from one thread execute in issue order; a commit fires only
 // when every earlier MMA has completed, so once a group sees S_w full its previous PV into O_w is
 // done and O_w may be rescaled in place.
-// Work items (user, head, 256-row query block) come from the cost-sorted queue; CTA c takes items
-// c, c + grid, c + 2 grid, ... so the longest items start first.
+// Work items (user, head, 256-row query block) come from the cost-sorted queue and are claimed at
+// run time from a global counter, so the longest items start first and a CTA that finishes early
+// takes the next one. The kernel is instantiated per mode: the main path, the per-user causal
+// variant (CAUSAL) and the training forward that also writes each row's log-sum-exp (LSE).
 #include <climits>
 #include <cmath>
 #include <cstdint>
