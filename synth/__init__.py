@@ -22,4 +22,7 @@ from .workloads import (  # noqa: F401
     custom_stack,
     upstream_grad,
     stack_users256,
+    UgBatch,
+    custom_ug,
+    ug_sep16k,
 )

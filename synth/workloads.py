@@ -311,3 +311,65 @@ def upstream_grad(shape, seed: int) -> torch.Tensor:
     ``torch.Generator().manual_seed(seed)``, cast to bf16."""
     gen = torch.Generator().manual_seed(int(seed))
     return torch.randn(*shape, generator=gen, dtype=torch.float32).to(torch.bfloat16)
+
+
+@dataclass
+class UgBatch:
+    """Inputs of UG-Sep's masked cross-attention (UG-Sep page, section 分离残差连接): per sample,
+    T_out query tokens (the Mixup + PFFN output, the first c_u of them U-tokens) attend to T_in
+    key/value tokens (the layer input, the first n_u of them U-tokens).
+
+    q, residual  bf16 [B, T_out, H, d]
+    k, v         bf16 [B, T_in, H, d]
+    """
+
+    name: str
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    residual: Optional[torch.Tensor]
+    c_u: int
+    n_u: int
+    seed: int
+
+    @property
+    def B(self) -> int:
+        return int(self.q.shape[0])
+
+    @property
+    def T_out(self) -> int:
+        return int(self.q.shape[1])
+
+    @property
+    def T_in(self) -> int:
+        return int(self.k.shape[1])
+
+    @property
+    def H(self) -> int:
+        return int(self.q.shape[2])
+
+    @property
+    def d(self) -> int:
+        return int(self.q.shape[3])
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / float(np.sqrt(self.d))
+
+
+def custom_ug(B: int, T_out: int, T_in: int, c_u: int, n_u: int, H: int, d: int, seed: int = 0,
+              residual: bool = True, name: str = "ug_custom") -> UgBatch:
+    """Q, K, V (and the residual) drawn in that order from ``torch.Generator().manual_seed(seed)``,
+    fp32 N(0, 1) cast to bf16."""
+    gen = torch.Generator().manual_seed(int(seed))
+    q = _draw(gen, B * T_out, H, d).reshape(B, T_out, H, d)
+    k = _draw(gen, B * T_in, H, d).reshape(B, T_in, H, d)
+    v = _draw(gen, B * T_in, H, d).reshape(B, T_in, H, d)
+    res = _draw(gen, B * T_out, H, d).reshape(B, T_out, H, d) if residual else None
+    return UgBatch(name, q, k, v, res, int(c_u), int(n_u), int(seed))
+
+
+def ug_sep16k() -> UgBatch:
+    """The separated-residual workload: 16,384 samples (candidates of a ranking batch), a pyramid
+    layer from 32 input tokens (16 U + 16 G) to 16 output tokens (8 U + 8 G), one head of 128."""
+    return custom_ug(16384, 16, 32, 8, 16, 1, 128, seed=11, name="ug_sep16k")
