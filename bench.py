@@ -385,6 +385,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         line["stack"] = run_stack_extras(args, dev, stream, peaks)
         line["backward"] = run_backward_extras(args, dev, stream, peaks)
         line["causal"] = run_causal_extras(args, dev, stream, peaks)
+        line["ug_sep"] = run_ug_extras(args, dev, stream, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         users = oracle_sample_users(batch, args.cpu_sample_stride, 3)
         fl, tok, times = time_oracle(batch, users, repeats=1)
@@ -484,6 +485,50 @@ def run_causal_extras(args, dev, stream, peaks):
     del q, k, v, out, ws
     torch.cuda.empty_cache()
     return res
+
+
+def run_ug_extras(args, dev, stream, peaks):
+    """UG-Sep's masked cross-attention (the separated residual of a pyramid TokenMixer) on 16,384
+    samples: 32 input tokens (16 U + 16 G) to 16 outputs (8 U + 8 G), one head of 128, with the
+    residual added and a bf16 output. One kernel per call, timed with CUDA events over repeated
+    calls; the inputs (about 460 MB) exceed L2. The op is bound by HBM: algorithmic bytes = Q, K,
+    V and the residual read once plus the output written once."""
+    import torch
+    import synth
+    from candidate_isolated_jagged_b200 import jca
+    b = synth.ug_sep16k()
+    B, To, Ti, H, d = b.B, b.T_out, b.T_in, b.H, b.d
+    pairs_per_sample = b.c_u * b.n_u + (To - b.c_u) * Ti
+    flops = 4.0 * d * H * pairs_per_sample * B
+    byts = 2.0 * H * d * B * (3 * To + 2 * Ti)
+    q, k, v, res = (t.to(dev) for t in (b.q, b.k, b.v, b.residual))
+    out = torch.empty_like(q)
+    st = jca.new_status(dev)
+    for _ in range(max(3, args.warmup)):
+        jca.ug_masked_cross_attn_fwd(q, k, v, out, b.c_u, b.n_u, residual=res, status=st,
+                                     stream=stream)
+    n_it = max(10, min(args.steps, 200))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(n_it):
+        jca.ug_masked_cross_attn_fwd(q, k, v, out, b.c_u, b.n_u, residual=res, status=st,
+                                     stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    jca.check_status(st, "ug")
+    ms = e0.elapsed_time(e1) / n_it
+    result = {
+        "workload": "ug_sep16k: B=%d samples, T_in=%d (n=%d U), T_out=%d (c_u=%d U), H=%d, d=%d, "
+                    "residual, bf16 out" % (B, Ti, b.n_u, To, b.c_u, H, d),
+        "ms": ms, "samples_per_s": B / ms * 1e3, "effective_tflops": flops / ms / 1e9,
+        "roofline": {"bound": "hbm", "achieved": byts / ms / 1e6, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": byts / ms / 1e6 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": byts},
+        "launches_timed": n_it}
+    del q, k, v, res, out
+    torch.cuda.empty_cache()
+    return result
 
 
 def run_backward_extras(args, dev, stream, peaks):
@@ -670,7 +715,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="skip the candidate-only workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-stride", type=int, default=4)
-    ap.add_argument("--only", choices=["cand_only", "rope", "stack", "backward", "causal"],
+    ap.add_argument("--only", choices=["cand_only", "rope", "stack", "backward", "causal",
+                                       "ug_sep"],
                     default=None,
                     help="run one extra section alone on one GPU and print its result (profiling)")
     ap.add_argument("--users", type=int, default=256,
@@ -690,7 +736,7 @@ def main():
         torch.cuda.set_device(dev)
         fn = {"cand_only": run_cand_only_extras, "rope": run_rope_extras,
               "stack": run_stack_extras, "backward": run_backward_extras,
-              "causal": run_causal_extras}[args.only]
+              "causal": run_causal_extras, "ug_sep": run_ug_extras}[args.only]
         print(json.dumps({args.only: fn(args, dev, torch.cuda.current_stream(dev), load_peaks())}),
               flush=True)
         return 0

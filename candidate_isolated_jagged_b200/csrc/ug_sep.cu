@@ -1,0 +1,588 @@
+// UG-Sep masked cross-attention (the separated residual) on sm_100a (tcgen05 + TMEM + TMA).
+//
+// What it computes (UG-Sep page, sections 分离残差连接 and UG-Separated Mixup 与 mask): for each
+// sample and head, R = softmax(scale * Q K^T under M_UG) V, where Q holds the sample's T_out output
+// tokens and K, V its T_in input tokens. M_UG keeps the U outputs (the first c_u) from reading the
+// G inputs: output i < c_u attends to inputs j < n_u only, every other output to all T_in inputs.
+// With a residual, Y = residual + R. A U output with n_u = 0 sees no key and yields 0 (+ residual).
+//
+// Design. A sample holds a few dozen tokens, so each input byte feeds only a few FLOPs and the op
+// is bound by HBM. Samples are streamed in packs: P consecutive samples whose P * T_out query rows
+// fit one 128-row MMA tile and whose P * T_in keys fit one key tile of at most 128 (rounded up to
+// 16). Because the samples of a pack are consecutive rows of the packed tensors, each pack is one
+// TMA box of Q, one of K and one of V. One tcgen05 MMA computes the pack's scores; the blocks that
+// pair a query with another sample's keys are computed and ignored (the tensor core has an order
+// of magnitude more throughput than this op needs). The softmax thread of a row reads only its
+// sample's block of S, writes P over S (zeros outside its block) and a second MMA forms O = P V.
+//
+// CTA: one persistent CTA per SM, 10 warps; units (pack, head) in a static stride over the grid.
+//   warp 0      TMA producer (lane 0): Q, K and V of a unit into one of STAGES shared stages
+//   warp 1      TMEM allocator and MMA issuer (lane 0), order QK(0), [QK(i+1), PV(i)] for i = 0..
+//   warps 2-5   softmax + epilogue group 0 (the CTA's even units), one query row per thread
+//   warps 6-9   group 1 (odd units)
+// TMEM columns: S_0 | O_0 | S_1 | O_1 (128 each).
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "jca_device.cuh"
+#include "jca_internal.h"
+
+namespace jca {
+namespace {
+
+struct UgArgs {
+  const __nv_bfloat16* residual;   // [B * T_out, H, D] or null
+  void* out;                       // [B * T_out, H, D] bf16 or fp32
+  int32_t* status;
+  int64_t B;
+  int64_t n_units;                 // packs * H
+  int T_out, T_in, c_u, n_u, H;
+  int per_pack;                    // samples per pack
+  int rows_q;                      // query rows per pack: per_pack * T_out (<= 128)
+  int keys;                        // key rows per pack, rounded up to 16 (<= 128)
+  float scale_log2;
+  int out_fp32;
+  int out_v8;                      // out rows may be written with 32-byte stores
+};
+
+constexpr int kUgThreads = 320;
+constexpr int kUgGroupThreads = 128;
+
+template <int D>
+struct UgCfg {
+  static constexpr int ROW_BYTES = D * 2;
+  static constexpr int SW = ROW_BYTES >= 128 ? 128 : ROW_BYTES;   // swizzle span (bytes)
+  static constexpr int NBLK = ROW_BYTES / SW;                     // column blocks per tile
+  static constexpr int BOX_X = SW / 2;
+  static constexpr int TILE_BYTES = 128 * ROW_BYTES;              // a 128-row tile
+  static constexpr int BLK_BYTES = 128 * SW;
+  static constexpr uint32_t LAYOUT = SW == 128 ? 2u : (SW == 64 ? 4u : 6u);
+  static constexpr int KSTEPS_QK = D / 16;
+  static constexpr int KSTEPS_PER_BLK = SW / 32;
+  static constexpr int STAGE_BYTES = 3 * TILE_BYTES;              // Q | K | V
+  static constexpr int STAGES_FIT = (192 * 1024) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;  // 2, 4, 8, 8 for D = 128..16
+  static constexpr int OFF_Q = 0, OFF_K = TILE_BYTES, OFF_V = 2 * TILE_BYTES;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int B_FULL = 0;                  // [STAGES] a unit's Q, K, V landed
+  static constexpr int B_EMPTY = B_FULL + STAGES;   // [STAGES] the unit's MMAs are done
+  static constexpr int B_SFULL = B_EMPTY + STAGES;  // [group] S written by QK
+  static constexpr int B_PFULL = B_SFULL + 2;       // [group] P written over S
+  static constexpr int B_OFULL = B_PFULL + 2;       // [group] O written by PV
+  static constexpr int B_TFREE = B_OFULL + 2;       // [group] O read: S and O may be reused
+  static constexpr int B_DRAIN = B_TFREE + 2;
+  static constexpr int NUM_BARS = B_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM_USED = OFF_MISC + 16;
+  static constexpr int SMEM_RAW = SMEM_USED + 1024;   // slack for 1 KB alignment
+  // At least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns).
+  static constexpr int SMEM_ALLOC = SMEM_RAW > 120 * 1024 ? SMEM_RAW : 120 * 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static_assert(SMEM_ALLOC <= 227 * 1024, "shared memory budget");
+  static_assert(TILE_BYTES % 1024 == 0, "swizzled tiles start on 1 KB boundaries");
+};
+
+// Units of this CTA under the static stride (unit u = blockIdx.x + i * gridDim.x).
+__device__ __forceinline__ int local_units(int64_t n_units) {
+  const int64_t b = blockIdx.x;
+  return b < n_units ? (int)((n_units - b + gridDim.x - 1) / gridDim.x) : 0;
+}
+
+template <int D>
+__device__ void ug_producer(const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                            const CUtensorMap* tmV, const UgArgs& a, uint32_t sbase,
+                            uint32_t bars, volatile int* abort_flag) {
+  using C = UgCfg<D>;
+  const int n_local = local_units(a.n_units);
+  const uint32_t tx = (uint32_t)(D * 2 * (a.rows_q + 2 * a.keys));
+  int issued = 0;
+  bool ok = true;
+  for (int i = 0; i < n_local; ++i) {
+    const int64_t u = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+    const int64_t pack = u / a.H;
+    const int h = (int)(u - pack * a.H);
+    const int s = i % C::STAGES;
+    ok = mbar_wait(bars + 8 * (C::B_EMPTY + s), ((i / C::STAGES) & 1) ^ 1, abort_flag, a.status);
+    if (!ok) break;
+    const uint32_t full = bars + 8 * (C::B_FULL + s);
+    mbar_arrive_expect_tx(full, tx);
+    ++issued;
+    const int qrow = (int)(pack * a.rows_q);
+    const int krow = (int)(pack * a.per_pack * a.T_in);
+    const uint32_t st = sbase + s * C::STAGE_BYTES;
+#pragma unroll
+    for (int c = 0; c < C::NBLK; ++c) {
+      tma_load_3d(st + C::OFF_Q + c * C::BLK_BYTES, tmQ, full, c * C::BOX_X, h, qrow);
+      tma_load_3d(st + C::OFF_K + c * C::BLK_BYTES, tmK, full, c * C::BOX_X, h, krow);
+      tma_load_3d(st + C::OFF_V + c * C::BLK_BYTES, tmV, full, c * C::BOX_X, h, krow);
+    }
+  }
+  if (!ok) {
+    // Aborting: let the copies already issued land before the CTA exits (load n of a stage
+    // completes phase n of its full barrier).
+    for (int n = issued > C::STAGES ? issued - C::STAGES : 0; n < issued; ++n)
+      mbar_wait_drain(bars + 8 * (C::B_FULL + n % C::STAGES), (n / C::STAGES) & 1);
+  }
+}
+
+template <int D>
+__device__ void ug_mma(const UgArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
+                       volatile int* abort_flag) {
+  using C = UgCfg<D>;
+  const int n_local = local_units(a.n_units);
+  const uint32_t idesc_qk = idesc_bf16_f32(128, a.keys, false, false);
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
+  const uint64_t dq = smem_desc(sbase + C::OFF_Q, 16, 8 * C::SW, C::LAYOUT);
+  const uint64_t dk = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
+  const uint64_t dv = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
+  const int kpv = a.keys >> 4;
+  // S_g = Q K^T of unit i (group g = i & 1), once its operands landed and the group has read the
+  // O of its previous unit (so S_g, where that unit's P lives, and O_g are both free).
+  auto issue_qk = [&](int i) -> bool {
+    const int s = i % C::STAGES, g = i & 1;
+    if (!mbar_wait(bars + 8 * (C::B_FULL + s), (i / C::STAGES) & 1, abort_flag, a.status))
+      return false;
+    if (i >= 2 &&
+        !mbar_wait(bars + 8 * (C::B_TFREE + g), ((i >> 1) - 1) & 1, abort_flag, a.status))
+      return false;
+    tc_fence_after();
+    const uint64_t so = (uint64_t)((s * C::STAGE_BYTES) >> 4);
+#pragma unroll
+    for (int kk = 0; kk < C::KSTEPS_QK; ++kk) {
+      const uint32_t off =
+          ((kk / C::KSTEPS_PER_BLK) * C::BLK_BYTES + (kk % C::KSTEPS_PER_BLK) * 32) >> 4;
+      tc_mma(tmem + (uint32_t)(g * 256), dq + so + off, dk + so + off, idesc_qk,
+             kk > 0 ? 1u : 0u);
+    }
+    tc_commit(bars + 8 * (C::B_SFULL + g));
+    return true;
+  };
+  // O_g = P_g V of unit i; P_g is read from the first keys / 2 columns of S_g (bf16 pairs).
+  auto issue_pv = [&](int i) -> bool {
+    const int s = i % C::STAGES, g = i & 1;
+    if (!mbar_wait(bars + 8 * (C::B_PFULL + g), (i >> 1) & 1, abort_flag, a.status)) return false;
+    tc_fence_after();
+    const uint64_t vb = dv + (uint64_t)((s * C::STAGE_BYTES) >> 4);
+    constexpr uint32_t kStep = (16 * C::SW) >> 4;   // 16 key rows of V per k-step
+    const uint32_t p_tmem = tmem + (uint32_t)(g * 256);
+    const uint32_t o_tmem = p_tmem + 128u;
+    for (int kk = 0; kk < kpv; ++kk)
+      tc_mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u, vb + (uint64_t)(kk * kStep), kIdescPV,
+                kk > 0 ? 1u : 0u);
+    tc_commit(bars + 8 * (C::B_EMPTY + s));
+    tc_commit(bars + 8 * (C::B_OFULL + g));
+    return true;
+  };
+  bool ok = true;
+  if (n_local > 0) ok = issue_qk(0);
+  for (int i = 0; ok && i < n_local; ++i) {
+    if (i + 1 < n_local) ok = issue_qk(i + 1);   // the other group's buffers
+    if (ok) ok = issue_pv(i);
+  }
+  if (!ok) {
+    // Aborting: wait until every MMA this thread issued has completed.
+    tc_commit(bars + 8 * C::B_DRAIN);
+    mbar_wait_drain(bars + 8 * C::B_DRAIN, 0);
+  }
+}
+
+// Writes 8 consecutive output values (bf16 or fp32).
+__device__ __forceinline__ void ug_store8(const UgArgs& a, size_t idx, const float* o) {
+  if (a.out_fp32) {
+    float* op = reinterpret_cast<float*>(a.out) + idx;
+    if (a.out_v8) {
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) w[i] = __float_as_uint(o[i]);
+      st_global_v8(op, w);
+    } else {
+      reinterpret_cast<float4*>(op)[0] = make_float4(o[0], o[1], o[2], o[3]);
+      reinterpret_cast<float4*>(op)[1] = make_float4(o[4], o[5], o[6], o[7]);
+    }
+  } else {
+    reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + idx)[0] =
+        make_uint4(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                   pack_bf16x2(o[6], o[7]));
+  }
+}
+
+__device__ __forceinline__ void ug_store16_bf16(const UgArgs& a, size_t idx, const float* o) {
+  uint32_t w[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w[i] = pack_bf16x2(o[2 * i], o[2 * i + 1]);
+  __nv_bfloat16* op = reinterpret_cast<__nv_bfloat16*>(a.out) + idx;
+  if (a.out_v8) {
+    st_global_v8(op, w);
+  } else {
+    reinterpret_cast<uint4*>(op)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(op)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  }
+}
+
+template <int D>
+__device__ void ug_softmax(const UgArgs& a, uint32_t bars, uint32_t tmem,
+                           volatile int* abort_flag, int warp, int lane) {
+  using C = UgCfg<D>;
+  const int grp = (warp - 2) >> 2;
+  const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
+  const int r = quarter * 32 + lane;            // query row of this thread inside a pack
+  const uint32_t t_s = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(grp * 256);
+  const uint32_t t_o = t_s + 128u;
+  // The row's place in every pack: sample sl of the pack, token ti of the sample. Its keys are
+  // the columns [col0, col0 + ncols) of S: its own sample's block, cut to the U inputs for a U
+  // output.
+  const bool in_pack = r < a.rows_q;
+  const int sl = in_pack ? r / a.T_out : 0;
+  const int ti = in_pack ? r - sl * a.T_out : 0;
+  const int col0 = sl * a.T_in;
+  const int ncols = in_pack ? (ti < a.c_u ? a.n_u : a.T_in) : 0;
+  const int kchunks = (a.keys + 31) >> 5;       // 32-key chunks of P the PV reads
+  const float sl2 = a.scale_log2;
+  const int n_local = local_units(a.n_units);
+  bool ok = true;
+  for (int i = grp; i < n_local; i += 2) {
+    const int64_t u = (int64_t)blockIdx.x + (int64_t)i * gridDim.x;
+    const int64_t pack = u / a.H;
+    const int h = (int)(u - pack * a.H);
+    const int64_t sample = pack * a.per_pack + sl;
+    const bool row_ok = in_pack && sample < a.B;
+    const int nc = row_ok ? ncols : 0;
+    const size_t base =
+        ((size_t)(row_ok ? sample * a.T_out + ti : 0) * (size_t)a.H + (size_t)h) * D;
+    // The residual row starts moving towards L2 while the scores are computed.
+    if (a.residual != nullptr && row_ok) {
+#pragma unroll
+      for (int c = 0; c < D * 2; c += 128)
+        asm volatile("prefetch.global.L2 [%0];" ::"l"(a.residual + base + c / 2));
+    }
+    ok = __all_sync(0xffffffffu,
+                    mbar_wait(bars + 8 * (C::B_SFULL + grp), (i >> 1) & 1, abort_flag, a.status));
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t x[128];
+    tmem_ld_x32(t_s + 0, x);
+    tmem_ld_x32(t_s + 32, x + 32);
+    tmem_ld_x32(t_s + 64, x + 64);
+    tmem_ld_x32(t_s + 96, x + 96);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 128; c += 16) reg_fence16(x + c);
+    // Only the row's own columns [col0, col0 + nc) count; the others are masked to -inf.
+    const int hi = col0 + nc;
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      mx = fmaxf(mx, (c >= col0 && c < hi) ? __uint_as_float(x[c]) : -INFINITY);
+    const float m = mx * sl2;
+    const float neg_m = (nc == 0) ? 0.f : -m;
+    float l = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      if (c >= kchunks) break;
+      uint32_t pk[16];
+      if (col0 < 32 * c + 32 && hi > 32 * c) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int c0 = 32 * c + 2 * k;
+          const float p0 = (c0 >= col0 && c0 < hi)
+                               ? fast_exp2(fmaf(__uint_as_float(x[c0]), sl2, neg_m)) : 0.f;
+          const float p1 = (c0 + 1 >= col0 && c0 + 1 < hi)
+                               ? fast_exp2(fmaf(__uint_as_float(x[c0 + 1]), sl2, neg_m)) : 0.f;
+          acc += p0 + p1;
+          pk[k] = pack_bf16x2(p0, p1);
+        }
+        l += acc;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pk[k] = 0u;
+      }
+      tmem_st_x16(t_s + 16 * c, pk);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bars + 8 * (C::B_PFULL + grp));
+
+    const float inv = l > 0.f ? 1.f / l : 0.f;   // no visible key: R = 0
+    // The residual row is read into registers while the PV runs.
+    uint4 rv[D / 8];
+#pragma unroll
+    for (int c = 0; c < D / 8; ++c)
+      rv[c] = (a.residual != nullptr && row_ok)
+                  ? ld_global_nc_v4(reinterpret_cast<const uint4*>(a.residual + base) + c)
+                  : make_uint4(0u, 0u, 0u, 0u);
+    ok = __all_sync(0xffffffffu,
+                    mbar_wait(bars + 8 * (C::B_OFULL + grp), (i >> 1) & 1, abort_flag, a.status));
+    if (!ok) break;
+    tc_fence_after();
+    constexpr int CW = D < 32 ? D : 32;   // columns per TMEM load
+#pragma unroll
+    for (int c0 = 0; c0 < D; c0 += CW) {
+      uint32_t w[CW];
+      if constexpr (CW == 32) tmem_ld_x32(t_o + c0, w);
+      else tmem_ld_x16(t_o + c0, w);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < CW; k += 16) reg_fence16(w + k);
+      if (c0 + CW >= D) {
+        // O_g has been read: the MMA warp may reuse S_g and O_g for the group's next unit.
+        tc_fence_before();
+        mbar_arrive(bars + 8 * (C::B_TFREE + grp));
+      }
+      if (!row_ok) continue;
+      float o[CW];
+#pragma unroll
+      for (int k = 0; k < CW / 8; ++k) {
+        const uint4 rr = rv[c0 / 8 + k];
+        const uint32_t rw[4] = {rr.x, rr.y, rr.z, rr.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          o[8 * k + 2 * e] = fmaf(__uint_as_float(w[8 * k + 2 * e]), inv, bf16_lo(rw[e]));
+          o[8 * k + 2 * e + 1] = fmaf(__uint_as_float(w[8 * k + 2 * e + 1]), inv, bf16_hi(rw[e]));
+        }
+      }
+      if (a.out_fp32) {
+#pragma unroll
+        for (int k = 0; k < CW; k += 8) ug_store8(a, base + c0 + k, o + k);
+      } else {
+#pragma unroll
+        for (int k = 0; k < CW; k += 16) ug_store16_bf16(a, base + c0 + k, o + k);
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kUgThreads, 1)
+    ug_cross_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
+                         const __grid_constant__ CUtensorMap tmK,
+                         const __grid_constant__ CUtensorMap tmV, const UgArgs a) {
+  using C = UgCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (sbase - raw);
+  const uint32_t bars = sbase + C::OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* skip = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // An error recorded earlier on the stream makes the launch a no-op.
+  if (threadIdx.x == 0) {
+    *skip = *a.status != 0;
+    for (int i = 0; i < C::STAGES; ++i) {
+      mbar_init(bars + 8 * (C::B_FULL + i), 1);
+      mbar_init(bars + 8 * (C::B_EMPTY + i), 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bars + 8 * (C::B_SFULL + g), 1);
+      mbar_init(bars + 8 * (C::B_PFULL + g), kUgGroupThreads);
+      mbar_init(bars + 8 * (C::B_OFULL + g), 1);
+      mbar_init(bars + 8 * (C::B_TFREE + g), kUgGroupThreads);
+    }
+    mbar_init(bars + 8 * C::B_DRAIN, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmQ);
+    tma_prefetch_map(&tmK);
+    tma_prefetch_map(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+    tc_fence_before();
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (!*skip) {
+    if (warp == 0) {
+      if (lane == 0) ug_producer<D>(&tmQ, &tmK, &tmV, a, sbase, bars, abort_flag);
+    } else if (warp == 1) {
+      if (lane == 0) ug_mma<D>(a, sbase, bars, tmem, abort_flag);
+    } else {
+      ug_softmax<D>(a, bars, tmem, abort_flag, warp, lane);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// Degenerate layer without input tokens (T_in = 0): every output sees no key, so Y = residual
+// (or 0). One thread per 8 output values.
+__global__ void ug_no_keys_kernel(const __nv_bfloat16* __restrict__ residual, void* out,
+                                  int out_fp32, int64_t n8, const int32_t* status) {
+  if (*status != 0) return;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 r = residual ? reinterpret_cast<const uint4*>(residual)[i]
+                             : make_uint4(0u, 0u, 0u, 0u);
+    if (out_fp32) {
+      float4* op = reinterpret_cast<float4*>(out) + 2 * i;
+      op[0] = make_float4(bf16_lo(r.x), bf16_hi(r.x), bf16_lo(r.y), bf16_hi(r.y));
+      op[1] = make_float4(bf16_lo(r.z), bf16_hi(r.z), bf16_lo(r.w), bf16_hi(r.w));
+    } else {
+      reinterpret_cast<uint4*>(out)[i] = r;
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Host side
+// ------------------------------------------------------------------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn ug_encode_fn() {
+  static EncodeTiledFn fn = []() -> EncodeTiledFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D map over a token-major [rows, H, D] bf16 tensor; box = {swizzle span, 1 head, box_rows}.
+// Rows past the end read as zeros.
+template <int D>
+bool ug_make_map(CUtensorMap* map, const void* base, int64_t rows, int H, int box_rows) {
+  using C = UgCfg<D>;
+  EncodeTiledFn enc = ug_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  const cuuint32_t box[3] = {(cuuint32_t)C::BOX_X, 1u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapSwizzle sw = C::SW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : C::SW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                              : CU_TENSOR_MAP_SWIZZLE_32B;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct UgDevice {
+  int sms = 0;
+  bool sm100 = false;
+  bool attr_set[4] = {false, false, false, false};
+};
+constexpr int kUgMaxDevices = 64;
+UgDevice g_ug_dev[kUgMaxDevices];
+std::mutex g_ug_mu;
+
+template <int D>
+int launch_ug(const void* q, const void* k, const void* v, UgArgs a, int64_t B, int T_out,
+              int T_in, cudaStream_t stream) {
+  using C = UgCfg<D>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kUgMaxDevices) return JCA_ERR_CUDA;
+  UgDevice* info = &g_ug_dev[dev];
+  const int di = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
+  {
+    std::lock_guard<std::mutex> lock(g_ug_mu);
+    if (info->sms == 0) {
+      int major = 0, sms = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return JCA_ERR_CUDA;
+      info->sm100 = (major == 10);
+      info->sms = sms;
+    }
+    if (!info->sm100) return JCA_ERR_DEVICE;
+    if (!info->attr_set[di]) {
+      if (cudaFuncSetAttribute(ug_cross_attn_kernel<D>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_ALLOC) != cudaSuccess)
+        return JCA_ERR_CUDA;
+      info->attr_set[di] = true;
+    }
+  }
+  CUtensorMap tmQ, tmK, tmV;
+  if (!ug_make_map<D>(&tmQ, q, B * T_out, a.H, a.rows_q) ||
+      !ug_make_map<D>(&tmK, k, B * T_in, a.H, a.keys) ||
+      !ug_make_map<D>(&tmV, v, B * T_in, a.H, a.keys))
+    return JCA_ERR_CUDA;
+  const int64_t grid64 = a.n_units < info->sms ? a.n_units : info->sms;
+  ug_cross_attn_kernel<D><<<(int)grid64, kUgThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, a);
+  return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace jca
+
+using namespace jca;
+
+extern "C" int ug_masked_cross_attn_fwd(const void* q, const void* k, const void* v,
+                                        const void* residual, void* out, int out_fp32, int64_t B,
+                                        int T_out, int T_in, int c_u, int n_u, int H, int d_head,
+                                        float scale, int32_t* status, cudaStream_t stream) {
+  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
+  if (B < 0 || T_out < 0 || T_in < 0 || T_out > 128 || T_in > 128 || H < 1 || H >= 65536 ||
+      c_u < 0 || c_u > T_out || n_u < 0 || n_u > T_in)
+    return JCA_ERR_SHAPE;
+  // TMA row coordinates are 32-bit.
+  if (B * (int64_t)(T_out > T_in ? T_out : T_in) + 128 >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  // Tensors without elements may be null (empty tensors often have no storage).
+  const bool has_q = B > 0 && T_out > 0, has_kv = B > 0 && T_in > 0;
+  if (!status || (has_q && (!q || !out)) || (has_kv && (!k || !v))) return JCA_ERR_NULL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (residual && !aligned(residual, 16)))
+    return JCA_ERR_ALIGN;
+  if (B == 0 || T_out == 0) return JCA_OK;
+  if (T_in == 0) {
+    const int64_t n8 = B * T_out * (int64_t)H * d_head / 8;
+    const int64_t blocks64 = (n8 + 255) / 256;
+    const int blocks = (int)(blocks64 < 4096 ? blocks64 : 4096);
+    ug_no_keys_kernel<<<blocks, 256, 0, stream>>>(
+        reinterpret_cast<const __nv_bfloat16*>(residual), out, out_fp32, n8, status);
+    return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
+  }
+  UgArgs a{};
+  a.residual = reinterpret_cast<const __nv_bfloat16*>(residual);
+  a.out = out;
+  a.status = status;
+  a.B = B;
+  a.T_out = T_out;
+  a.T_in = T_in;
+  a.c_u = c_u;
+  a.n_u = n_u;
+  a.H = H;
+  const int by_q = 128 / T_out, by_k = 128 / T_in;
+  a.per_pack = by_q < by_k ? by_q : by_k;
+  a.rows_q = a.per_pack * T_out;
+  a.keys = (a.per_pack * T_in + 15) & ~15;
+  const int64_t packs = (B + a.per_pack - 1) / a.per_pack;
+  a.n_units = packs * H;
+  const float sc = scale > 0.f ? scale : 1.0f / sqrtf((float)d_head);
+  a.scale_log2 = sc * 1.4426950408889634f;
+  a.out_fp32 = out_fp32 ? 1 : 0;
+  a.out_v8 = aligned(out, 32) ? 1 : 0;
+  switch (d_head) {
+    case 16: return launch_ug<16>(q, k, v, a, B, T_out, T_in, stream);
+    case 32: return launch_ug<32>(q, k, v, a, B, T_out, T_in, stream);
+    case 64: return launch_ug<64>(q, k, v, a, B, T_out, T_in, stream);
+    default: return launch_ug<128>(q, k, v, a, B, T_out, T_in, stream);
+  }
+}

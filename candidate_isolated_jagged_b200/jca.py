@@ -56,6 +56,8 @@ _SIGNATURES = {
     "jca_bwd_workspace_bytes": (c_sz, [c_i64, c_i64, c_i32, c_i32]),
     "jagged_causal_attn_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_i64, c_i64, c_i32,
                                        c_i32, c_f32, c_i32, c_vp, c_sz, c_vp, c_vp]),
+    "ug_masked_cross_attn_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_i32,
+                                         c_i32, c_i32, c_i32, c_i32, c_i32, c_f32, c_vp, c_vp]),
     "jagged_cand_attn_bwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_f32,
                                      c_i32, c_vp, c_sz, c_vp, c_vp]),
@@ -336,6 +338,23 @@ def jagged_causal_attn_fwd(q, k, v, out, offsets, scale: float = 0.0,
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), B, T, H, d, float(scale),
         _idx_bits(offsets), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
         "jagged_causal_attn_fwd")
+
+
+def ug_masked_cross_attn_fwd(q, k, v, out, c_u: int, n_u: int, residual=None,
+                             scale: float = 0.0, status: Optional[torch.Tensor] = None,
+                             stream=None) -> int:
+    """UG-Sep's masked cross-attention: q [B, T_out, H, d], k and v [B, T_in, H, d] (bf16); the
+    first c_u outputs read only the first n_u inputs. out [B, T_out, H, d] (bf16 or fp32) gets
+    residual + R when a residual is given."""
+    B, T_out, H, d = q.shape
+    T_in = k.shape[1]
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().ug_masked_cross_attn_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(residual), _ptr(out),
+        out_fp32, B, T_out, T_in, int(c_u), int(n_u), H, d, float(scale), _ptr(status),
+        _stream(stream)), "ug_masked_cross_attn_fwd")
 
 
 def jca_bwd_workspace_bytes(B: int, T: int, H: int, d_head: int) -> int:

@@ -305,6 +305,30 @@ int jagged_causal_attn_fwd(const void* q, const void* k, const void* v, void* ou
                            int32_t* status, jca_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Variant: UG-Sep's masked cross-attention, the separated residual of a pyramid TokenMixer (UG-Sep
+ * page, "Compute Only Once: UG-Separated TokenMixer", sections 分离残差连接 and UG-Separated
+ * Mixup 与 mask). Per sample and head, the T_out output tokens (queries) attend to the T_in input
+ * tokens (keys and values) under M_UG: an output i < c_u (a U-token) reads only the inputs
+ * j < n_u (the U-tokens), every other output reads all T_in inputs. The page's formulas for R and
+ * Y were lost in extraction; the op computes R = softmax(scale Q K^T under M_UG) V and, with a
+ * residual, Y = residual + R. A U output with n_u = 0 sees no key: R = 0 there.
+ *   q, residual  [B, T_out, H, d_head] bf16, read (residual nullable: then out = R).
+ *   k, v         [B, T_in, H, d_head] bf16, read (may be the same tensor).
+ *   out          [B, T_out, H, d_head], written: bf16, or fp32 when out_fp32 != 0.
+ *   All caller-owned device memory, 16-byte aligned, token-major with row stride H * d_head.
+ *   0 <= T_out, T_in <= 128 (TokenMixer token counts), 0 <= c_u <= T_out, 0 <= n_u <= T_in;
+ *   scale <= 0 means 1/sqrt(d_head).
+ * Errors: JCA_ERR_SHAPE (a size outside those ranges, H < 1, or B * max(T_out, T_in) beyond the
+ * 32-bit row range), JCA_ERR_HEAD_DIM, JCA_ERR_NULL, JCA_ERR_ALIGN, JCA_ERR_DEVICE, JCA_ERR_CUDA.
+ * The launch is a no-op when *status is already nonzero; a pipeline wait that gives up records
+ * JCA_STATUS_TIMEOUT. No workspace.
+ * ------------------------------------------------------------------------------------------- */
+int ug_masked_cross_attn_fwd(const void* q, const void* k, const void* v, const void* residual,
+                             void* out, int out_fp32, int64_t B, int T_out, int T_in, int c_u,
+                             int n_u, int H, int d_head, float scale, int32_t* status,
+                             jca_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Training: the forward with its log-sum-exp, and the backward pass. The pages train on the same
  * packed layout they serve (候选隔离注意力掩码, section 训练时的序列打包: several users' sequences
  * in one packed matrix, split at cu_seqlens = the offsets here), under the same mask.

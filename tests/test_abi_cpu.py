@@ -28,7 +28,7 @@ def test_header_declares_the_entry_points():
               "jagged_cand_attn_plan", "jagged_cand_attn_run", "cand_only_attn_plan",
               "cand_only_attn_run", "jca_stack_workspace_bytes", "jca_stack_fwd",
               "jagged_cand_attn_fwd_lse", "jca_bwd_workspace_bytes", "jagged_cand_attn_bwd",
-              "jagged_causal_attn_fwd"]:
+              "jagged_causal_attn_fwd", "ug_masked_cross_attn_fwd"]:
         assert n in names
 
 
@@ -181,3 +181,32 @@ def test_causal_host_argument_errors(L):
     assert L.jagged_causal_attn_fwd(*args[:5], None, *args[6:]) == -1         # offsets
     assert L.jagged_causal_attn_fwd(*args[:3], _addr(0x10002), *args[4:]) == -4
     assert L.jagged_causal_attn_fwd(*args[:13], 16, *args[14:]) == -6         # workspace
+
+
+def test_ug_host_argument_errors(L):
+    p = _addr(0x10000)  # never dereferenced: every call below returns before any device work
+    st = _addr(0x20000)
+
+    def call(q=p, k=p, v=p, res=None, out=p, B=4, T_out=16, T_in=32, c_u=8, n_u=16, H=1, d=128,
+             status=st):
+        return L.ug_masked_cross_attn_fwd(q, k, v, res, out, 0, B, T_out, T_in, c_u, n_u, H, d,
+                                          0.0, status, None)
+
+    assert call(d=48) == -3
+    assert call(T_in=129) == -2
+    assert call(T_out=129) == -2
+    assert call(c_u=17) == -2
+    assert call(n_u=33) == -2
+    assert call(c_u=-1) == -2
+    assert call(H=0) == -2
+    assert call(B=-1) == -2
+    assert call(B=1 << 40) == -2          # row coordinates beyond 32 bits
+    assert call(q=None) == -1
+    assert call(status=None) == -1
+    assert call(k=None) == -1
+    assert call(out=None) == -1
+    assert call(q=None, k=None, v=None, T_in=0, n_u=0) == -1   # k, v may be null, q may not
+    assert call(v=_addr(0x10004)) == -4
+    assert call(res=_addr(0x10008)) == -4
+    assert call(B=0) == 0                 # nothing to do, nothing launched
+    assert call(T_out=0, c_u=0) == 0
