@@ -75,8 +75,7 @@ struct UgCfg {
   static constexpr int B_SFULL = B_EMPTY + STAGES;  // [group] S written by QK
   static constexpr int B_PFULL = B_SFULL + 2;       // [group] P written over S
   static constexpr int B_OFULL = B_PFULL + 2;       // [group] O written by PV
-  static constexpr int B_TFREE = B_OFULL + 2;       // [group] O read: S and O may be reused
-  static constexpr int B_DRAIN = B_TFREE + 2;
+  static constexpr int B_DRAIN = B_OFULL + 2;
   static constexpr int NUM_BARS = B_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_USED = OFF_MISC + 16;
@@ -142,14 +141,14 @@ __device__ void ug_mma(const UgArgs& a, uint32_t sbase, uint32_t bars, uint32_t 
   const uint64_t dk = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
   const uint64_t dv = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
   const int kpv = a.keys >> 4;
-  // S_g = Q K^T of unit i (group g = i & 1), once its operands landed and the group has read the
-  // O of its previous unit (so S_g, where that unit's P lives, and O_g are both free).
+  // S_g = Q K^T of unit i (group g = i & 1) once its operands landed. It is issued after PV(i - 2),
+  // the last reader of S_g (the P of the group's previous unit), and MMAs from one thread execute
+  // in issue order; the group reads this S only after its SFULL, so the QK may run while the group
+  // still finishes its previous unit. O_g is overwritten only by PV(i), which waits for the
+  // group's P of unit i, written after the group read the previous O_g.
   auto issue_qk = [&](int i) -> bool {
     const int s = i % C::STAGES, g = i & 1;
     if (!mbar_wait(bars + 8 * (C::B_FULL + s), (i / C::STAGES) & 1, abort_flag, a.status))
-      return false;
-    if (i >= 2 &&
-        !mbar_wait(bars + 8 * (C::B_TFREE + g), ((i >> 1) - 1) & 1, abort_flag, a.status))
       return false;
     tc_fence_after();
     const uint64_t so = (uint64_t)((s * C::STAGE_BYTES) >> 4);
@@ -190,6 +189,12 @@ __device__ void ug_mma(const UgArgs& a, uint32_t sbase, uint32_t bars, uint32_t 
     tc_commit(bars + 8 * C::B_DRAIN);
     mbar_wait_drain(bars + 8 * C::B_DRAIN, 0);
   }
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // Writes 8 consecutive output values (bf16 or fp32).
@@ -243,6 +248,15 @@ __device__ void ug_softmax(const UgArgs& a, uint32_t bars, uint32_t tmem,
   const int col0 = sl * a.T_in;
   const int ncols = in_pack ? (ti < a.c_u ? a.n_u : a.T_in) : 0;
   const int kchunks = (a.keys + 31) >> 5;       // 32-key chunks of P the PV reads
+  // The warp's rows lie in samples [w_first, w_last] of a pack, whose blocks of S fill the 32-key
+  // chunks [ch_lo, ch_hi]; a warp without a row in the pack reads no chunk (its lanes' P and O
+  // rows feed no output).
+  const int r0 = quarter * 32;
+  const bool warp_in = r0 < a.rows_q;
+  const int w_first = warp_in ? r0 / a.T_out : 0;
+  const int w_last = warp_in ? min(r0 + 31, a.rows_q - 1) / a.T_out : 0;
+  const int ch_lo = warp_in ? (w_first * a.T_in) >> 5 : 4;
+  const int ch_hi = warp_in ? ((w_last + 1) * a.T_in - 1) >> 5 : -1;
   const float sl2 = a.scale_log2;
   const int n_local = local_units(a.n_units);
   bool ok = true;
@@ -265,46 +279,61 @@ __device__ void ug_softmax(const UgArgs& a, uint32_t bars, uint32_t tmem,
                     mbar_wait(bars + 8 * (C::B_SFULL + grp), (i >> 1) & 1, abort_flag, a.status));
     if (!ok) break;
     tc_fence_after();
-    uint32_t x[128];
-    tmem_ld_x32(t_s + 0, x);
-    tmem_ld_x32(t_s + 32, x + 32);
-    tmem_ld_x32(t_s + 64, x + 64);
-    tmem_ld_x32(t_s + 96, x + 96);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < 128; c += 16) reg_fence16(x + c);
-    // Only the row's own columns [col0, col0 + nc) count; the others are masked to -inf.
+    // Only the 32-key chunks of S that hold the blocks of the warp's samples are read (twice: the
+    // row max, then the probabilities), 32 columns at a time; inside a chunk a bit mask keeps the
+    // row's own columns [col0, col0 + nc).
     const int hi = col0 + nc;
-    float mx = -INFINITY;
+    auto chunk_bits = [&](int c) -> uint32_t {
+      const int lo_c = min(max(col0 - 32 * c, 0), 32), hi_c = min(max(hi - 32 * c, 0), 32);
+      return (hi_c >= 32 ? 0xffffffffu : ((1u << hi_c) - 1u)) &
+             ~(lo_c >= 32 ? 0xffffffffu : ((1u << lo_c) - 1u));
+    };
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+    for (int c = ch_lo; c <= ch_hi; ++c) {
+      uint32_t x[32];
+      tmem_ld_x32(t_s + 32 * c, x);
+      tmem_wait_ld();
+      reg_fence16(x);
+      reg_fence16(x + 16);
+      const uint32_t bits = chunk_bits(c);
 #pragma unroll
-    for (int c = 0; c < 128; ++c)
-      mx = fmaxf(mx, (c >= col0 && c < hi) ? __uint_as_float(x[c]) : -INFINITY);
-    const float m = mx * sl2;
+      for (int j = 0; j < 32; j += 4) {
+        const uint32_t b = bits >> j;
+        mx0 = fmax3(mx0, (b & 1u) ? __uint_as_float(x[j]) : -INFINITY,
+                    (b & 2u) ? __uint_as_float(x[j + 1]) : -INFINITY);
+        mx1 = fmax3(mx1, (b & 4u) ? __uint_as_float(x[j + 2]) : -INFINITY,
+                    (b & 8u) ? __uint_as_float(x[j + 3]) : -INFINITY);
+      }
+    }
+    const float m = fmaxf(mx0, mx1) * sl2;
     const float neg_m = (nc == 0) ? 0.f : -m;
-    float l = 0.f;
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      if (c >= kchunks) break;
+    float l0 = 0.f, l1 = 0.f;
+    for (int c = 0; c < kchunks; ++c) {
       uint32_t pk[16];
-      if (col0 < 32 * c + 32 && hi > 32 * c) {
-        float acc = 0.f;
+      if (c >= ch_lo && c <= ch_hi) {
+        uint32_t x[32];
+        tmem_ld_x32(t_s + 32 * c, x);
+        tmem_wait_ld();
+        reg_fence16(x);
+        reg_fence16(x + 16);
+        const uint32_t bits = chunk_bits(c);
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const int c0 = 32 * c + 2 * k;
-          const float p0 = (c0 >= col0 && c0 < hi)
-                               ? fast_exp2(fmaf(__uint_as_float(x[c0]), sl2, neg_m)) : 0.f;
-          const float p1 = (c0 + 1 >= col0 && c0 + 1 < hi)
-                               ? fast_exp2(fmaf(__uint_as_float(x[c0 + 1]), sl2, neg_m)) : 0.f;
-          acc += p0 + p1;
+          const uint32_t b = bits >> (2 * k);
+          const float p0 = (b & 1u) ? fast_exp2(fmaf(__uint_as_float(x[2 * k]), sl2, neg_m)) : 0.f;
+          const float p1 =
+              (b & 2u) ? fast_exp2(fmaf(__uint_as_float(x[2 * k + 1]), sl2, neg_m)) : 0.f;
+          l0 += p0;
+          l1 += p1;
           pk[k] = pack_bf16x2(p0, p1);
         }
-        l += acc;
       } else {
 #pragma unroll
         for (int k = 0; k < 16; ++k) pk[k] = 0u;
       }
       tmem_st_x16(t_s + 16 * c, pk);
     }
+    const float l = l0 + l1;
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(bars + 8 * (C::B_PFULL + grp));
@@ -330,11 +359,6 @@ __device__ void ug_softmax(const UgArgs& a, uint32_t bars, uint32_t tmem,
       tmem_wait_ld();
 #pragma unroll
       for (int k = 0; k < CW; k += 16) reg_fence16(w + k);
-      if (c0 + CW >= D) {
-        // O_g has been read: the MMA warp may reuse S_g and O_g for the group's next unit.
-        tc_fence_before();
-        mbar_arrive(bars + 8 * (C::B_TFREE + grp));
-      }
       if (!row_ok) continue;
       float o[CW];
 #pragma unroll
@@ -385,7 +409,6 @@ __global__ void __launch_bounds__(kUgThreads, 1)
       mbar_init(bars + 8 * (C::B_SFULL + g), 1);
       mbar_init(bars + 8 * (C::B_PFULL + g), kUgGroupThreads);
       mbar_init(bars + 8 * (C::B_OFULL + g), 1);
-      mbar_init(bars + 8 * (C::B_TFREE + g), kUgGroupThreads);
     }
     mbar_init(bars + 8 * C::B_DRAIN, 1);
     *abort_flag = 0;
