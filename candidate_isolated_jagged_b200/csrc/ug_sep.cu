@@ -93,6 +93,25 @@ __device__ __forceinline__ int local_units(int64_t n_units) {
   return b < n_units ? (int)((n_units - b + gridDim.x - 1) / gridDim.x) : 0;
 }
 
+// Non-blocking test of an mbarrier phase (the MMA thread polls two barriers).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 template <int D>
 __device__ void ug_producer(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                             const CUtensorMap* tmV, const UgArgs& a, uint32_t sbase,
@@ -146,10 +165,8 @@ __device__ void ug_mma(const UgArgs& a, uint32_t sbase, uint32_t bars, uint32_t 
   // in issue order; the group reads this S only after its SFULL, so the QK may run while the group
   // still finishes its previous unit. O_g is overwritten only by PV(i), which waits for the
   // group's P of unit i, written after the group read the previous O_g.
-  auto issue_qk = [&](int i) -> bool {
+  auto issue_qk = [&](int i) {
     const int s = i % C::STAGES, g = i & 1;
-    if (!mbar_wait(bars + 8 * (C::B_FULL + s), (i / C::STAGES) & 1, abort_flag, a.status))
-      return false;
     tc_fence_after();
     const uint64_t so = (uint64_t)((s * C::STAGE_BYTES) >> 4);
 #pragma unroll
@@ -160,12 +177,10 @@ __device__ void ug_mma(const UgArgs& a, uint32_t sbase, uint32_t bars, uint32_t 
              kk > 0 ? 1u : 0u);
     }
     tc_commit(bars + 8 * (C::B_SFULL + g));
-    return true;
   };
   // O_g = P_g V of unit i; P_g is read from the first keys / 2 columns of S_g (bf16 pairs).
-  auto issue_pv = [&](int i) -> bool {
+  auto issue_pv = [&](int i) {
     const int s = i % C::STAGES, g = i & 1;
-    if (!mbar_wait(bars + 8 * (C::B_PFULL + g), (i >> 1) & 1, abort_flag, a.status)) return false;
     tc_fence_after();
     const uint64_t vb = dv + (uint64_t)((s * C::STAGE_BYTES) >> 4);
     constexpr uint32_t kStep = (16 * C::SW) >> 4;   // 16 key rows of V per k-step
@@ -176,25 +191,44 @@ __device__ void ug_mma(const UgArgs& a, uint32_t sbase, uint32_t bars, uint32_t 
                 kk > 0 ? 1u : 0u);
     tc_commit(bars + 8 * (C::B_EMPTY + s));
     tc_commit(bars + 8 * (C::B_OFULL + g));
-    return true;
   };
+  auto full_bar = [&](int i) { return bars + 8 * (C::B_FULL + i % C::STAGES); };
+  auto full_par = [&](int i) { return (uint32_t)((i / C::STAGES) & 1); };
   bool ok = true;
-  if (n_local > 0) ok = issue_qk(0);
+  if (n_local > 0) {
+    ok = mbar_wait(full_bar(0), full_par(0), abort_flag, a.status);
+    if (ok) issue_qk(0);
+  }
+  // After PV(i - 1), both QK(i + 1) (the other group's S, last read by PV(i - 1)) and PV(i) may be
+  // issued; whichever becomes ready first goes first, PV(i) when both are, so that a late load of
+  // unit i + 1 never holds back the PV that releases unit i's stage.
   for (int i = 0; ok && i < n_local; ++i) {
-    if (i + 1 < n_local) ok = issue_qk(i + 1);   // the other group's buffers
-    if (ok) ok = issue_pv(i);
+    bool qk_done = i + 1 >= n_local, pv_done = false;
+    const uint32_t pbar = bars + 8 * (C::B_PFULL + (i & 1)), ppar = (uint32_t)((i >> 1) & 1);
+    const uint64_t t0 = global_timer_ns();
+    while (!(qk_done && pv_done)) {
+      if (!qk_done && mbar_test(full_bar(i + 1), full_par(i + 1))) {
+        issue_qk(i + 1);
+        qk_done = true;
+      } else if (!pv_done && mbar_test(pbar, ppar)) {
+        issue_pv(i);
+        pv_done = true;
+      } else if (*abort_flag) {
+        ok = false;
+        break;
+      } else if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+        *abort_flag = 1;
+        atomicCAS(a.status, 0, (int32_t)JCA_STATUS_TIMEOUT);
+        ok = false;
+        break;
+      }
+    }
   }
   if (!ok) {
     // Aborting: wait until every MMA this thread issued has completed.
     tc_commit(bars + 8 * C::B_DRAIN);
     mbar_wait_drain(bars + 8 * C::B_DRAIN, 0);
   }
-}
-
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
 }
 
 // Writes 8 consecutive output values (bf16 or fp32).
