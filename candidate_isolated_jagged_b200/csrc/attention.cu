@@ -272,6 +272,7 @@ struct MmaState {
   uint32_t p_seen[2];   // P-full completions consumed, per softmax group
   uint32_t o_items[2];  // items whose O_w was written, per group (O-free completions expected)
   uint32_t q_seen[2];   // Q-full completions consumed, per query tile
+  uint32_t v_seen;      // global key tiles whose V stage was seen full (the second PV skips it)
   // Operand descriptors of Q buffer 0 and of K / V stage 0 (start address of the first k-step);
   // a buffer, stage or k-step adds an offset to the low bits (shared addresses stay below 256 KB,
   // so the 14-bit field never carries).
@@ -320,8 +321,11 @@ __device__ __forceinline__ bool issue_pv(int grp, uint32_t gg, int jj, int valid
                                          volatile int* abort_flag) {
   using C = Cfg<D>;
   const int s = (int)(gg % C::KVS);
-  if (!mbar_wait(bars + 8 * (C::B_VFULL + s), (gg / C::KVS) & 1, abort_flag, a.status))
-    return false;
+  if (gg + 1 != st.v_seen) {
+    if (!mbar_wait(bars + 8 * (C::B_VFULL + s), (gg / C::KVS) & 1, abort_flag, a.status))
+      return false;
+    st.v_seen = gg + 1;
+  }
   if (!mbar_wait(bars + 8 * (C::B_PFULL + grp), st.p_seen[grp] & 1, abort_flag, a.status))
     return false;
   ++st.p_seen[grp];
@@ -357,6 +361,7 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
   st.p_seen[0] = st.p_seen[1] = 0;
   st.o_items[0] = st.o_items[1] = 0;
   st.q_seen[0] = st.q_seen[1] = 0;
+  st.v_seen = 0;
   st.q = smem_desc(sbase + C::OFF_Q, 16, 8 * C::SW, C::LAYOUT);
   st.k = smem_desc(sbase + C::OFF_K, 16, 8 * C::SW, C::LAYOUT);
   st.v = smem_desc(sbase + C::OFF_V, C::BLK_BYTES, 8 * C::SW, C::LAYOUT);
