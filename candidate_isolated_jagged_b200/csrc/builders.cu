@@ -282,27 +282,44 @@ __global__ void __launch_bounds__(1024) work_queue_kernel(
     }
     return;
   }
-  // Pass 2, one thread per user (all users at once, so that the loads of a user's offsets and
-  // bounds are not serialised behind other users'): the thread claims the user's run of nq * H
-  // slots and writes it.
-  for (int64_t b = tid; b < B; b += blockDim.x) {
-    const long long s = (long long)qoff[b], e = (long long)qoff[b + 1];
-    const long long lo = (long long)kvlo[b], hi = (long long)kvhi[b];
-    const long long nq = (e - s + kItemRows - 1) / kItemRows;
-    if (nq == 0) continue;
-    const long long nkv = (hi - lo + kTileN - 1) / kTileN;
-    const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
-    const unsigned long long pos = atomicAdd(&s_cursor[key], (unsigned long long)(nq * H));
-    const int holes = (kv_count != nullptr && (long long)kv_count[b] != hi - lo) ? 1 : 0;
-    const int w = (int)(hi - lo) | (holes << 31);
-    for (int h = 0; h < H; ++h) {
-      for (long long t = 0; t < nq; ++t) {
-        const long long row0 = s + t * kItemRows;
-        const int rows = (int)min((long long)kItemRows, e - row0);
-        items[pos + (unsigned long long)(h * nq + t)] =
-            make_int4((int)row0, (h << 9) | rows, (int)lo, w);
+  // Pass 2, per chunk of 1024 users: one thread per user claims the user's run of nq * H slots
+  // (all users at once, so that no user's loads wait behind another's), then one thread per
+  // (user, head) writes that head's nq items, so that no thread writes more than one head's run.
+  __shared__ unsigned long long s_pos[1024];
+  __shared__ int s_nq[1024];
+  for (int64_t b0 = 0; b0 < B; b0 += blockDim.x) {
+    const int64_t b = b0 + tid;
+    int nq_b = 0;
+    if (b < B) {
+      const long long s = (long long)qoff[b], e = (long long)qoff[b + 1];
+      const long long lo = (long long)kvlo[b], hi = (long long)kvhi[b];
+      nq_b = (int)((e - s + kItemRows - 1) / kItemRows);
+      if (nq_b > 0) {
+        const long long nkv = (hi - lo + kTileN - 1) / kTileN;
+        const int key = (int)min(nkv, (long long)(kQueueBuckets - 1));
+        s_pos[tid] = atomicAdd(&s_cursor[key], (unsigned long long)nq_b * (unsigned long long)H);
       }
     }
+    s_nq[tid] = nq_b;
+    __syncthreads();
+    const int nb = (int)min((int64_t)blockDim.x, B - b0);
+    for (int p = tid; p < nb * H; p += blockDim.x) {
+      const int ub = p / H, h = p - ub * H;
+      const int nq = s_nq[ub];
+      if (nq == 0) continue;
+      const int64_t bb = b0 + ub;
+      const long long s = (long long)qoff[bb], e = (long long)qoff[bb + 1];
+      const long long lo = (long long)kvlo[bb], hi = (long long)kvhi[bb];
+      const int holes = (kv_count != nullptr && (long long)kv_count[bb] != hi - lo) ? 1 : 0;
+      const int w = (int)(hi - lo) | (holes << 31);
+      const unsigned long long pos = s_pos[ub] + (unsigned long long)h * (unsigned long long)nq;
+      for (int t = 0; t < nq; ++t) {
+        const long long row0 = s + (long long)t * kItemRows;
+        const int rows = (int)min((long long)kItemRows, e - row0);
+        items[pos + (unsigned long long)t] = make_int4((int)row0, (h << 9) | rows, (int)lo, w);
+      }
+    }
+    __syncthreads();
   }
   if (tid == 0) *n_items = (int32_t)s_total;
 }
