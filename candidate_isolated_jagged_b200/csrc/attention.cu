@@ -350,7 +350,7 @@ struct PendingPV {
   bool last;     // the item's last key tile: its completion makes O ready
 };
 
-template <int D>
+template <int D, bool CAUSAL>
 __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort_flag, ItemRing ring) {
   using C = Cfg<D>;
@@ -400,6 +400,10 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
       const int s = (int)(g % C::KVS);
       const uint32_t ph = (g / C::KVS) & 1;
       const bool last = j == w.n_kv - 1;
+      // Causal variant: an item's key tiles end at its last row, which tile B holds; tile A's
+      // rows end 128 rows earlier and see none of the last key tile, so A stops one tile early.
+      const bool a_skips = CAUSAL && has_b && last;
+      const bool last_a = (CAUSAL && has_b) ? j == w.n_kv - 2 : last;
       const int valid = min(C::BN, w.kv_len - j * C::BN);
       const uint32_t idesc_qk =
           valid == C::BN ? kIdescQKFull
@@ -409,9 +413,11 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
       if (!ok) break;
       tc_fence_after();
       // QK_A(t)
-      mma_qk<D>(tmem + C::TMEM_S0, qa, kb, idesc_qk);
-      tc_commit(bars + 8 * C::B_SFULL);
-      if (last) tc_commit(bars + 8 * (C::B_QEMPTY + qslot_a));
+      if (!a_skips) {
+        mma_qk<D>(tmem + C::TMEM_S0, qa, kb, idesc_qk);
+        tc_commit(bars + 8 * C::B_SFULL);
+        if (last_a) tc_commit(bars + 8 * (C::B_QEMPTY + qslot_a));
+      }
       // PV_B(t-1), possibly of the previous item
       ok = flush_b();
       if (!ok) break;
@@ -430,12 +436,14 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
       }
       tc_commit(bars + 8 * (C::B_KEMPTY + s));
       // PV_A(t); the V stage is released here when the item has no tile B, else after PV_B(t).
-      ok = issue_pv<D>(0, g, j, valid, st, bars, tmem, a, abort_flag);
-      if (!ok) break;
-      if (!has_b) tc_commit(bars + 8 * (C::B_VEMPTY + s));
-      if (last) {
-        tc_commit(bars + 8 * C::B_OREADY);
-        ++st.o_items[0];
+      if (!a_skips) {
+        ok = issue_pv<D>(0, g, j, valid, st, bars, tmem, a, abort_flag);
+        if (!ok) break;
+        if (!has_b) tc_commit(bars + 8 * (C::B_VEMPTY + s));
+        if (last_a) {
+          tc_commit(bars + 8 * C::B_OREADY);
+          ++st.o_items[0];
+        }
       }
       if (has_b) pend = PendingPV{g, j, valid, last};
     }
@@ -711,7 +719,9 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
     const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
     const int seg = row_ok ? (CAUSAL ? 1 : (a.q_seg ? (int)a.q_seg[row] : -1)) : 0;
     float m = -INFINITY, l = 0.f;             // running max (log2 units) and row sum
-    for (int j = 0; j < w.n_kv; ++j, ++lt) {
+    // Causal variant: tile A of a two-tile item sees none of the item's last key tile.
+    const int n_kv_g = (CAUSAL && grp == 0 && w.nrows > C::BM) ? w.n_kv - 1 : w.n_kv;
+    for (int j = 0; j < n_kv_g; ++j, ++lt) {
       const int valid = min(C::BN, w.kv_len - j * C::BN);
       const int nchunks = (valid + 31) >> 5;
       // Edge tiles (the trimmed last tile, or any tile of a user with padding holes) are masked
@@ -916,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane < 2)
         producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag, lane == 1, ring);
     } else if (warp == 1) {
-      if (lane == 0) mma_role<D>(a, sbase, bars, tmem, abort_flag, ring);
+      if (lane == 0) mma_role<D, CAUSAL>(a, sbase, bars, tmem, abort_flag, ring);
     } else if (warp < 10) {
       softmax_role<D, CAUSAL, LSE>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
                       abort_flag, warp, lane, ring);
