@@ -314,7 +314,9 @@ int jagged_causal_attn_fwd(const void* q, const void* k, const void* v, void* ou
  * residual, Y = residual + R. A U output with n_u = 0 sees no key: R = 0 there.
  *   q, residual  [B, T_out, H, d_head] bf16, read (residual nullable: then out = R).
  *   k, v         [B, T_in, H, d_head] bf16, read (may be the same tensor).
- *   out          [B, T_out, H, d_head], written: bf16, or fp32 when out_fp32 != 0.
+ *   out          [B, T_out, H, d_head], written: bf16, or fp32 when out_fp32 != 0. With a bf16
+ *                output, out may be the residual tensor itself (Y = X + R in place: each row is
+ *                read before the same thread writes it, and no other thread touches it).
  *   All caller-owned device memory, 16-byte aligned, token-major with row stride H * d_head.
  *   0 <= T_out, T_in <= 128 (TokenMixer token counts), 0 <= c_u <= T_out, 0 <= n_u <= T_in;
  *   scale <= 0 means 1/sqrt(d_head).

@@ -6,7 +6,8 @@ Covered: packs of several samples with a ragged last pack, token counts that do 
 one sample per pack at the 128-token limit, head sizes 16-128, several heads, bf16 and fp32
 outputs, with and without a residual; the degenerate cases (no U output, only U outputs, no U
 input, no input at all, one token); U outputs bit-identical when the G inputs change; a preset
-status word; and the 16,384-sample workload the benchmark times, on sampled samples."""
+status word; the residual updated in place; and the 16,384-sample workload the benchmark times,
+on sampled samples."""
 
 import numpy as np
 import pytest
@@ -119,3 +120,15 @@ def test_ug_sep16k_sampled(out_fp32):
     else:
         assert_close_bf16(got_s, ref, "ug_sep16k bf16")
     assert bool(torch.isfinite(got.float()).all())
+
+
+def test_ug_in_place_residual():
+    """out may be the residual tensor itself (bf16): Y = X + R in place."""
+    b = synth.custom_ug(37, 16, 32, 8, 16, 2, 64, seed=31)
+    x = b.residual.to(dev()).clone()
+    st = jca.new_status(dev())
+    jca.ug_masked_cross_attn_fwd(b.q.to(dev()), b.k.to(dev()), b.v.to(dev()), x, b.c_u, b.n_u,
+                                 residual=x, status=st)
+    torch.cuda.synchronize()
+    jca.check_status(st, "ug in place")
+    assert_close_bf16(x, _ref(b), "ug in place")
