@@ -956,51 +956,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
-// 3-D map over a token-major [rows, H, D] bf16 tensor; box = {swizzle span, 1 head, 128 rows}.
-template <int D>
-bool make_map(CUtensorMap* map, const void* base, int64_t rows, int H) {
-  using C = Cfg<D>;
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)C::BOX_X, 1u, (cuuint32_t)C::BM};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUtensorMapSwizzle sw = C::SW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : C::SW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                              : CU_TENSOR_MAP_SWIZZLE_32B;
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-struct DeviceInfo {
-  int sms = 0;
-  bool sm100 = false;
-  bool attr_set[4] = {false, false, false, false};
-};
-
+// Kernel attributes set so far, per device and head size.
 constexpr int kMaxDevices = 64;
-DeviceInfo g_dev[kMaxDevices];
-std::mutex g_dev_mu;
+bool g_attr_set[kMaxDevices][4];
+std::mutex g_attr_mu;
 
 int d_index(int d) { return d == 16 ? 0 : d == 32 ? 1 : d == 64 ? 2 : 3; }
 
@@ -1008,21 +967,12 @@ template <int D>
 int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void* k,
                        const void* v, int64_t Tkv, cudaStream_t stream) {
   using C = Cfg<D>;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return JCA_ERR_CUDA;
-  DeviceInfo* info = &g_dev[dev];
+  int dev = 0, sms = 0;
+  const int rc = current_device(&dev, &sms);
+  if (rc) return rc;
   {
-    std::lock_guard<std::mutex> lock(g_dev_mu);
-    if (info->sms == 0) {
-      int major = 0, sms = 0;
-      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return JCA_ERR_CUDA;
-      info->sm100 = (major == 10);
-      info->sms = sms;
-    }
-    if (!info->sm100) return JCA_ERR_DEVICE;
-    if (!info->attr_set[d_index(D)]) {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (!g_attr_set[dev][d_index(D)]) {
       if (cudaFuncSetAttribute(jagged_attn_kernel<D, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess ||
@@ -1033,25 +983,26 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess)
         return JCA_ERR_CUDA;
-      info->attr_set[d_index(D)] = true;
+      g_attr_set[dev][d_index(D)] = true;
     }
   }
   CUtensorMap tmQ, tmK, tmV;
-  if (!make_map<D>(&tmQ, q, Tq, a.H) || !make_map<D>(&tmK, k, Tkv, a.H) ||
-      !make_map<D>(&tmV, v, Tkv, a.H))
+  if (!make_rows_map_bf16(&tmQ, q, Tq, a.H, D, C::BM) ||
+      !make_rows_map_bf16(&tmK, k, Tkv, a.H, D, C::BM) ||
+      !make_rows_map_bf16(&tmV, v, Tkv, a.H, D, C::BM))
     return JCA_ERR_CUDA;
   AttnArgs args = a;
   args.out_v8 = aligned(a.out, 32) ? 1 : 0;
   // Instantiations: the main path, the causal variant, and the training forward (log-sum-exp
   // output); each mode is compile-time so that the main path carries none of the others' code.
   if (a.causal)
-    jagged_attn_kernel<D, true, false><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
+    jagged_attn_kernel<D, true, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
                                                                                         tmV, args);
   else if (a.lse != nullptr)
-    jagged_attn_kernel<D, false, true><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
+    jagged_attn_kernel<D, false, true><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
                                                                                         tmV, args);
   else
-    jagged_attn_kernel<D, false, false><<<info->sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
+    jagged_attn_kernel<D, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
                                                                                          tmV, args);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }

@@ -823,49 +823,9 @@ __global__ void __launch_bounds__(1024) dkv_queue_kernel(const IdxT* __restrict_
 // ------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn bwd_encode_fn() {
-  static EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
-// 3-D map over a token-major [rows, H, D] bf16 tensor; box = {swizzle span, 1 head, 128 rows}.
-template <int D>
-bool bwd_map(CUtensorMap* map, const void* base, int64_t rows, int H) {
-  using C = BCfg<D>;
-  EncodeTiledFn enc = bwd_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)C::BOX_X, 1u, (cuuint32_t)C::BM};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUtensorMapSwizzle sw = C::SW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : C::SW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                              : CU_TENSOR_MAP_SWIZZLE_32B;
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
+// Kernel attributes set so far, per device, head size and mode.
 constexpr int kMaxDevices = 64;
-struct BwdDevice {
-  int sms = 0;
-  bool sm100 = false;
-  bool attr_set[4][2] = {};
-};
-BwdDevice g_bwd_dev[kMaxDevices];
+bool g_bwd_attr[kMaxDevices][4][2];
 std::mutex g_bwd_mu;
 
 int d_slot(int d) { return d == 16 ? 0 : d == 32 ? 1 : d == 64 ? 2 : 3; }
@@ -874,33 +834,26 @@ template <int D, int MODE>
 int launch_bwd_mode(const BwdArgs& a, const void* o1, const void* o2, const void* i1,
                     const void* i2, int64_t T, cudaStream_t stream) {
   using C = BCfg<D>;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return JCA_ERR_CUDA;
-  BwdDevice* info = &g_bwd_dev[dev];
+  int dev = 0, sms = 0;
+  const int rc = current_device(&dev, &sms);
+  if (rc) return rc;
   {
     std::lock_guard<std::mutex> lock(g_bwd_mu);
-    if (info->sms == 0) {
-      int major = 0, sms = 0;
-      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return JCA_ERR_CUDA;
-      info->sm100 = major == 10;
-      info->sms = sms;
-    }
-    if (!info->sm100) return JCA_ERR_DEVICE;
-    if (!info->attr_set[d_slot(D)][MODE]) {
+    if (!g_bwd_attr[dev][d_slot(D)][MODE]) {
       if (cudaFuncSetAttribute(jagged_attn_bwd_kernel<D, MODE>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess)
         return JCA_ERR_CUDA;
-      info->attr_set[d_slot(D)][MODE] = true;
+      g_bwd_attr[dev][d_slot(D)][MODE] = true;
     }
   }
   CUtensorMap m1, m2, m3, m4;
-  if (!bwd_map<D>(&m1, o1, T, a.H) || !bwd_map<D>(&m2, o2, T, a.H) ||
-      !bwd_map<D>(&m3, i1, T, a.H) || !bwd_map<D>(&m4, i2, T, a.H))
+  if (!make_rows_map_bf16(&m1, o1, T, a.H, D, C::BM) ||
+      !make_rows_map_bf16(&m2, o2, T, a.H, D, C::BM) ||
+      !make_rows_map_bf16(&m3, i1, T, a.H, D, C::BM) ||
+      !make_rows_map_bf16(&m4, i2, T, a.H, D, C::BM))
     return JCA_ERR_CUDA;
-  jagged_attn_bwd_kernel<D, MODE><<<info->sms, kBwdThreads, C::SMEM_ALLOC, stream>>>(m1, m2, m3,
+  jagged_attn_bwd_kernel<D, MODE><<<sms, kBwdThreads, C::SMEM_ALLOC, stream>>>(m1, m2, m3,
                                                                                       m4, a);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }

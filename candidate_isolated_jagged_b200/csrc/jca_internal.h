@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "jca.h"
@@ -23,6 +24,16 @@ inline bool aligned(const void* p, size_t a) {
 inline bool head_dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 
 int64_t max_work_items(int64_t B, int64_t rows, int H);
+
+// TMA map over a token-major [rows, H, D] bf16 tensor (3-D: D, H, rows), box = {swizzle span,
+// 1 head, box_rows}; swizzle span = min(128, 2 D) bytes. Rows past the end read as zeros. Returns
+// false when the driver's encoder is unavailable or rejects the map.
+bool make_rows_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int H, int D,
+                        int box_rows);
+
+// The current device (index < 64) and its multiprocessor count, cached per device. Returns
+// JCA_ERR_DEVICE on a device that is not sm_100, JCA_ERR_CUDA when a query fails.
+int current_device(int* dev, int* sms);
 
 // Carve-up of the caller's workspace (all offsets 256-byte aligned).
 struct WorkspaceLayout {

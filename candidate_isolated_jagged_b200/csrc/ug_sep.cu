@@ -503,85 +503,35 @@ __global__ void ug_no_keys_kernel(const __nv_bfloat16* __restrict__ residual, vo
 // ------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn ug_encode_fn() {
-  static EncodeTiledFn fn = []() -> EncodeTiledFn {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return nullptr;
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
-
-// 3-D map over a token-major [rows, H, D] bf16 tensor; box = {swizzle span, 1 head, box_rows}.
-// Rows past the end read as zeros.
-template <int D>
-bool ug_make_map(CUtensorMap* map, const void* base, int64_t rows, int H, int box_rows) {
-  using C = UgCfg<D>;
-  EncodeTiledFn enc = ug_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  const cuuint32_t box[3] = {(cuuint32_t)C::BOX_X, 1u, (cuuint32_t)box_rows};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUtensorMapSwizzle sw = C::SW == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
-                                : C::SW == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
-                                              : CU_TENSOR_MAP_SWIZZLE_32B;
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
-             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-struct UgDevice {
-  int sms = 0;
-  bool sm100 = false;
-  bool attr_set[4] = {false, false, false, false};
-};
+// Kernel attributes set so far, per device and head size.
 constexpr int kUgMaxDevices = 64;
-UgDevice g_ug_dev[kUgMaxDevices];
+bool g_ug_attr[kUgMaxDevices][4];
 std::mutex g_ug_mu;
 
 template <int D>
 int launch_ug(const void* q, const void* k, const void* v, UgArgs a, int64_t B, int T_out,
               int T_in, cudaStream_t stream) {
   using C = UgCfg<D>;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kUgMaxDevices) return JCA_ERR_CUDA;
-  UgDevice* info = &g_ug_dev[dev];
+  int dev = 0, sms = 0;
+  const int rc = current_device(&dev, &sms);
+  if (rc) return rc;
   const int di = D == 16 ? 0 : D == 32 ? 1 : D == 64 ? 2 : 3;
   {
     std::lock_guard<std::mutex> lock(g_ug_mu);
-    if (info->sms == 0) {
-      int major = 0, sms = 0;
-      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-          cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return JCA_ERR_CUDA;
-      info->sm100 = (major == 10);
-      info->sms = sms;
-    }
-    if (!info->sm100) return JCA_ERR_DEVICE;
-    if (!info->attr_set[di]) {
+    if (!g_ug_attr[dev][di]) {
       if (cudaFuncSetAttribute(ug_cross_attn_kernel<D>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess)
         return JCA_ERR_CUDA;
-      info->attr_set[di] = true;
+      g_ug_attr[dev][di] = true;
     }
   }
   CUtensorMap tmQ, tmK, tmV;
-  if (!ug_make_map<D>(&tmQ, q, B * T_out, a.H, a.rows_q) ||
-      !ug_make_map<D>(&tmK, k, B * T_in, a.H, a.keys) ||
-      !ug_make_map<D>(&tmV, v, B * T_in, a.H, a.keys))
+  if (!make_rows_map_bf16(&tmQ, q, B * T_out, a.H, D, a.rows_q) ||
+      !make_rows_map_bf16(&tmK, k, B * T_in, a.H, D, a.keys) ||
+      !make_rows_map_bf16(&tmV, v, B * T_in, a.H, D, a.keys))
     return JCA_ERR_CUDA;
-  const int64_t grid64 = a.n_units < info->sms ? a.n_units : info->sms;
+  const int64_t grid64 = a.n_units < sms ? a.n_units : sms;
   ug_cross_attn_kernel<D><<<(int)grid64, kUgThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK, tmV, a);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }
