@@ -120,3 +120,41 @@ def test_planted_mask_mistakes_are_caught():
         finally:
             ou.ug_mask = orig
         assert np.max(np.abs(wrong - good)) > 1e-6
+
+
+def _brute(b, c_u, n_u):
+    """Pure-Python restatement (math.exp): output i of a sample reads inputs [0, n_u) if i < c_u,
+    else all inputs; no key -> 0; plus the residual."""
+    q, k, v, r = (t.double().tolist() for t in (b.q, b.k, b.v, b.residual))
+    out = np.zeros((b.B, b.T_out, b.H, b.d))
+    for s in range(b.B):
+        for i in range(b.T_out):
+            keys = list(range(min(n_u, b.T_in) if i < c_u else b.T_in))
+            for h in range(b.H):
+                row = [0.0] * b.d
+                if keys:
+                    sc = [b.scale * math.fsum(x * y for x, y in zip(q[s][i][h], k[s][j][h]))
+                          for j in keys]
+                    top = max(sc)
+                    w = [math.exp(x - top) for x in sc]
+                    tot = math.fsum(w)
+                    row = [math.fsum(wj / tot * v[s][j][h][c] for wj, j in zip(w, keys))
+                           for c in range(b.d)]
+                for c in range(b.d):
+                    out[s, i, h, c] = row[c] + r[s][i][h][c]
+    return out
+
+
+def test_matches_brute_force_random_shapes():
+    rng = np.random.default_rng(123)
+    for case in range(24):
+        B = int(rng.integers(1, 4))
+        T_out = int(rng.integers(1, 6))
+        T_in = int(rng.integers(1, 7))
+        c_u = int(rng.integers(0, T_out + 1))
+        n_u = int(rng.integers(0, T_in + 1))
+        H = int(rng.integers(1, 3))
+        d = int(rng.choice([4, 8]))
+        b = synth.custom_ug(B, T_out, T_in, c_u, n_u, H, d, seed=1000 + case)
+        got = ou.ug_cross_attn(b.q, b.k, b.v, c_u, n_u, b.scale, residual=b.residual)
+        assert np.max(np.abs(got - _brute(b, c_u, n_u))) < 1e-12, (B, T_out, T_in, c_u, n_u)
