@@ -10,8 +10,8 @@
 //
 // The array is a file-scope static __device__ object: every GPU that loads the library holds
 // kNoAllocScratchBytes of it until the process exits. Host code cannot use its name as a device
-// address; the first call on each device looks the address up with cudaGetSymbolAddress (with
-// that device current) and caches it.
+// address; jca_noalloc_prepare(), or else the first call on each device, looks the address up with
+// cudaGetSymbolAddress (with that device current) and caches it.
 #include <climits>
 #include <cstdint>
 #include <mutex>
@@ -51,6 +51,11 @@ int scratch_address(void** out) {
 }  // namespace jca
 
 extern "C" size_t jca_noalloc_scratch_bytes(void) { return jca::kNoAllocScratchBytes; }
+
+extern "C" int jca_noalloc_prepare(void) {
+  void* scratch = nullptr;
+  return jca::scratch_address(&scratch);
+}
 
 extern "C" int jagged_cand_attn_fwd_noalloc(const void* q, const void* k, const void* v,
                                             void* out, int out_fp32, const void* offsets,

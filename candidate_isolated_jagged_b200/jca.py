@@ -66,6 +66,9 @@ _SIGNATURES = {
                               c_i64, c_i32, c_i32, c_f32, c_i64, c_f32, c_i32, c_vp, c_sz, c_vp,
                               c_vp]),
     "jca_noalloc_scratch_bytes": (c_sz, []),
+    "jca_noalloc_prepare": (c_i32, []),
+    "jca_user_tile_cost": (c_i64, [c_i64, c_i64]),
+    "jca_shard_users": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_vp, c_vp]),
     "jagged_cand_attn_fwd_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp,
                                              c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp,
                                              c_vp]),
@@ -271,21 +274,54 @@ def cand_only_attn_run(cand_q, own_k, own_v, hist_k, hist_v, hist_seg, out, B: i
         workspace.numel(), _ptr(status), _stream(stream)), "cand_only_attn_run")
 
 
+def jca_noalloc_prepare() -> int:
+    """Caches the static scratch array's device address for the current device (call it before
+    capturing a stream that will hold jagged_cand_attn_fwd_noalloc)."""
+    return _check(lib().jca_noalloc_prepare(), "jca_noalloc_prepare")
+
+
 def jagged_cand_attn_fwd_noalloc(q, k, v, out, offsets, candidate_start=None, seg=None,
                                  scale: float = 0.0, status: Optional[torch.Tensor] = None,
                                  stream=None) -> int:
     """jagged_cand_attn_fwd for callers that cannot allocate device memory at call time: the
     library uses its own fixed 8 MiB static scratch array instead of a caller workspace (see
-    include/jca.h for the size limit and the sharing rules)."""
+    include/jca.h for the size limit and the sharing rules). The caller passes the int32 status
+    word too (device memory it owns), so that nothing here allocates either; only the C call is
+    allocation-free when called some other way."""
     T, H, d = q.shape
     B = offsets.numel() - 1
     if status is None:
-        status = new_status(q.device)
+        raise ValueError("jagged_cand_attn_fwd_noalloc needs a caller-owned status tensor "
+                         "(new_status() once, outside the allocation-free region)")
     out_fp32 = 1 if out.dtype == torch.float32 else 0
     return _check(lib().jagged_cand_attn_fwd_noalloc(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), _ptr(candidate_start),
         _ptr(seg), B, T, H, d, float(scale), _idx_bits(offsets), _ptr(status), _stream(stream)),
         "jagged_cand_attn_fwd_noalloc")
+
+
+def shard_users(row_lengths, n_keys, n_shards: int):
+    """Host-side LPT split of a batch's users over n_shards GPUs (jca_shard_users).
+
+    row_lengths, n_keys: per-user rows and segment-1 keys (array-likes of int). Returns
+    (shard [B] int32, load [n_shards] int64) as numpy arrays."""
+    import numpy as np
+    rl = np.ascontiguousarray(np.asarray(row_lengths, dtype=np.int64))
+    nk = np.ascontiguousarray(np.asarray(n_keys, dtype=np.int64))
+    if rl.shape != nk.shape or rl.ndim != 1:
+        raise ValueError("row_lengths and n_keys must be 1-D arrays of the same length")
+    shard = np.empty(rl.shape[0], dtype=np.int32)
+    load = np.empty(int(n_shards), dtype=np.int64)
+    _check(lib().jca_shard_users(rl.ctypes.data if rl.size else None,
+                                 nk.ctypes.data if nk.size else None, rl.shape[0], int(n_shards),
+                                 shard.ctypes.data if shard.size else None, load.ctypes.data),
+           "jca_shard_users")
+    return shard, load
+
+
+def user_tile_cost(row_length: int, n_keys: int) -> int:
+    """Tile cost of one user (jca_user_tile_cost)."""
+    return int(lib().jca_user_tile_cost(int(row_length), int(n_keys)))
 
 
 def jca_rope_positions(seg, offsets, positions, history_end: int, status, stream=None) -> int:

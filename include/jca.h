@@ -184,6 +184,11 @@ int jagged_cand_attn_fwd(const void* q, const void* k, const void* v, void* out,
  *                          any number of times after one plan, as long as `workspace` and the
  *                          layout arguments (seg, B, T, H, d_head) are the same as at plan time.
  * Arguments, errors and workspace size are as for jagged_cand_attn_fwd.
+ * Sharing a workspace: the attention kernel claims its work items at run time from a counter in
+ * the workspace (zeroed by the plan, reset by the kernel's last block for the next run). Calls that
+ * use one workspace must therefore not overlap on the GPU: order them on one stream (or with
+ * events). Runs that may overlap, e.g. on two streams, each need their own workspace (and plan).
+ * The same holds for every entry point below that takes a workspace.
  */
 int jagged_cand_attn_plan(const void* offsets, const void* candidate_start, const int8_t* seg,
                           int64_t B, int64_t T, int H, int d_head, int idx_bits, void* workspace,
@@ -245,8 +250,10 @@ int cand_only_attn_run(const void* cand_q, const void* own_k, const void* own_v,
  *   Size limit: when jca_workspace_bytes(B, T, H, d_head) exceeds jca_noalloc_scratch_bytes(),
  *   the call returns JCA_ERR_SCRATCH_LIMIT before enqueuing anything (use jagged_cand_attn_fwd
  *   with a workspace then). Roughly: T + 44 B + 16 H (T/128 + B + 1) bytes must fit in 8 MiB.
- *   First call per device: it looks up the array's device address (cudaGetSymbolAddress, with
- *   that device current) and caches it; make that first call before any stream capture.
+ *   First use per device: the array's device address is looked up (cudaGetSymbolAddress, with
+ *   that device current) and cached, by jca_noalloc_prepare() or else by the first call. Call
+ *   jca_noalloc_prepare() with each device current before any stream capture (inside a capture
+ *   the lookup may fail, and the call then returns JCA_ERR_CUDA).
  *   Sharing: all calls on a device use the same array, which keeps the last call's contents (no
  *   part of it needs to start at zero). Calls whose execution overlaps on the GPU — on different
  *   streams without ordering between them, or from several host threads — race on it; order them
@@ -254,10 +261,39 @@ int cand_only_attn_run(const void* cand_q, const void* own_k, const void* own_v,
  */
 size_t jca_noalloc_scratch_bytes(void);
 
+/* Looks up and caches the static array's device address for the current device, so that later
+ * jagged_cand_attn_fwd_noalloc calls on it do no CUDA runtime call beyond their launches.
+ * Returns JCA_OK, or JCA_ERR_CUDA when the lookup fails (no usable device). Enqueues nothing. */
+int jca_noalloc_prepare(void);
+
 int jagged_cand_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
                                  int out_fp32, const void* offsets, const void* candidate_start,
                                  const int8_t* seg, int64_t B, int64_t T, int H, int d_head,
                                  float scale, int idx_bits, int32_t* status, jca_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Several GPUs: users are independent (no position reads across a user boundary: 候选隔离注意力掩码,
+ * section 段 ID：掩码的表达方式; 'HSTU scale' tutorial, section 手算 padding 的浪费与 offset), so one
+ * batch's users are split over the GPUs with no exchange in the forward pass; each GPU plans and
+ * runs its own users and keeps its outputs. These two calls are HOST functions on HOST memory: they
+ * enqueue nothing and need no GPU.
+ * ------------------------------------------------------------------------------------------- */
+
+/* Tile cost of one user as the attention kernel sees it: ceil(row_len / 128) query tiles times
+ * max(1, ceil(n_keys / 128)) key tiles (n_keys = the user's segment-1 keys); 0 for an empty row. */
+int64_t jca_user_tile_cost(int64_t row_len, int64_t n_keys);
+
+/* Longest-processing-time-first split of B users over n_shards GPUs: users in order of decreasing
+ * jca_user_tile_cost (ties in user order), each to the least-loaded shard so far (ties to the lowest
+ * shard index). Deterministic, so every rank computes the same split from the same lengths. The
+ * largest shard load stays within Graham's list-scheduling bound, total / n_shards + (1 - 1 /
+ * n_shards) * max cost, and within 4/3 - 1/(3 n_shards) of the best split.
+ *   row_len [B], n_keys [B]  int64, host memory, read (0 <= n_keys <= row_len).
+ *   shard   [B] int32, host memory, written: the shard of each user, in [0, n_shards).
+ *   load    [n_shards] int64, host memory, written (nullable): total cost per shard.
+ * Errors: JCA_ERR_SHAPE (B < 0, n_shards < 1, a negative length, n_keys > row_len), JCA_ERR_NULL. */
+int jca_shard_users(const int64_t* row_len, const int64_t* n_keys, int64_t B, int n_shards,
+                    int32_t* shard, int64_t* load);
 
 /* ---------------------------------------------------------------------------------------------
  * Right-anchored rotary position embedding (候选隔离注意力掩码, section 位置编码：候选共用一个位置):

@@ -8,9 +8,10 @@ roundoff 2^-9, and the rounding enters every gradient linearly, so the error sca
 gradient itself. An fp64 computation with only that rounding added differs from the exact
 gradients by a relative L2 of 1.5e-3 to 2e-3 and a max-abs of 0.2 % to 0.4 % of the largest
 gradient on the 256-user workload (up to 1.5e-2 where 4 history keys collect the gradient of 68
-queries and |dV| reaches 9). The bar is therefore max-abs <= 1e-2 * max(1, max |ref|) and relative
-L2 <= 1e-2 (fp32 gradient outputs). The log-sum-exp is fp32 arithmetic on exact bf16 products:
-max-abs <= 1e-3.
+queries and |dV| reaches 9). The bar is therefore the spec relative L2 of 5e-3 (2.5x the
+modelled rounding) with a max-abs of 1e-2 * max(1, max |ref|): the absolute 1e-2 for gradients of
+order one, scaled with the gradient where the bf16 rounding of P and dS scales with it (fp32
+gradient outputs). The log-sum-exp is fp32 arithmetic on exact bf16 products: max-abs <= 1e-3.
 """
 
 import numpy as np
@@ -26,7 +27,7 @@ from helpers import FullRun, assert_close, dev
 pytestmark = pytest.mark.gpu
 
 GRAD_MAX_ABS = 1e-2
-GRAD_REL_L2 = 1e-2
+GRAD_REL_L2 = 5e-3
 
 
 def _fwd_bwd(r: FullRun, dout, out_fp32=True, grad_fp32=True):

@@ -4,8 +4,9 @@ It serves callers that cannot allocate device memory when they call (fixed-memor
 plugins handed only their tensors, code that must avoid cudaMalloc's implicit synchronisation):
 the library keeps the scratch in its own static device array. These tests call it through the C
 ABI, twice in a row on the same array, and compare each result with jagged_cand_attn_fwd given a
-caller workspace, under the tolerance of the other parity tests. This file is collected last so
-that a run stopping at its first failure has already run every other test.
+caller workspace, under the tolerance of the other parity tests, and with the CPU oracle directly.
+This file is collected last so that a run stopping at its first failure has already run every
+other test.
 """
 
 import numpy as np
@@ -51,6 +52,18 @@ def test_no_alloc_matches_workspace_call_twice(name, out_fp32):
     for got in (first, second):
         assert_close(got, ref, f"no-alloc {name}")
     assert torch.equal(first, second)
+    if out_fp32:
+        assert_close(first, r.reference(), f"no-alloc {name} vs oracle")
+
+
+def test_no_alloc_prepare_then_call():
+    # jca_noalloc_prepare caches the array's address for the current device (what a caller does
+    # before capturing a stream); calls after it give the same result as before, bit for bit.
+    r = FullRun(synth.three_users())
+    before = _no_alloc(r, True)
+    assert jca.jca_noalloc_prepare() == 0
+    after = _no_alloc(r, True)
+    assert torch.equal(before, after)
 
 
 def test_no_alloc_after_a_different_problem():
@@ -67,14 +80,13 @@ def test_no_alloc_rejects_problems_beyond_the_array():
     assert limit == 8 << 20
     rows = 1 << 30                        # segment IDs alone would need 1 GiB of scratch
     assert jca.jca_workspace_bytes(1, rows, 1, 16) > limit
-    p = ctypes_addr = 0x100000
     L = jca.lib()
     import ctypes
     st = jca.new_status(dev())
-    code = L.jagged_cand_attn_fwd_noalloc(
-        ctypes.c_void_p(p), ctypes.c_void_p(p), ctypes.c_void_p(p), ctypes.c_void_p(p), 1,
-        ctypes.c_void_p(ctypes_addr), ctypes.c_void_p(ctypes_addr), None, 1, rows, 1, 16, 0.0, 64,
-        ctypes.c_void_p(st.data_ptr()), None)
+    # No tensor is passed: the size check comes first, so the call must return before it would
+    # look at any pointer (and, were that check ever lost, stop at the null-pointer check).
+    code = L.jagged_cand_attn_fwd_noalloc(None, None, None, None, 1, None, None, None, 1, rows, 1,
+                                          16, 0.0, 64, ctypes.c_void_p(st.data_ptr()), None)
     assert code == -9
     assert "static array" in jca.status_string(code)
     assert int(st.item()) == 0
