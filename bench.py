@@ -231,12 +231,32 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         import torch.distributed as dist  # noqa: F811
 
     peaks = load_peaks()
-    batch = synth.users256()
+    shard_info = None
+    if args.shard == "users":
+        # One global batch split over the ranks by users (LPT over tile cost); each rank draws and
+        # computes only its own users, and its outputs stay on its GPU.
+        G = args.global_users or 256 * world
+        hist = synth.lognormal_history_lengths(G, 0)
+        shard, load = jca.shard_users(hist + 68, hist + 4, world)
+        mine = np.nonzero(shard == rank)[0]
+        batch = synth.users_batch(hist, mine, 4, 64, 8, 128, seed=0, name=f"users{G}_shard{rank}")
+        g_pairs = metrics.allowed_pairs_from_counts(hist + 4, np.full(G, 64))
+        job_flops = metrics.effective_flops(g_pairs, 8, 128)
+        job_tokens = int((hist + 68).sum())
+        shard_info = {"global_users": int(G), "users_this_rank": int(mine.size),
+                      "tile_cost_per_rank": [int(x) for x in load],
+                      "imbalance": float(load.max() / max(load.mean(), 1e-30))}
+        scaling = "weak" if args.global_users is None else "strong"
+    else:
+        batch = synth.users256()
+        scaling = "weak"
     B, T, H, d = batch.B, batch.T, batch.H, batch.d
     n1 = batch.prefix + batch.hist_real
     pairs = metrics.allowed_pairs_from_counts(n1, batch.n_cand)
     flops = metrics.effective_flops(pairs, H, d)
     valid_tokens = int(batch.row_lengths.sum()) if batch.valid is None else int(batch.valid.sum())
+    if shard_info is None:   # replicas: every rank runs its own copy of the batch
+        job_flops, job_tokens = world * flops, world * valid_tokens
 
     stream = torch.cuda.current_stream(dev)
     q, k, v = (t.to(dev) for t in (batch.q, batch.k, batch.v))
@@ -283,7 +303,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     kernel_ms = float(np.mean([a.elapsed_time(b) for a, b in kev]))
     elapsed_ms, kernel_ms = max_over_ranks([elapsed_ms, kernel_ms], dist, dev)
     ms_per_step = elapsed_ms / args.steps
-    value = weak_scaling_value(flops, world, args.steps, elapsed_ms) / 1e12
+    value = job_flops * args.steps / (elapsed_ms / 1e3) / 1e12
 
     # ---- end to end through the public API: host inputs in, host output back ----
     # Every step copies its inputs from pinned host memory and reads its output back. The copies
@@ -345,13 +365,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     e2e_ms = max_over_ranks([e2e_run(e2e_steps)], dist, dev)[0]
     jca.check_status(status, "end-to-end")
     assert torch.equal(out_hs[(e2e_steps - 1) & 1], out.cpu()), "end-to-end output differs"
-    e2e_value = weak_scaling_value(flops, world, e2e_steps, e2e_ms) / 1e12
+    e2e_value = job_flops * e2e_steps / (e2e_ms / 1e3) / 1e12
 
-    achieved = flops / (kernel_ms / 1e3) / 1e12
+    # Per GPU: this rank's work over its own kernel time (replicas), or the job's average work per
+    # rank over the slowest rank's kernel time (users split over the ranks).
+    achieved = (flops if shard_info is None else job_flops / world) / (kernel_ms / 1e3) / 1e12
     roofline = {
         "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
         "frac": achieved / peaks["bf16_tflops"],
-        "traffic": profiled_traffic("attn_users256_d128"),
+        "traffic": profiled_traffic("attn_users256_d128") if shard_info is None else None,
         "kernel": "jagged_attn_kernel<128>", "kernel_ms": kernel_ms,
         "peak_source": f"{peaks['source']} bf16_tflops (burst)",
         "frac_of_sustained": achieved / peaks["bf16_tflops_sustained"],
@@ -359,16 +381,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "algorithmic_bytes_per_launch": metrics.full_attention_bytes(T, H, d),
     }
 
+    if shard_info is None:
+        workload = WORKLOAD
+        parallelism = f"dp{world}: one batch per rank (replicas), no collective"
+    else:
+        workload = (f"users{shard_info['global_users']}: {shard_info['global_users']} users drawn "
+                    "like users256 (lognormal histories, median 280, clipped to [0, 4096], 4 prefix"
+                    " + 64 candidates, H=8, d_head=128, per-user seeded bf16 N(0,1))")
+        parallelism = (f"dp{world}: the batch's users split over the ranks (LPT over tile cost), "
+                       "outputs stay sharded, no collective")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": scaling, "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "rows": T, "valid_tokens": valid_tokens,
+        "config": {"workload": workload, "rows": T, "valid_tokens": valid_tokens,
                    "allowed_pairs": pairs, "effective_flops_per_step": flops,
+                   "job_effective_flops_per_step": job_flops,
                    "l2": "inputs (Q/K/V 837 MB) larger than L2 (126 MB); no flush",
-                   "parallelism": f"dp{world}: users sharded by batch, no collective"},
-        "tokens_per_s": weak_scaling_value(valid_tokens, world, args.steps, elapsed_ms),
+                   "parallelism": parallelism},
+        "tokens_per_s": job_tokens * args.steps / (elapsed_ms / 1e3),
         "pct_of_bf16_peak": 100.0 * value / (world * peaks["bf16_tflops"]),
         "roofline": roofline,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
@@ -377,6 +409,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": sampler.summary(),
     }
+    if shard_info is not None:
+        line["config"]["shard"] = shard_info
     del q_h, k_h, v_h, out_hs, bufs
 
     if rank == 0 and world == 1 and not args.no_extras:
@@ -719,6 +753,12 @@ def main():
                                        "ug_sep"],
                     default=None,
                     help="run one extra section alone on one GPU and print its result (profiling)")
+    ap.add_argument("--shard", choices=["replicas", "users"], default="replicas",
+                    help="replicas: every rank runs its own 256-user batch; users: one global "
+                         "batch split over the ranks by users (LPT), outputs stay sharded")
+    ap.add_argument("--global-users", type=int, default=None,
+                    help="--shard users: users in the global batch (default 256 per rank: weak "
+                         "scaling; a fixed number makes it strong scaling)")
     ap.add_argument("--users", type=int, default=256,
                     help="--only backward: use the first N users of the 256-user workload")
     args = ap.parse_args()

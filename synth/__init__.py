@@ -18,6 +18,8 @@ from .workloads import (  # noqa: F401
     custom_batch,
     custom_cand_only,
     users256_history_lengths,
+    lognormal_history_lengths,
+    users_batch,
     StackBatch,
     custom_stack,
     upstream_grad,

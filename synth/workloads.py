@@ -264,6 +264,43 @@ def users256_history_lengths(seed: int = 0) -> np.ndarray:
     return n
 
 
+def lognormal_history_lengths(n_users: int, seed: int = 0) -> np.ndarray:
+    """History lengths of a batch of n_users users drawn like the 256-user workload:
+    floor(lognormal(ln 280, sigma=1)) clipped to [0, 4096], users whose index is a multiple of 64
+    empty and user 1 at the 4096 cap."""
+    rng = np.random.default_rng(seed)
+    n = np.floor(rng.lognormal(mean=np.log(280.0), sigma=1.0, size=int(n_users)))
+    n = np.clip(n, 0, 4096).astype(np.int64)
+    n[::64] = 0
+    if n_users > 1:
+        n[1] = 4096
+    return n
+
+
+def users_batch(hist_lengths: Sequence[int], users: Sequence[int], prefix: int, n_cand: int,
+                H: int, d: int, seed: int, name: str = "users") -> Batch:
+    """The rows of the listed users of a larger batch (histories ``hist_lengths``, no padding), as a
+    batch of their own, in the order listed. Each user's Q, K, V are drawn, in that order, from a
+    generator of its own, ``torch.Generator().manual_seed(seed * 1000003 + user)``, so that a
+    process that owns some of the users draws only theirs and every process draws the same rows
+    for the same user."""
+    users = [int(u) for u in users]
+    n = np.asarray(hist_lengths, dtype=np.int64)[users] if users else np.zeros(0, np.int64)
+    B = len(users)
+    pre = np.full(B, int(prefix), dtype=np.int64)
+    nc = np.full(B, int(n_cand), dtype=np.int64)
+    row_lengths = pre + n + nc
+    qs, ks, vs = [], [], []
+    for u, L in zip(users, row_lengths):
+        gen = torch.Generator().manual_seed(int(seed) * 1000003 + u)
+        qs.append(_draw(gen, int(L), H, d))
+        ks.append(_draw(gen, int(L), H, d))
+        vs.append(_draw(gen, int(L), H, d))
+    cat = (lambda xs: torch.cat(xs) if xs else torch.zeros(0, H, d, dtype=torch.bfloat16))
+    return Batch(name, row_lengths, pre + n, None, cat(qs), cat(ks), cat(vs), int(H), int(d),
+                 int(seed), pre, n.copy(), n.copy(), nc)
+
+
 def users256(H: int = 8, d: int = 128) -> Batch:
     """256 users, lognormal histories (median 280), 4 prefix tokens, 64 candidates each;
     H=8, d=128, seed 0."""
