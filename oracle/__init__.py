@@ -5,7 +5,7 @@ package. It computes, slowly and in fp64, what the jagged candidate-isolated att
 computes, restating the source pages' rules; it imports nothing from the CUDA package.
 """
 
-from . import jagged_oracle, brute, rope, stack, backward, variants, ug_sep  # noqa: F401
+from . import jagged_oracle, brute, rope, stack, backward, variants, ug_sep, seqpack  # noqa: F401
 from .jagged_oracle import (  # noqa: F401
     offsets_from_lengths,
     split_by_offsets,

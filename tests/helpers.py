@@ -112,3 +112,17 @@ def sample_rows(offsets, per_user=3, seed=0, extra=()):
         rows.update({s, e - 1})
         rows.update(int(x) for x in rng.integers(s, e, size=per_user))
     return np.asarray(sorted(rows), dtype=np.int64)
+
+
+def seqpack_layout(batch):
+    """The rows of a serving-layout batch rearranged for training with candidate packing: every
+    user's prefix + history run first (split at hist_offsets), then every user's candidate run
+    (split at cand_offsets, relative to the candidate block). Returns (perm, hist_offsets,
+    cand_offsets): packed row i holds serving row perm[i]."""
+    off = oracle.offsets_from_lengths(batch.row_lengths)
+    cs = np.asarray(batch.cand_start, dtype=np.int64)
+    L = np.asarray(batch.row_lengths, dtype=np.int64)
+    hist = [np.arange(off[b], off[b] + cs[b]) for b in range(batch.B)]
+    cand = [np.arange(off[b] + cs[b], off[b + 1]) for b in range(batch.B)]
+    perm = np.concatenate(hist + cand).astype(np.int64) if batch.B else np.zeros(0, np.int64)
+    return perm, oracle.offsets_from_lengths(cs), oracle.offsets_from_lengths(L - cs)
