@@ -1315,6 +1315,43 @@ extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const v
                             Th, H, d_head, scale, workspace, workspace_bytes, status, stream);
 }
 
+extern "C" size_t jca_seqpack_workspace_bytes(int64_t B, int64_t Th, int64_t Nc, int H,
+                                              int d_head) {
+  if (B < 0 || Th < 0 || Nc < 0 || H < 1 || !head_dim_ok(d_head)) return 0;
+  return seqpack_layout(B, Th + Nc, H).total;
+}
+
+extern "C" int jagged_cand_attn_seqpack_fwd(const void* q, const void* k, const void* v,
+                                            void* out, int out_fp32, float* lse,
+                                            const void* hist_offsets, const void* cand_offsets,
+                                            const int8_t* seg, int64_t B, int64_t Th, int64_t Nc,
+                                            int H, int d_head, float scale, int idx_bits,
+                                            void* workspace, size_t workspace_bytes,
+                                            int32_t* status, jca_stream_t stream) {
+  if (Th < 0 || Nc < 0 || 2 * B >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  const int64_t T = Th + Nc;
+  int rc = check_sizes(idx_bits, d_head, 2 * B, T, T, H);
+  if (rc) return rc;
+  if (!status || !hist_offsets || !cand_offsets) return JCA_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !out)) return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+                (lse && !aligned(lse, 4))))
+    return JCA_ERR_ALIGN;
+  if (!workspace) return JCA_ERR_NULL;
+  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+  const SeqpackLayout S = seqpack_layout(B, T, H);
+  if (workspace_bytes < S.total) return JCA_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_seqpack_plan(hist_offsets, cand_offsets, seg, B, Th, Nc, H, idx_bits,
+                          static_cast<char*>(workspace), S.base, S.q_off2, status,
+                          st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  // The 2B query runs go through the attention kernel as 2B "users" of the packed matrix; without
+  // a caller's segment IDs the kernel reads the ones the plan wrote into the workspace.
+  return run_full(q, k, v, out, out_fp32, lse, seg, 2 * B, T, H, d_head, scale, workspace,
+                  workspace_bytes, status, stream);
+}
+
 extern "C" const char* jca_status_string(int code) {
   switch (code) {
     case JCA_OK: return "ok";

@@ -63,6 +63,7 @@ struct BwdArgs {
   const float* lse2;       // [H][T]: log2-units log-sum-exp of each row; +inf = row sees no key
   const float* dsum;       // [H][T]: rowsum(dO * O)
   const int4* items;
+  const int2* items2;      // dKV only, or null: a second query run {row start, rows} per item
   const int32_t* n_items;
   int32_t* status;
   int64_t T;
@@ -114,10 +115,22 @@ struct BCfg {
 };
 
 // One unit of work: `orows` outer rows starting at `orow0` for head h, against the inner rows
-// [in_lo, in_lo + in_len) walked in tiles of 128.
+// [in_lo, in_lo + in_len) and then [in_lo2, in_lo2 + in_len2), walked in tiles of 128 (n_in1
+// tiles over the first run, n_in in all). The second run is empty except for dKV units of the
+// candidate-packed layout, where a user's candidate queries sit apart from its history.
 struct Unit {
-  int orow0, orows, h, in_lo, in_len, holes, n_in;
+  int orow0, orows, h, in_lo, in_len, holes, n_in, in_lo2, in_len2, n_in1;
 };
+
+// First row and valid rows of inner tile i of a unit.
+__device__ __forceinline__ int in_row(const Unit& u, int i) {
+  return i < u.n_in1 ? u.in_lo + i * kTileN : u.in_lo2 + (i - u.n_in1) * kTileN;
+}
+
+__device__ __forceinline__ int in_valid(const Unit& u, int i) {
+  return i < u.n_in1 ? min(kTileN, u.in_len - i * kTileN)
+                     : min(kTileN, u.in_len2 - (i - u.n_in1) * kTileN);
+}
 
 // Units of an item. dQ items are the forward's work items (up to 256 query rows: two units);
 // dKV items hold one key tile.
@@ -128,7 +141,7 @@ __device__ __forceinline__ int unit_count(int4 v) {
 }
 
 template <int MODE>
-__device__ __forceinline__ Unit decode_unit(int4 v, int t) {
+__device__ __forceinline__ Unit decode_unit(int4 v, int t, const int2* items2, int it) {
   Unit u;
   u.h = v.y >> 9;
   const int rows = v.y & 511;
@@ -142,7 +155,15 @@ __device__ __forceinline__ Unit decode_unit(int4 v, int t) {
     u.in_len = v.w;
     u.holes = 0;
   }
-  u.n_in = (u.in_len + kTileN - 1) / kTileN;
+  u.n_in1 = (u.in_len + kTileN - 1) / kTileN;
+  u.in_lo2 = 0;
+  u.in_len2 = 0;
+  if (MODE == kModeDKV && items2 != nullptr) {
+    const int2 w = items2[it];
+    u.in_lo2 = w.x;
+    u.in_len2 = w.y;
+  }
+  u.n_in = u.n_in1 + (u.in_len2 + kTileN - 1) / kTileN;
   return u;
 }
 
@@ -161,7 +182,7 @@ __device__ void bwd_producer(const CUtensorMap* tmO1, const CUtensorMap* tmO2,
     const int4 raw = a.items[it];
     const int nu = unit_count<MODE>(raw);
     for (int t = 0; ok && t < nu; ++t) {
-      const Unit u = decode_unit<MODE>(raw, t);
+      const Unit u = decode_unit<MODE>(raw, t, a.items2, it);
       if (u.n_in == 0) continue;
       ok = mbar_wait(bars + 8 * C::B_OUTEMPTY, (u_count & 1) ^ 1, abort_flag, a.status);
       if (!ok) break;
@@ -181,7 +202,7 @@ __device__ void bwd_producer(const CUtensorMap* tmO1, const CUtensorMap* tmO2,
         if (!ok) break;
         mbar_arrive_expect_tx(bars + 8 * (C::B_INFULL + s), 2 * C::TILE_BYTES);
         const uint32_t dst = sbase + C::OFF_IN + s * 2 * C::TILE_BYTES;
-        const int row = u.in_lo + i * kTileN;
+        const int row = in_row(u, i);
 #pragma unroll
         for (int c = 0; c < C::NBLK; ++c) {
           tma_load_3d(dst + c * C::BLK_BYTES, tmI1, bars + 8 * (C::B_INFULL + s), c * C::BOX_X,
@@ -236,7 +257,7 @@ struct HalfStep {
 };
 
 __device__ __forceinline__ bool next_half(const Unit& u, HalfStep& h) {
-  const int tile_valid = min(kTileN, u.in_len - h.i * kTileN);
+  const int tile_valid = in_valid(u, h.i);
   if (h.hh == 0 && tile_valid > kHalf) {
     h.hh = 1;
   } else {
@@ -244,7 +265,7 @@ __device__ __forceinline__ bool next_half(const Unit& u, HalfStep& h) {
     ++h.i;
     h.hh = 0;
   }
-  h.valid = min(kHalf, min(kTileN, u.in_len - h.i * kTileN) - h.hh * kHalf);
+  h.valid = min(kHalf, in_valid(u, h.i) - h.hh * kHalf);
   return true;
 }
 
@@ -303,13 +324,13 @@ __device__ void bwd_mma(const BwdArgs& a, uint32_t sbase, uint32_t bars, uint32_
     const int4 raw = a.items[it];
     const int nu = unit_count<MODE>(raw);
     for (int t = 0; ok && t < nu; ++t) {
-      const Unit u = decode_unit<MODE>(raw, t);
+      const Unit u = decode_unit<MODE>(raw, t, a.items2, it);
       if (u.n_in == 0) continue;
       ok = mbar_wait(bars + 8 * C::B_OUTFULL, u_count & 1, abort_flag, a.status);
       if (!ok) break;
       ++u_count;
       // One half step of lookahead: S/dP of step t + 1 are issued before the TS MMAs of step t.
-      HalfStep cur{0, 0, min(kHalf, min(kTileN, u.in_len))};
+      HalfStep cur{0, 0, min(kHalf, in_valid(u, 0))};
       uint32_t cur_stage = g % kBwdStages;
       ok = mbar_wait(bars + 8 * (C::B_INFULL + (int)cur_stage), (g / kBwdStages) & 1, abort_flag,
                      a.status);
@@ -441,7 +462,7 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
     const int4 raw = a.items[it];
     const int nu = unit_count<MODE>(raw);
     for (int t = 0; ok && t < nu; ++t) {
-      const Unit u = decode_unit<MODE>(raw, t);
+      const Unit u = decode_unit<MODE>(raw, t, a.items2, it);
       const bool row_ok = r < u.orows;
       const int64_t row = (int64_t)u.orow0 + (row_ok ? r : 0);
       const int seg = row_ok ? (int)a.seg[row] : 0;
@@ -465,14 +486,14 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
       // that those columns get P = 0), stored negated in shared memory (warps of column half 0
       // fill -lse2, half 1 -D). The value for tile i + 1 is fetched while tile i is computed.
       auto col_stat = [&](int i) -> float {
-        const int v = min(kTileN, u.in_len - i * kTileN);
+        const int v = in_valid(u, i);
         if (r >= v) return ch == 0 ? -INFINITY : 0.f;
-        const size_t qs = (size_t)u.h * (size_t)T + (size_t)((int64_t)u.in_lo + i * kTileN + r);
+        const size_t qs = (size_t)u.h * (size_t)T + (size_t)((int64_t)in_row(u, i) + r);
         return ch == 0 ? -a.lse2[qs] : -a.dsum[qs];
       };
       float next_stat = (MODE == kModeDKV && u.n_in > 0) ? col_stat(0) : 0.f;
       for (int i = 0; i < u.n_in; ++i) {
-        const int valid = min(kTileN, u.in_len - i * kTileN);
+        const int valid = in_valid(u, i);
         float* cl = cols + (cols_n & 1) * 2 * kTileN;   // dKV: -lse2 | -dsum of the 128 columns
         if (MODE == kModeDKV) {
           cl[ch * kTileN + r] = next_stat;
@@ -503,7 +524,7 @@ __device__ void bwd_compute(const BwdArgs& a, uint32_t bars, uint32_t tmem, floa
               // Key columns past the interval or on padding holes are masked.
               const int c = 32 * ch + lane;
               bool keep = lane < cvalid;
-              if (keep && u.holes) keep = a.seg[u.in_lo + i * kTileN + hh * kHalf + c] == 1;
+              if (keep && u.holes) keep = a.seg[in_row(u, i) + hh * kHalf + c] == 1;
               bits = __ballot_sync(0xffffffffu, keep);
             }
             tmem_wait_ld();
@@ -739,7 +760,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const void* __restrict__ 
 // Work queue of the dKV kernel: one item per (user, head, 128-key tile of the history interval),
 // sorted by the number of the user's 128-row query tiles, largest first (counting sort in one
 // block, as the forward's queue). Item = {first key row, (h << 9) | key rows, row start, row
-// length}.
+// length}. With `coff` (the candidate-packed layout) the user's queries are its run
+// [off[b], off[b+1]) plus its candidate run [cbase + coff[b], cbase + coff[b+1]), which goes to
+// items2 = {row start, rows}.
 // ------------------------------------------------------------------------------------------
 template <typename IdxT>
 __global__ void __launch_bounds__(1024) dkv_queue_kernel(const IdxT* __restrict__ off,
@@ -747,7 +770,9 @@ __global__ void __launch_bounds__(1024) dkv_queue_kernel(const IdxT* __restrict_
                                                          const IdxT* __restrict__ hhi, int64_t B,
                                                          int H, int4* __restrict__ items,
                                                          int64_t max_items, int32_t* n_items,
-                                                         int32_t* status) {
+                                                         int32_t* status,
+                                                         const IdxT* __restrict__ coff,
+                                                         int64_t cbase, int2* __restrict__ items2) {
   __shared__ unsigned long long s_cnt[kQueueBuckets];
   __shared__ unsigned long long s_cursor[kQueueBuckets];
   __shared__ unsigned long long s_warp[32];
@@ -761,7 +786,8 @@ __global__ void __launch_bounds__(1024) dkv_queue_kernel(const IdxT* __restrict_
   __syncthreads();
   for (int64_t b = tid; b < B; b += blockDim.x) {
     const long long nk = ((long long)hhi[b] - (long long)hlo[b] + kTileN - 1) / kTileN;
-    const long long nq = ((long long)off[b + 1] - (long long)off[b] + kTileM - 1) / kTileM;
+    long long nq = ((long long)off[b + 1] - (long long)off[b] + kTileM - 1) / kTileM;
+    if (coff) nq += ((long long)coff[b + 1] - (long long)coff[b] + kTileM - 1) / kTileM;
     const int key = (int)min(nq, (long long)(kQueueBuckets - 1));
     if (nk) atomicAdd(&s_cnt[key], (unsigned long long)(nk * H));
   }
@@ -804,7 +830,13 @@ __global__ void __launch_bounds__(1024) dkv_queue_kernel(const IdxT* __restrict_
     const long long s = (long long)off[b], e = (long long)off[b + 1];
     const long long nk = (hi - lo + kTileN - 1) / kTileN;
     if (nk == 0) continue;
-    const long long nq = (e - s + kTileM - 1) / kTileM;
+    long long nq = (e - s + kTileM - 1) / kTileM;
+    long long c0 = 0, c1 = 0;
+    if (coff) {
+      c0 = cbase + (long long)coff[b];
+      c1 = cbase + (long long)coff[b + 1];
+      nq += (c1 - c0 + kTileM - 1) / kTileM;
+    }
     const int key = (int)min(nq, (long long)(kQueueBuckets - 1));
     unsigned long long pos = 0;
     if (lane == 0) pos = atomicAdd(&s_cursor[key], (unsigned long long)(nk * H));
@@ -815,6 +847,7 @@ __global__ void __launch_bounds__(1024) dkv_queue_kernel(const IdxT* __restrict_
       const long long k0 = lo + t * kTileN;
       const int rows = (int)min((long long)kTileN, hi - k0);
       items[pos + (unsigned long long)i] = make_int4((int)k0, (h << 9) | rows, (int)s, (int)(e - s));
+      if (items2) items2[pos + (unsigned long long)i] = make_int2((int)c0, (int)(c1 - c0));
     }
   }
   if (tid == 0) *n_items = (int32_t)s_total;
@@ -859,19 +892,27 @@ int launch_bwd_mode(const BwdArgs& a, const void* o1, const void* o2, const void
 }
 
 // Workspace of the backward pass: the forward's plan (segment IDs, bounds, dQ work queue), then
-// the dKV queue and the transposed row statistics.
+// the dKV queue (with its second query runs for the candidate-packed layout) and the transposed
+// row statistics.
 struct BwdLayout {
-  size_t plan = 0, dkv_items = 0, dkv_n = 0, lse2 = 0, dsum = 0, total = 0;
+  size_t plan = 0, dkv_items = 0, dkv_items2 = 0, dkv_n = 0, lse2 = 0, dsum = 0, total = 0;
   int64_t dkv_max = 0;
 };
 
-BwdLayout bwd_layout(int64_t B, int64_t T, int H) {
+// plan_bytes: size of the forward plan at the start of the workspace; key_rows: rows that can hold
+// history keys (T, or Th for the candidate-packed layout).
+BwdLayout bwd_layout_after(size_t plan_bytes, int64_t B, int64_t T, int64_t key_rows, int H,
+                           bool runs2) {
   BwdLayout L;
-  size_t o = align_up(workspace_layout(B, T, H).total, 256);
+  size_t o = align_up(plan_bytes, 256);
   L.plan = 0;
-  L.dkv_max = (T / kTileN + B + 1) * (int64_t)H;
+  L.dkv_max = (key_rows / kTileN + B + 1) * (int64_t)H;
   L.dkv_items = o;
   o = align_up(o + 16 * (size_t)L.dkv_max, 256);
+  if (runs2) {
+    L.dkv_items2 = o;
+    o = align_up(o + 8 * (size_t)L.dkv_max, 256);
+  }
   L.dkv_n = o;
   o = align_up(o + 16, 256);
   L.lse2 = o;
@@ -882,10 +923,14 @@ BwdLayout bwd_layout(int64_t B, int64_t T, int H) {
   return L;
 }
 
+BwdLayout bwd_layout(int64_t B, int64_t T, int H) {
+  return bwd_layout_after(workspace_layout(B, T, H).total, B, T, T, H, false);
+}
+
 template <int D>
 int launch_backward(const BwdArgs& base_args, const void* out, int out_fp32, const float* lse,
                     int64_t T, void* ws, const WorkspaceLayout& W, const BwdLayout& L,
-                    cudaStream_t st) {
+                    cudaStream_t st, bool runs2 = false) {
   char* w = static_cast<char*>(ws);
   const int64_t n = T * base_args.H;
   const int64_t want = (n + 255) / 256;
@@ -900,10 +945,12 @@ int launch_backward(const BwdArgs& base_args, const void* out, int out_fp32, con
   a.dsum = reinterpret_cast<const float*>(w + L.dsum);
   // Keys of segment 1: dK, dV.
   a.items = reinterpret_cast<const int4*>(w + L.dkv_items);
+  a.items2 = runs2 ? reinterpret_cast<const int2*>(w + L.dkv_items2) : nullptr;
   a.n_items = reinterpret_cast<const int32_t*>(w + L.dkv_n);
   int rc = launch_bwd_mode<D, kModeDKV>(a, a.k, a.v, a.q, a.dout, T, st);
   if (rc) return rc;
   // Every query: dQ, plus dK, dV of the other rows (candidates' diagonal terms; padding zeros).
+  a.items2 = nullptr;
   a.items = reinterpret_cast<const int4*>(w + W.items);
   a.n_items = reinterpret_cast<const int32_t*>(w + W.n_items);
   return launch_bwd_mode<D, kModeDQ>(a, a.q, a.dout, a.k, a.v, T, st);
@@ -953,12 +1000,12 @@ extern "C" int jagged_cand_attn_bwd(const void* q, const void* k, const void* v,
     dkv_queue_kernel<int32_t><<<1, kQueueBuckets, 0, st>>>(
         (const int32_t*)offsets, (const int32_t*)(w + W.hist_lo), (const int32_t*)(w + W.hist_hi),
         B, H, reinterpret_cast<int4*>(w + L.dkv_items), L.dkv_max,
-        reinterpret_cast<int32_t*>(w + L.dkv_n), status);
+        reinterpret_cast<int32_t*>(w + L.dkv_n), status, nullptr, 0, nullptr);
   else
     dkv_queue_kernel<int64_t><<<1, kQueueBuckets, 0, st>>>(
         (const int64_t*)offsets, (const int64_t*)(w + W.hist_lo), (const int64_t*)(w + W.hist_hi),
         B, H, reinterpret_cast<int4*>(w + L.dkv_items), L.dkv_max,
-        reinterpret_cast<int32_t*>(w + L.dkv_n), status);
+        reinterpret_cast<int32_t*>(w + L.dkv_n), status, nullptr, 0, nullptr);
   if (cudaGetLastError() != cudaSuccess) return JCA_ERR_CUDA;
   if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
   BwdArgs a;
@@ -973,6 +1020,7 @@ extern "C" int jagged_cand_attn_bwd(const void* q, const void* k, const void* v,
   a.lse2 = nullptr;
   a.dsum = nullptr;
   a.items = nullptr;
+  a.items2 = nullptr;
   a.n_items = nullptr;
   a.status = status;
   a.T = T;
@@ -985,5 +1033,85 @@ extern "C" int jagged_cand_attn_bwd(const void* q, const void* k, const void* v,
     case 32: return launch_backward<32>(a, out, out_fp32, lse, T, workspace, W, L, st);
     case 64: return launch_backward<64>(a, out, out_fp32, lse, T, workspace, W, L, st);
     default: return launch_backward<128>(a, out, out_fp32, lse, T, workspace, W, L, st);
+  }
+}
+
+extern "C" size_t jca_seqpack_bwd_workspace_bytes(int64_t B, int64_t Th, int64_t Nc, int H,
+                                                  int d_head) {
+  if (B < 0 || Th < 0 || Nc < 0 || H < 1 || !head_dim_ok(d_head)) return 0;
+  const SeqpackLayout S = seqpack_layout(B, Th + Nc, H);
+  return bwd_layout_after(S.total, B, Th + Nc, Th, H, true).total;
+}
+
+extern "C" int jagged_cand_attn_seqpack_bwd(
+    const void* q, const void* k, const void* v, const void* out, int out_fp32, const void* dout,
+    const float* lse, void* dq, void* dk, void* dv, int grad_fp32, const void* hist_offsets,
+    const void* cand_offsets, const int8_t* seg, int64_t B, int64_t Th, int64_t Nc, int H,
+    int d_head, float scale, int idx_bits, void* workspace, size_t workspace_bytes,
+    int32_t* status, jca_stream_t stream) {
+  if (idx_bits != 32 && idx_bits != 64) return JCA_ERR_IDX_BITS;
+  if (!head_dim_ok(d_head)) return JCA_ERR_HEAD_DIM;
+  const int64_t T = Th + Nc;
+  if (B < 0 || Th < 0 || Nc < 0 || H < 1 || H >= 65536 || T >= (int64_t)INT_MAX ||
+      2 * B >= (int64_t)INT_MAX || (B == 0 && T != 0))
+    return JCA_ERR_SHAPE;
+  if (!status || !hist_offsets || !cand_offsets || !workspace) return JCA_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv))
+    return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+                !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+                !aligned(lse, 4)))
+    return JCA_ERR_ALIGN;
+  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+  const SeqpackLayout S = seqpack_layout(B, T, H);
+  if (S.base.max_items >= (int64_t)INT_MAX) return JCA_ERR_SHAPE;
+  const BwdLayout L = bwd_layout_after(S.total, B, T, Th, H, true);
+  if (workspace_bytes < L.total) return JCA_ERR_WORKSPACE;
+  if (T == 0) return JCA_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(workspace);
+  if (launch_seqpack_plan(hist_offsets, cand_offsets, seg, B, Th, Nc, H, idx_bits, w, S.base,
+                          S.q_off2, status, st) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  // dK, dV of each history key tile come from the user's history run and its candidate run.
+  if (idx_bits == 32)
+    dkv_queue_kernel<int32_t><<<1, kQueueBuckets, 0, st>>>(
+        (const int32_t*)hist_offsets, (const int32_t*)(w + S.base.hist_lo),
+        (const int32_t*)(w + S.base.hist_hi), B, H, reinterpret_cast<int4*>(w + L.dkv_items),
+        L.dkv_max, reinterpret_cast<int32_t*>(w + L.dkv_n), status,
+        (const int32_t*)cand_offsets, Th, reinterpret_cast<int2*>(w + L.dkv_items2));
+  else
+    dkv_queue_kernel<int64_t><<<1, kQueueBuckets, 0, st>>>(
+        (const int64_t*)hist_offsets, (const int64_t*)(w + S.base.hist_lo),
+        (const int64_t*)(w + S.base.hist_hi), B, H, reinterpret_cast<int4*>(w + L.dkv_items),
+        L.dkv_max, reinterpret_cast<int32_t*>(w + L.dkv_n), status,
+        (const int64_t*)cand_offsets, Th, reinterpret_cast<int2*>(w + L.dkv_items2));
+  if (cudaGetLastError() != cudaSuccess) return JCA_ERR_CUDA;
+  if (!(scale > 0.f)) scale = 1.0f / sqrtf((float)d_head);
+  BwdArgs a;
+  a.q = static_cast<const bf16*>(q);
+  a.k = static_cast<const bf16*>(k);
+  a.v = static_cast<const bf16*>(v);
+  a.dout = static_cast<const bf16*>(dout);
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.seg = seg ? seg : reinterpret_cast<const int8_t*>(w + S.base.seg);
+  a.lse2 = nullptr;
+  a.dsum = nullptr;
+  a.items = nullptr;
+  a.items2 = nullptr;
+  a.n_items = nullptr;
+  a.status = status;
+  a.T = T;
+  a.H = H;
+  a.grad_fp32 = grad_fp32 ? 1 : 0;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  switch (d_head) {
+    case 16: return launch_backward<16>(a, out, out_fp32, lse, T, workspace, S.base, L, st, true);
+    case 32: return launch_backward<32>(a, out, out_fp32, lse, T, workspace, S.base, L, st, true);
+    case 64: return launch_backward<64>(a, out, out_fp32, lse, T, workspace, S.base, L, st, true);
+    default: return launch_backward<128>(a, out, out_fp32, lse, T, workspace, S.base, L, st, true);
   }
 }

@@ -422,6 +422,58 @@ __global__ void __launch_bounds__(1024) causal_queue_kernel(
 
 inline int grid_for_rows(int64_t B) { return (int)(B < (1 << 20) ? B : (1 << 20)); }
 
+// ---------------------------------------------------------------------------------------------
+// Training with candidate packing (候选隔离注意力掩码, section 训练时的序列打包): the packed matrix
+// holds every user's prefix + history run in rows [0, Th) (split at hist_off) and every user's
+// candidate run in rows [Th, Th + Nc) (split at cand_off, relative to Th). The attention kernels
+// take it as 2B "query runs" over B key intervals: run b < B is user b's history run, run B + b
+// its candidate run, and both read user b's history keys.
+// ---------------------------------------------------------------------------------------------
+
+// Segment IDs of the packed matrix when the caller gives none (history rows 1, candidate rows -1),
+// or a check of the caller's candidate rows (only -1 or 0 there; the history rows are checked by
+// the bounds pass, which admits only 1 and 0).
+__global__ void __launch_bounds__(256) seqpack_seg_kernel(int8_t* __restrict__ seg_out,
+                                                          const int8_t* __restrict__ seg_in,
+                                                          int64_t Th, int64_t T,
+                                                          int32_t* status) {
+  if (*status != 0) return;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < T;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    if (seg_out) {
+      seg_out[i] = i < Th ? (int8_t)1 : (int8_t)-1;
+    } else if (i >= Th) {
+      const int x = seg_in[i];
+      if (x != -1 && x != 0) set_status(status, JCA_STATUS_BAD_SEG_VALUE);
+    }
+  }
+}
+
+// Checks the candidate offsets and writes the 2B query runs: q_off2[0..B] = hist_off,
+// q_off2[B + b] = Th + cand_off[b]; the key interval and key count of run B + b are user b's,
+// copied from entry b (written by the bounds pass over the history block).
+template <typename IdxT>
+__global__ void __launch_bounds__(256) seqpack_runs_kernel(
+    const IdxT* __restrict__ hist_off, const IdxT* __restrict__ cand_off, int64_t B, int64_t Th,
+    int64_t Nc, IdxT* __restrict__ q_off2, IdxT* __restrict__ kv_lo, IdxT* __restrict__ kv_hi,
+    int32_t* __restrict__ kv_count, int32_t* status) {
+  if (*status != 0) return;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b <= B;
+       b += (int64_t)gridDim.x * blockDim.x) {
+    const long long c = (long long)cand_off[b];
+    const bool bad = (b == 0 && c != 0) || (b == B && c != Nc) ||
+                     (b < B && (long long)cand_off[b + 1] < c) || c < 0 || c > Nc;
+    if (bad) set_status(status, JCA_STATUS_BAD_OFFSETS);
+    q_off2[b] = hist_off[b];
+    if (b > 0) q_off2[B + b] = (IdxT)(Th + c);
+    if (b < B) {
+      kv_lo[B + b] = kv_lo[b];
+      kv_hi[B + b] = kv_hi[b];
+      kv_count[B + b] = kv_count[b];
+    }
+  }
+}
+
 }  // namespace
 
 int64_t max_work_items(int64_t B, int64_t rows, int H) {
@@ -523,6 +575,42 @@ cudaError_t launch_work_queue(const void* q_offsets, const void* kv_lo, const vo
         (const int64_t*)q_offsets, (const int64_t*)kv_lo, (const int64_t*)kv_hi, kv_count, B,
         q_rows, kv_rows, H, (int4*)items, max_items, n_items, status, queue_ctl);
   return cudaGetLastError();
+}
+
+cudaError_t launch_seqpack_plan(const void* hist_off, const void* cand_off, const int8_t* seg,
+                                int64_t B, int64_t Th, int64_t Nc, int H, int idx_bits, char* ws,
+                                const WorkspaceLayout& L, size_t q_off2, int32_t* status,
+                                cudaStream_t stream) {
+  const int64_t T = Th + Nc;
+  int8_t* seg_ws = reinterpret_cast<int8_t*>(ws + L.seg);
+  const int8_t* segp = seg ? seg : seg_ws;
+  if (T > 0) {
+    const int64_t blocks = (T + 255) / 256;
+    seqpack_seg_kernel<<<(int)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, stream>>>(
+        seg ? nullptr : seg_ws, seg, Th, T, status);
+    if (cudaGetLastError() != cudaSuccess) return cudaErrorLaunchFailure;
+  }
+  cudaError_t e = launch_bounds(segp, hist_off, B, Th, idx_bits, ws + L.hist_lo, ws + L.hist_hi,
+                                nullptr, nullptr, reinterpret_cast<int32_t*>(ws + L.kv_count), 1,
+                                status, stream);
+  if (e != cudaSuccess) return e;
+  const int grid = (int)((B + 1 + 255) / 256);
+  if (idx_bits == 32)
+    seqpack_runs_kernel<int32_t><<<grid, 256, 0, stream>>>(
+        (const int32_t*)hist_off, (const int32_t*)cand_off, B, Th, Nc, (int32_t*)(ws + q_off2),
+        (int32_t*)(ws + L.hist_lo), (int32_t*)(ws + L.hist_hi),
+        reinterpret_cast<int32_t*>(ws + L.kv_count), status);
+  else
+    seqpack_runs_kernel<int64_t><<<grid, 256, 0, stream>>>(
+        (const int64_t*)hist_off, (const int64_t*)cand_off, B, Th, Nc, (int64_t*)(ws + q_off2),
+        (int64_t*)(ws + L.hist_lo), (int64_t*)(ws + L.hist_hi),
+        reinterpret_cast<int32_t*>(ws + L.kv_count), status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return launch_work_queue(ws + q_off2, ws + L.hist_lo, ws + L.hist_hi,
+                           reinterpret_cast<int32_t*>(ws + L.kv_count), 2 * B, T, T, H, idx_bits,
+                           reinterpret_cast<int32_t*>(ws + L.items), L.max_items,
+                           reinterpret_cast<int32_t*>(ws + L.n_items), status, stream,
+                           reinterpret_cast<int32_t*>(ws + L.queue));
 }
 
 }  // namespace jca

@@ -79,4 +79,29 @@ cudaError_t launch_causal_queue(const void* offsets, int64_t B, int64_t rows, in
                                 int idx_bits, int32_t* items, int64_t max_items, int32_t* n_items,
                                 int32_t* status, cudaStream_t stream, int32_t* queue_ctl);
 
+// Training with candidate packing: the packed matrix [history runs | candidate runs] as 2B query
+// runs over B key intervals. `L` is workspace_layout(2B, Th + Nc, H); q_off2 is the byte offset of
+// 2B + 1 offsets (idx_bits type) in the workspace. Writes the segment IDs (when seg is NULL), the
+// bounds of the history block, the runs and the work queue.
+cudaError_t launch_seqpack_plan(const void* hist_off, const void* cand_off, const int8_t* seg,
+                                int64_t B, int64_t Th, int64_t Nc, int H, int idx_bits, char* ws,
+                                const WorkspaceLayout& L, size_t q_off2, int32_t* status,
+                                cudaStream_t stream);
+
+// Workspace of the candidate-packing entry points: workspace_layout(2B, T, H) followed by the
+// 2B + 1 query-run offsets.
+struct SeqpackLayout {
+  WorkspaceLayout base;
+  size_t q_off2 = 0;
+  size_t total = 0;
+};
+
+inline SeqpackLayout seqpack_layout(int64_t B, int64_t T, int H) {
+  SeqpackLayout s;
+  s.base = workspace_layout(2 * B, T, H);
+  s.q_off2 = align_up(s.base.total, 256);
+  s.total = align_up(s.q_off2 + 8 * (size_t)(2 * B + 1), 256);
+  return s;
+}
+
 }  // namespace jca

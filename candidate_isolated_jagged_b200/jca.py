@@ -61,6 +61,14 @@ _SIGNATURES = {
     "jagged_cand_attn_bwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_f32,
                                      c_i32, c_vp, c_sz, c_vp, c_vp]),
+    "jca_seqpack_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i32, c_i32]),
+    "jca_seqpack_bwd_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i32, c_i32]),
+    "jagged_cand_attn_seqpack_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp,
+                                             c_i64, c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp,
+                                             c_sz, c_vp, c_vp]),
+    "jagged_cand_attn_seqpack_bwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp,
+                                             c_vp, c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64,
+                                             c_i32, c_i32, c_f32, c_i32, c_vp, c_sz, c_vp, c_vp]),
     "jca_stack_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i64, c_i32, c_i32]),
     "jca_stack_fwd": (c_i32, [c_vp, c_vp, c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i64,
                               c_i64, c_i32, c_i32, c_f32, c_i64, c_f32, c_i32, c_vp, c_sz, c_vp,
@@ -417,6 +425,69 @@ def jagged_cand_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, offsets, candidate
         _ptr(dv), grad_fp32, _ptr(offsets), _ptr(candidate_start), _ptr(seg), B, T, H, d,
         float(scale), _idx_bits(offsets), _ptr(workspace), workspace.numel(), _ptr(status),
         _stream(stream)), "jagged_cand_attn_bwd")
+
+
+def jca_seqpack_workspace_bytes(B: int, Th: int, Nc: int, H: int, d_head: int) -> int:
+    return int(lib().jca_seqpack_workspace_bytes(int(B), int(Th), int(Nc), int(H), int(d_head)))
+
+
+def jca_seqpack_bwd_workspace_bytes(B: int, Th: int, Nc: int, H: int, d_head: int) -> int:
+    return int(lib().jca_seqpack_bwd_workspace_bytes(int(B), int(Th), int(Nc), int(H),
+                                                     int(d_head)))
+
+
+def jagged_cand_attn_seqpack_fwd(q, k, v, out, hist_offsets, cand_offsets, seg=None, lse=None,
+                                 scale: float = 0.0, workspace: Optional[torch.Tensor] = None,
+                                 status: Optional[torch.Tensor] = None, stream=None,
+                                 Th: Optional[int] = None) -> int:
+    """Forward over the candidate-packed matrix [history runs | candidate runs] (rows [0, Th)
+    split at hist_offsets, rows [Th, T) split at cand_offsets); lse [T, H] fp32 optional.
+    Th (history rows) is read back from hist_offsets when not given."""
+    T, H, d = q.shape
+    B = hist_offsets.numel() - 1
+    Th = _seqpack_th(hist_offsets) if Th is None else int(Th)
+    Nc = T - Th
+    if workspace is None:
+        workspace = torch.empty(max(1, jca_seqpack_workspace_bytes(B, Th, Nc, H, d)),
+                                dtype=torch.uint8, device=q.device)
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().jagged_cand_attn_seqpack_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(lse), _ptr(hist_offsets),
+        _ptr(cand_offsets), _ptr(seg), B, Th, Nc, H, d, float(scale), _idx_bits(hist_offsets),
+        _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
+        "jagged_cand_attn_seqpack_fwd")
+
+
+def jagged_cand_attn_seqpack_bwd(q, k, v, out, dout, lse, dq, dk, dv, hist_offsets, cand_offsets,
+                                 seg=None, scale: float = 0.0,
+                                 workspace: Optional[torch.Tensor] = None,
+                                 status: Optional[torch.Tensor] = None, stream=None,
+                                 Th: Optional[int] = None) -> int:
+    """Gradients dq, dk, dv over the candidate-packed matrix (see jagged_cand_attn_seqpack_fwd)."""
+    T, H, d = q.shape
+    B = hist_offsets.numel() - 1
+    Th = _seqpack_th(hist_offsets) if Th is None else int(Th)
+    Nc = T - Th
+    if workspace is None:
+        workspace = torch.empty(max(1, jca_seqpack_bwd_workspace_bytes(B, Th, Nc, H, d)),
+                                dtype=torch.uint8, device=q.device)
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    grad_fp32 = 1 if dq.dtype == torch.float32 else 0
+    assert dk.dtype == dq.dtype and dv.dtype == dq.dtype
+    return _check(lib().jagged_cand_attn_seqpack_bwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+        _ptr(dv), grad_fp32, _ptr(hist_offsets), _ptr(cand_offsets), _ptr(seg), B, Th, Nc, H, d,
+        float(scale), _idx_bits(hist_offsets), _ptr(workspace), workspace.numel(), _ptr(status),
+        _stream(stream)), "jagged_cand_attn_seqpack_bwd")
+
+
+def _seqpack_th(hist_offsets) -> int:
+    """Th = hist_offsets[B], read back to the host (the caller's layout; a device read)."""
+    return int(hist_offsets[-1].item())
 
 
 def jca_stack_workspace_bytes(B: int, T: int, Nc: int, Th: int, H: int, d_head: int) -> int:

@@ -407,6 +407,63 @@ int jagged_cand_attn_bwd(const void* q, const void* k, const void* v, const void
                          jca_stream_t stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * Training with candidate packing (候选隔离注意力掩码, section 训练时的序列打包: users' sequences are
+ * packed into one matrix split at cu_seqlens, and the candidates are stored apart, all in one
+ * block, each candidate's representation read back at its candidate_positions entry). Packing
+ * changes where rows sit, not what they compute: the mask is the serving one.
+ *
+ * Layout (a reading; the pages name it without drawing it): one packed matrix of T = Th + Nc rows.
+ * Rows [0, Th) hold every user's prefix + history run back to back, split at hist_offsets [B+1]
+ * (hist_offsets[0] = 0, hist_offsets[B] = Th: the cu_seqlens). Rows [Th, T) hold every user's
+ * candidate run back to back, split at cand_offsets [B+1], relative to the block (cand_offsets[0]
+ * = 0, cand_offsets[B] = Nc). Candidate c therefore sits at row Th + c: candidate_positions is
+ * Th + [0, Nc). User b's history rows see the segment-1 rows of its own history run, and its
+ * candidates see those plus themselves.
+ *   seg [T] int8 or NULL: NULL means history rows 1 and candidate rows -1; when given, history
+ *       rows hold 1 or 0 (padding) and candidate rows -1 or 0 (an empty candidate slot).
+ * ------------------------------------------------------------------------------------------- */
+
+/* Workspace bytes of jagged_cand_attn_seqpack_fwd (0 for invalid sizes). */
+size_t jca_seqpack_workspace_bytes(int64_t B, int64_t Th, int64_t Nc, int H, int d_head);
+
+/*
+ * Forward over the candidate-packed matrix.
+ *   q, k, v [T, H, d_head] bf16, read; out [T, H, d_head] bf16 or fp32 (out_fp32), written.
+ *   lse [T, H] fp32 or NULL: when given, the natural-log softmax denominator of every row and head
+ *       (as jagged_cand_attn_fwd_lse; -inf for padding rows), for the backward pass.
+ *   hist_offsets, cand_offsets [B+1] (idx_bits type), read; seg as above.
+ *   workspace >= jca_seqpack_workspace_bytes(B, Th, Nc, H, d_head) bytes, 256-byte aligned.
+ * Device errors: bad hist_offsets or cand_offsets -> JCA_STATUS_BAD_OFFSETS (nothing written); a
+ * segment ID outside the values above -> JCA_STATUS_BAD_SEG_VALUE; JCA_STATUS_TIMEOUT.
+ */
+int jagged_cand_attn_seqpack_fwd(const void* q, const void* k, const void* v, void* out,
+                                 int out_fp32, float* lse, const void* hist_offsets,
+                                 const void* cand_offsets, const int8_t* seg, int64_t B,
+                                 int64_t Th, int64_t Nc, int H, int d_head, float scale,
+                                 int idx_bits, void* workspace, size_t workspace_bytes,
+                                 int32_t* status, jca_stream_t stream);
+
+/* Workspace bytes of jagged_cand_attn_seqpack_bwd (0 for invalid sizes). */
+size_t jca_seqpack_bwd_workspace_bytes(int64_t B, int64_t Th, int64_t Nc, int H, int d_head);
+
+/*
+ * Gradients over the candidate-packed matrix, as jagged_cand_attn_bwd: dq, dk, dv [T, H, d_head]
+ * (bf16, or fp32 with grad_fp32), every row written; a history key's dK and dV collect the
+ * gradient of its user's history rows and candidate rows, a candidate's own key and value that of
+ * the candidate alone, padding rows get 0.
+ *   out and lse from jagged_cand_attn_seqpack_fwd on the same inputs; other arguments as the
+ *   forward. workspace >= jca_seqpack_bwd_workspace_bytes(B, Th, Nc, H, d_head) bytes.
+ * Device errors: as the forward, plus JCA_STATUS_QUEUE_OVERFLOW (internal).
+ */
+int jagged_cand_attn_seqpack_bwd(const void* q, const void* k, const void* v, const void* out,
+                                 int out_fp32, const void* dout, const float* lse, void* dq,
+                                 void* dk, void* dv, int grad_fp32, const void* hist_offsets,
+                                 const void* cand_offsets, const int8_t* seg, int64_t B,
+                                 int64_t Th, int64_t Nc, int H, int d_head, float scale,
+                                 int idx_bits, void* workspace, size_t workspace_bytes,
+                                 int32_t* status, jca_stream_t stream);
+
+/* ---------------------------------------------------------------------------------------------
  * Layer stack with candidate-only tail layers (候选隔离注意力掩码, section 只更新候选的末尾层 and its
  * flowchart): the first n_layers - n_cand_only layers run over whole rows [prefix | history |
  * candidates] under the isolation mask; then the states are split into the frozen history
