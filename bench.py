@@ -89,8 +89,9 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x2: "applications_clocks_setting", 0x1: "gpu_idle"}
 
-    def __init__(self, index: int, period_s: float = 0.02):
-        self.samples, self.reasons, self.ok = [], set(), False
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.times, self.reasons, self.ok = [], [], set(), False
+        self.t_mark = None
         self.max_mhz = None
         self._stop = threading.Event()
         self.period = period_s
@@ -108,6 +109,7 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.times.append(time.perf_counter())
                 r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
                 for bit, name in self.REASONS.items():
                     if r & bit:
@@ -127,12 +129,22 @@ class ClockSampler:
             self._stop.set()
             self._t.join()
 
+    def mark(self):
+        """Start of the timed region (the samples before it cover the warm-up's identical load)."""
+        self.t_mark = time.perf_counter()
+
     def summary(self):
         if not self.ok or not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
                     "note": "NVML unavailable" if not self.ok else "no samples"}
+        timed = [c for c, t in zip(self.samples, self.times)
+                 if self.t_mark is not None and t >= self.t_mark]
         return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples),
+                "samples_timed_region": len(timed),
+                "sm_mhz_timed_region": float(statistics.median(timed)) if timed else None,
+                "window_ms": 1e3 * (self.times[-1] - self.times[0]),
+                "covers": "back-to-back warm-up steps (at least 100 ms) and the timed region"}
 
 
 def max_over_ranks(values, dist=None, device="cpu"):
@@ -277,20 +289,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         if ev is not None:
             ev[1].record(stream)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-    jca.check_status(status, "warm-up")
-    assert bool(torch.isfinite(out.float()).all()), "non-finite attention output"
-
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(dev.index if dev.index is not None else 0)
     with sampler:
+        # Warm-up under the clock sampler: at least W steps and at least 100 ms of back-to-back
+        # steps, so that the clock record covers the same load even when the timed region is short.
+        t_w, n_w = time.perf_counter(), 0
+        while n_w < args.warmup or time.perf_counter() - t_w < 0.1:
+            step()
+            n_w += 1
+            if n_w % 32 == 0:
+                torch.cuda.synchronize(dev)
+        torch.cuda.synchronize(dev)
+        jca.check_status(status, "warm-up")
+        assert bool(torch.isfinite(out.float()).all()), "non-finite attention output"
         if dist:
             dist.barrier()
         torch.cuda.synchronize(dev)
+        sampler.mark()
         t_start.record(stream)
         for i in range(args.steps):
             step(kev[i])
@@ -418,8 +436,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         line["rope"] = run_rope_extras(args, dev, stream, peaks)
         line["stack"] = run_stack_extras(args, dev, stream, peaks)
         line["backward"] = run_backward_extras(args, dev, stream, peaks)
+        line["seqpack"] = run_seqpack_extras(args, dev, stream, peaks)
         line["causal"] = run_causal_extras(args, dev, stream, peaks)
         line["ug_sep"] = run_ug_extras(args, dev, stream, peaks)
+        line["configs"] = run_config_block(args, dev, stream, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         users = oracle_sample_users(batch, args.cpu_sample_stride, 3)
         fl, tok, times = time_oracle(batch, users, repeats=1)
@@ -431,6 +451,131 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def time_calls(fn, stream, dev, n: int, flush=None, warmup: int = 10):
+    """Per-call device times (ms) of `fn` on `stream`, each bracketed by its own CUDA events; with
+    `flush`, the L2 is overwritten before every call (outside the events)."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(n)]
+    torch.cuda.synchronize(dev)
+    for a, b in ev:
+        if flush is not None:
+            flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def run_config_block(args, dev, stream, peaks):
+    """Every workload of the benchmark's configuration list, each through its public entry point
+    (plan + attention kernel per call, as a caller runs it): the median device time of 50 calls
+    with the L2 flushed before each call (a 512 MB write) and of 50 back-to-back calls (warm L2),
+    the effective TFLOP/s, the roofline fraction of the bound that applies, and the CPU oracle
+    timed on the host cores on a stated sample of the same workload."""
+    import torch
+    import oracle
+    import synth
+    from candidate_isolated_jagged_b200 import jca, metrics
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    n_calls = 50
+    out = {}
+    cores = blas_threads()
+
+    def gpu_entry(fl, byts, bound, fn):
+        cold = time_calls(fn, stream, dev, n_calls, flush)
+        warm = time_calls(fn, stream, dev, n_calls)
+        mc, mw = statistics.median(cold), statistics.median(warm)
+        tf = fl / mc / 1e9
+        gbs = byts / mc / 1e6
+        frac = tf / peaks["bf16_tflops"] if bound == "tensor" else gbs / peaks["hbm_gbs"]
+        return {"ms_cold_l2_median": mc, "ms_warm_l2_median": mw, "calls": n_calls,
+                "effective_tflops_cold": tf, "effective_tflops_warm": fl / mw / 1e9,
+                "algorithmic_gb_s_cold": gbs, "bound": bound, "roofline_frac_cold": frac,
+                "effective_flops": fl, "algorithmic_bytes": byts}
+
+    # ---- full op: tiny, three_users, users256 ----
+    for name, make, bound, sample_users in (
+            ("tiny", synth.tiny, "latency", None),
+            ("three_users", synth.three_users, "latency", None),
+            ("users256", synth.users256, "tensor", "every 16th user (index = 3 mod 16)")):
+        b = make()
+        B, T, H, d = b.B, b.T, b.H, b.d
+        off_np = oracle.offsets_from_lengths(b.row_lengths)
+        seg_np = oracle.segment_ids(off_np, b.cand_start, b.valid)
+        q, k, v = (t.to(dev) for t in (b.q, b.k, b.v))
+        off = torch.tensor(off_np, device=dev)
+        cs = torch.tensor(b.cand_start, device=dev)
+        seg = torch.tensor(seg_np, device=dev) if b.valid is not None else None
+        o = torch.empty(T, H, d, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(jca.jca_workspace_bytes(B, T, H, d), dtype=torch.uint8, device=dev)
+        st = jca.new_status(dev)
+        fl = metrics.effective_flops(metrics.allowed_pairs_from_counts(b.prefix + b.hist_real,
+                                                                       b.n_cand), H, d)
+        byts = metrics.full_attention_bytes(T, H, d)
+        entry = gpu_entry(fl, byts, bound, lambda: jca.jagged_cand_attn_fwd(
+            q, k, v, o, off, None if seg is not None else cs, seg, workspace=ws, status=st,
+            stream=stream))
+        jca.check_status(st, name)
+        users = list(range(B)) if sample_users is None else [u for u in range(B) if u % 16 == 3]
+        ofl = metrics.effective_flops(metrics.allowed_pairs_from_counts(
+            (b.prefix + b.hist_real)[users], b.n_cand[users]), H, d)
+        t0 = time.perf_counter()
+        oracle.jagged_cand_attn(b.q, b.k, b.v, off_np, seg_np, b.scale, users=users)
+        osec = time.perf_counter() - t0
+        entry["oracle"] = {"seconds": osec, "effective_tflops": ofl / osec / 1e12, "cores": cores,
+                           "sample": "whole workload" if sample_users is None else
+                           f"{sample_users}: {len(users)} of {B} users, {ofl / 1e9:.1f} GFLOP"}
+        out[name] = entry
+        del q, k, v, o, ws
+
+    # ---- candidate-only: cand_only256, retrieval ----
+    for name, make, per_user in (("cand_only256", synth.cand_only256, 64),
+                                 ("retrieval", synth.retrieval, 500)):
+        cb = make()
+        coff_np = oracle.offsets_from_lengths(cb.cand_counts)
+        hoff_np = oracle.offsets_from_lengths(cb.hist_lengths)
+        coff, hoff = torch.tensor(coff_np, device=dev), torch.tensor(hoff_np, device=dev)
+        cq, ck, cv, hk, hv = (t.to(dev) for t in (cb.cq, cb.ck, cb.cv, cb.hk, cb.hv))
+        o = torch.empty(cq.shape, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(jca.jca_workspace_bytes(cb.B, cb.Nc, cb.H, cb.d), dtype=torch.uint8,
+                         device=dev)
+        st = jca.new_status(dev)
+        pairs = int(np.sum(cb.cand_counts * (cb.hist_lengths + 1)))
+        fl = metrics.effective_flops(pairs, cb.H, cb.d)
+        byts = metrics.cand_only_bytes(cb.Nc, cb.Th, cb.H, cb.d)
+        entry = gpu_entry(fl, byts, "hbm", lambda: jca.cand_only_attn_fwd(
+            cq, ck, cv, coff, hk, hv, hoff, o, None, workspace=ws, status=st, stream=stream))
+        jca.check_status(st, name)
+        # oracle: the first `per_user` candidates of every 8th user (request)
+        users = list(range(0, cb.B, 8)) if cb.B > 2 else list(range(cb.B))
+        rows = np.concatenate([np.arange(coff_np[u], coff_np[u] + min(per_user, cb.cand_counts[u]))
+                               for u in users])
+        ucount = np.array([min(per_user, cb.cand_counts[u]) for u in users])
+        ofl = metrics.effective_flops(int(np.sum(ucount * (cb.hist_lengths[users] + 1))), cb.H,
+                                      cb.d)
+        t0 = time.perf_counter()
+        oracle.cand_only_attn(cb.cq, cb.ck, cb.cv, coff_np, cb.hk, cb.hv, hoff_np, None, cb.scale,
+                              cand_rows=rows)
+        osec = time.perf_counter() - t0
+        entry["oracle"] = {"seconds": osec, "effective_tflops": ofl / osec / 1e12, "cores": cores,
+                           "candidates_per_s": rows.size / osec,
+                           "sample": f"the first {per_user} candidates of every 8th user or "
+                                     f"request ({len(users)} of {cb.B}, {rows.size} candidates)"}
+        out[name] = entry
+        del cq, ck, cv, hk, hv, o, ws
+    del flush_buf
+    torch.cuda.empty_cache()
+    return out
 
 
 def run_rope_extras(args, dev, stream, peaks):
@@ -637,6 +782,75 @@ def run_backward_extras(args, dev, stream, peaks):
     return res
 
 
+def run_seqpack_extras(args, dev, stream, peaks):
+    """Training with candidate packing on the 256-user workload: every user's prefix + history
+    first, then all candidates in one block (rows rearranged once on the host, as a data loader
+    would pack them); the forward with its log-sum-exp and the backward through
+    jagged_cand_attn_seqpack_fwd / _bwd, timed with CUDA events over repeated calls. FLOPs as for
+    the serving-layout training path (backward: 2.5x the forward)."""
+    import torch
+    import synth
+    from candidate_isolated_jagged_b200 import jca, metrics
+    b = synth.users256()
+    cs = np.asarray(b.cand_start, dtype=np.int64)
+    L = np.asarray(b.row_lengths, dtype=np.int64)
+    off = np.concatenate([[0], np.cumsum(L)])
+    perm = np.concatenate([np.arange(off[u], off[u] + cs[u]) for u in range(b.B)] +
+                          [np.arange(off[u] + cs[u], off[u + 1]) for u in range(b.B)])
+    hoff = torch.tensor(np.concatenate([[0], np.cumsum(cs)]), dtype=torch.int64, device=dev)
+    coff = torch.tensor(np.concatenate([[0], np.cumsum(L - cs)]), dtype=torch.int64, device=dev)
+    Th = int(cs.sum())
+    p = torch.from_numpy(perm)
+    q, k, v = (t[p].to(dev) for t in (b.q, b.k, b.v))
+    dout = synth.upstream_grad(b.q.shape, 15)[p].to(dev)
+    T, H, d = q.shape
+    out = torch.empty_like(q)
+    lse = torch.empty(T, H, dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    wsf = torch.empty(jca.jca_seqpack_workspace_bytes(b.B, Th, T - Th, H, d), dtype=torch.uint8,
+                      device=dev)
+    wsb = torch.empty(jca.jca_seqpack_bwd_workspace_bytes(b.B, Th, T - Th, H, d),
+                      dtype=torch.uint8, device=dev)
+    st = jca.new_status(dev)
+    fwd_flops = metrics.effective_flops(
+        metrics.allowed_pairs_from_counts(b.prefix + b.hist_real, b.n_cand), H, d)
+
+    def fwd():
+        jca.jagged_cand_attn_seqpack_fwd(q, k, v, out, hoff, coff, None, lse, workspace=wsf,
+                                         status=st, stream=stream, Th=Th)
+
+    def bwd():
+        jca.jagged_cand_attn_seqpack_bwd(q, k, v, out, dout, lse, dq, dk, dv, hoff, coff, None,
+                                         workspace=wsb, status=st, stream=stream, Th=Th)
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+        bwd()
+    n = max(1, min(args.steps, 20))
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    torch.cuda.synchronize(dev)
+    ev[0].record(stream)
+    for _ in range(n):
+        fwd()
+    ev[1].record(stream)
+    for _ in range(n):
+        bwd()
+    ev[2].record(stream)
+    torch.cuda.synchronize(dev)
+    jca.check_status(st, "seqpack")
+    f_ms = ev[0].elapsed_time(ev[1]) / n
+    b_ms = ev[1].elapsed_time(ev[2]) / n
+    res = {"workload": "users256 rearranged: %d history rows, then %d candidates in one block "
+                       "(H=%d, d=%d), dO ~ N(0,1) seed 15" % (Th, T - Th, H, d),
+           "fwd_lse_ms": f_ms, "fwd_lse_effective_tflops": fwd_flops / f_ms / 1e9,
+           "bwd_ms": b_ms, "bwd_effective_tflops": 2.5 * fwd_flops / b_ms / 1e9,
+           "bwd_pct_of_bf16_peak": 100 * 2.5 * fwd_flops / b_ms / 1e9 / peaks["bf16_tflops"],
+           "launches_timed": 2 * n}
+    del q, k, v, dout, out, lse, dq, dk, dv, wsf, wsb
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_stack_extras(args, dev, stream, peaks):
     """The layer stack on the 256-user rows: 8 layers (D = 1024, H = 8, d = 128) whose last 2 are
     candidate-only, with right-anchored RoPE, through jca_stack_fwd; and, for comparison, the same
@@ -750,7 +964,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-stride", type=int, default=4)
     ap.add_argument("--only", choices=["cand_only", "rope", "stack", "backward", "causal",
-                                       "ug_sep"],
+                                       "ug_sep", "configs", "seqpack"],
                     default=None,
                     help="run one extra section alone on one GPU and print its result (profiling)")
     ap.add_argument("--shard", choices=["replicas", "users"], default="replicas",
@@ -776,7 +990,8 @@ def main():
         torch.cuda.set_device(dev)
         fn = {"cand_only": run_cand_only_extras, "rope": run_rope_extras,
               "stack": run_stack_extras, "backward": run_backward_extras,
-              "causal": run_causal_extras, "ug_sep": run_ug_extras}[args.only]
+              "causal": run_causal_extras, "ug_sep": run_ug_extras,
+              "configs": run_config_block, "seqpack": run_seqpack_extras}[args.only]
         print(json.dumps({args.only: fn(args, dev, torch.cuda.current_stream(dev), load_peaks())}),
               flush=True)
         return 0
