@@ -612,6 +612,36 @@ def run_rope_extras(args, dev, stream, peaks):
     pos_ms = ev[0].elapsed_time(ev[1]) / n
     rot_ms = ev[1].elapsed_time(ev[2]) / (2 * n)
     byts = 2 * q.numel() * 2   # one bf16 read and one bf16 write per element
+    # Attention with RoPE: in-kernel rotation (one call) against the pre-pass path (positions, two
+    # rotations, attention) and against attention without RoPE, each per call with its plan.
+    q0, k0 = b.q.to(dev), b.k.to(dev)
+    v0 = b.v.to(dev)
+    cs = torch.tensor(b.cand_start, device=dev)
+    out = torch.empty_like(q0)
+    wsr = torch.empty(jca.jca_rope_attn_workspace_bytes(b.B, b.T, b.H, b.d), dtype=torch.uint8,
+                      device=dev)
+    wsa = torch.empty(jca.jca_workspace_bytes(b.B, b.T, b.H, b.d), dtype=torch.uint8, device=dev)
+    qr, kr = torch.empty_like(q0), torch.empty_like(k0)
+
+    def fused():
+        jca.jagged_cand_attn_rope_fwd(q0, k0, v0, out, off, cs, None, history_end=4096,
+                                      workspace=wsr, status=st, stream=stream)
+
+    def prepass():
+        jca.jca_rope_positions(seg, off, pos, 4096, st, stream=stream)
+        jca.jca_apply_rope(q0, qr, pos, stream=stream)
+        jca.jca_apply_rope(k0, kr, pos, stream=stream)
+        jca.jagged_cand_attn_fwd(qr, kr, v0, out, off, cs, None, workspace=wsa, status=st,
+                                 stream=stream)
+
+    def plain():
+        jca.jagged_cand_attn_fwd(q0, k0, v0, out, off, cs, None, workspace=wsa, status=st,
+                                 stream=stream)
+
+    times = {}
+    for name, fn in (("plain", plain), ("fused", fused), ("prepass", prepass)):
+        times[name] = statistics.median(time_calls(fn, stream, dev, 30))
+    jca.check_status(st, "rope attention")
     res = {
         "workload": "users256 queries and keys (T=%d, H=%d, d=%d), history_end 4096" % (b.T, b.H, b.d),
         "positions_ms": pos_ms,
@@ -620,8 +650,14 @@ def run_rope_extras(args, dev, stream, peaks):
                      "unit": "GB/s", "frac": byts / rot_ms / 1e6 / peaks["hbm_gbs"],
                      "algorithmic_bytes_per_launch": byts},
         "launches_timed": 3 * n,
+        "attention_with_rope": {
+            "workload": "users256, history_end 4096; median of 30 calls each, plan included",
+            "fused_ms": times["fused"], "prepass_path_ms": times["prepass"],
+            "no_rope_ms": times["plain"],
+            "fused_over_no_rope": times["fused"] / times["plain"],
+            "prepass_over_no_rope": times["prepass"] / times["plain"]},
     }
-    del q, k
+    del q, k, q0, k0, v0, out, wsr, wsa, qr, kr
     torch.cuda.empty_cache()
     return res
 

@@ -42,6 +42,7 @@
 
 #include "jca_device.cuh"
 #include "jca_internal.h"
+#include "rope_device.cuh"
 
 namespace jca {
 namespace {
@@ -66,6 +67,14 @@ struct AttnArgs {
   int causal = 0;           // per-user causal variant: row i sees the keys j <= i of its user,
                             // no candidate or padding rows (items come from the causal queue);
                             // selects the CAUSAL instantiation of the kernel
+  // Right-anchored RoPE applied inside the kernel (the ROPE instantiation): every Q and K tile is
+  // rotated in shared memory after it lands and before the tensor core reads it.
+  const int32_t* q_pos = nullptr;      // [Tq] position of each query row
+  const int32_t* kv_pos = nullptr;     // [Tkv] position of each key row
+  const float2* rope_coarse = nullptr; // [n_coarse][D/2] (cos, sin)(128 (qmax - i) theta_j)
+  const float2* rope_fine = nullptr;   // [128][D/2] (cos, sin)(r theta_j)
+  long long rope_qmax = 0;
+  int rope = 0;                        // selects the ROPE instantiation
 };
 
 // Depth of the shared ring through which every role receives the claimed work items.
@@ -110,7 +119,11 @@ struct Cfg {
   static constexpr int B_DIAGEMPTY = B_DIAGFULL + 2;       // [slot]: scores taken
   static constexpr int B_RINGFULL = B_DIAGEMPTY + 2;       // [kRing]: claimed item index written
   static constexpr int B_RINGEMPTY = B_RINGFULL + kRing;   // [kRing]: index read by every role
-  static constexpr int NUM_BARS = B_RINGEMPTY + kRing;
+  // ROPE instantiation: a landed Q / K tile has been rotated in place (the MMA waits on these
+  // instead of the TMA's full barriers).
+  static constexpr int B_QREADY = B_RINGEMPTY + kRing;     // [group][QS]
+  static constexpr int B_KREADY = B_QREADY + 2 * QS;       // [KVS]
+  static constexpr int NUM_BARS = B_KREADY + KVS;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // Diagonal scores of the candidate rows: two item slots of kItemRows floats.
   static constexpr int OFF_RING = OFF_MISC + 16;           // kRing claimed item indices
@@ -133,12 +146,6 @@ constexpr int kSoftmaxThreads = 256;
 constexpr int kDiagThreads = 64;
 // Readers of the item ring: V producer lane, MMA thread, softmax and diagonal threads.
 constexpr int kRingReaders = 1 + 1 + kSoftmaxThreads + kDiagThreads;
-// Key pairs (of every 16 in a 32-key chunk) whose 2^x is evaluated on the FMA pipe; even.
-#ifndef JCA_EMU_PAIRS
-#define JCA_EMU_PAIRS 0
-#endif
-constexpr int kEmuPairs = JCA_EMU_PAIRS;
-static_assert(kEmuPairs % 2 == 0 && kEmuPairs >= 0 && kEmuPairs <= 16, "emulated pairs per chunk");
 
 struct Item {
   int q_row0, h, nrows, kv_lo, kv_len, holes, n_kv;
@@ -350,10 +357,13 @@ struct PendingPV {
   bool last;     // the item's last key tile: its completion makes O ready
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool ROPE>
 __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort_flag, ItemRing ring) {
   using C = Cfg<D>;
+  // With in-kernel RoPE a landed tile is usable only once the diagonal warps have rotated it.
+  constexpr int QF = ROPE ? C::B_QREADY : C::B_QFULL;
+  constexpr int KF = ROPE ? C::B_KREADY : C::B_KFULL;
   constexpr uint32_t kIdescQKFull = idesc_bf16_f32(C::BM, C::BN, false, false);
   // QK^T of a trimmed tile: N = keys of the tile rounded up to 16.
   constexpr uint32_t kIdescQK0 = kIdescQKFull & ~(0x3Fu << 17);
@@ -391,7 +401,7 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     const int qslot_b = C::QS + (int)(st.q_seen[1] % C::QS);
     const uint64_t qa = st.q + (uint64_t)((qslot_a * C::TILE_BYTES) >> 4);
     const uint64_t qb = st.q + (uint64_t)((qslot_b * C::TILE_BYTES) >> 4);
-    ok = mbar_wait(bars + 8 * (C::B_QFULL + qslot_a), (st.q_seen[0] / C::QS) & 1, abort_flag,
+    ok = mbar_wait(bars + 8 * (QF + qslot_a), (st.q_seen[0] / C::QS) & 1, abort_flag,
                    a.status);
     if (!ok) break;
     ++st.q_seen[0];
@@ -409,7 +419,7 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
           valid == C::BN ? kIdescQKFull
                          : (kIdescQK0 | ((uint32_t)(((valid + 15) & ~15) >> 3) << 17));
       const uint64_t kb = st.k + (uint64_t)((s * C::TILE_BYTES) >> 4);
-      ok = mbar_wait(bars + 8 * (C::B_KFULL + s), ph, abort_flag, a.status);
+      ok = mbar_wait(bars + 8 * (KF + s), ph, abort_flag, a.status);
       if (!ok) break;
       tc_fence_after();
       // QK_A(t)
@@ -424,7 +434,7 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
       if (has_b) {
         // QK_B(t)
         if (j == 0) {
-          ok = mbar_wait(bars + 8 * (C::B_QFULL + qslot_b), (st.q_seen[1] / C::QS) & 1,
+          ok = mbar_wait(bars + 8 * (QF + qslot_b), (st.q_seen[1] / C::QS) & 1,
                          abort_flag, a.status);
           if (!ok) break;
           ++st.q_seen[1];
@@ -508,11 +518,6 @@ __device__ __forceinline__ void rescale_o_row(uint32_t t_o, float alpha) {
   tmem_wait_st();
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
 
 // Score of a candidate row against its own key, scaled to log2 units (the diagonal term of the
 // mask). Plain CUDA-core dot product over 16-byte loads, half a row at a time.
@@ -647,22 +652,203 @@ __device__ __forceinline__ void finish_row(const AttnArgs& a, bool row_ok, int s
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// In-kernel right-anchored RoPE (ROPE instantiation)
+// ------------------------------------------------------------------------------------------
+// Swizzled shared-memory address of byte `byte_in_row` of row r of a landed tile: column block
+// byte_in_row / SW, and inside it the TMA's swizzle, which XORs the 16-byte chunk index with the
+// address bits three above it (tiles start on 1 KB boundaries).
+template <int D>
+__device__ __forceinline__ uint32_t tile_addr(uint32_t tile, int r, int byte_in_row) {
+  using C = Cfg<D>;
+  constexpr uint32_t kSwz = (uint32_t)(C::SW / 16 - 1) << 4;
+  const uint32_t a = tile + (uint32_t)((byte_in_row / C::SW) * C::BLK_BYTES + r * C::SW +
+                                       (byte_in_row % C::SW));
+  return a ^ ((a >> 3) & kSwz);
+}
+
+__device__ __forceinline__ uint4 lds_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+// (cos, sin) of the 8 pairs j = 8 cp .. 8 cp + 7 at position p, from the factor tables.
+template <int D>
+__device__ __forceinline__ void rope_factors(const AttnArgs& a, int p, int cp, float2 (&cs)[8]) {
+  constexpr int HALF = D / 2;
+  int64_t q;
+  int r;
+  rope_split((int64_t)p, q, r);
+  const float4* cq = reinterpret_cast<const float4*>(a.rope_coarse +
+                                                     (size_t)(a.rope_qmax - q) * HALF + 8 * cp);
+  const float4* cf = reinterpret_cast<const float4*>(a.rope_fine + (size_t)r * HALF + 8 * cp);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float4 c4 = __ldg(cq + e), f4 = __ldg(cf + e);
+    cs[2 * e] = rope_compose(make_float2(c4.x, c4.y), make_float2(f4.x, f4.y));
+    cs[2 * e + 1] = rope_compose(make_float2(c4.z, c4.w), make_float2(f4.z, f4.w));
+  }
+}
+
+// Rotates 8 pairs held as bf16 in (wa, wb) (first-half and second-half chunks of a row) and
+// rounds them to bf16 again, as the rotation pre-pass does.
+__device__ __forceinline__ void rope_chunk(uint4& va, uint4& vb, const float2 (&cs)[8]) {
+  uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+  uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float oa0, ob0, oa1, ob1;
+    rope_rotate(bf16_lo(wa[k]), bf16_lo(wb[k]), cs[2 * k], oa0, ob0);
+    rope_rotate(bf16_hi(wa[k]), bf16_hi(wb[k]), cs[2 * k + 1], oa1, ob1);
+    wa[k] = pack_bf16x2(oa0, oa1);
+    wb[k] = pack_bf16x2(ob0, ob1);
+  }
+  va = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+  vb = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+}
+
+// Rotates rows [0, rows) of a landed 128-row tile in place (kDiagThreads threads, index t): thread
+// t takes chunk pair cp = t % CP (pairs 8 cp .. 8 cp + 7, whose elements sit at bytes 16 cp and
+// 16 cp + D of the row) on every (kDiagThreads / CP)-th row. The rows of a tile belong to one user
+// and their positions rise by at most one per row, so they span fewer than 128 positions: two
+// coarse blocks q0, q0 + 1 at most, whose factors the thread loads once; the fine factors are
+// loaded for two rows at a time, so that their latencies overlap. Then the thread makes its
+// writes visible to the tensor core's reads.
+template <int D>
+__device__ __forceinline__ void rope_tile(const AttnArgs& a, uint32_t tile, const int32_t* pos,
+                                          int row0, int rows, int t) {
+  constexpr int CP = D / 16;
+  constexpr int STEP = kDiagThreads / CP;
+  constexpr int HALF = D / 2;
+  const int cp = t % CP;
+  if (rows > 0) {
+    int64_t q0;
+    int r_unused;
+    rope_split((int64_t)pos[row0], q0, r_unused);
+    float4 co[2][4];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      // Block q0 + 1 lies past the table when q0 is the last block; no position reaches it then.
+      const long long ci = a.rope_qmax - q0 - k;
+      const float4* cq = reinterpret_cast<const float4*>(
+          a.rope_coarse + (size_t)(ci < 0 ? 0 : ci) * HALF + 8 * cp);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) co[k][e] = __ldg(cq + e);
+    }
+    for (int r = t / CP; r < rows; r += 2 * STEP) {
+      const bool two = r + STEP < rows;
+      int64_t qq[2];
+      int rr[2];
+      rope_split((int64_t)pos[row0 + r], qq[0], rr[0]);
+      rope_split((int64_t)pos[row0 + (two ? r + STEP : r)], qq[1], rr[1]);
+      float4 fi[2][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float4* cf = reinterpret_cast<const float4*>(a.rope_fine + (size_t)rr[u] * HALF +
+                                                           8 * cp);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) fi[u][e] = __ldg(cf + e);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (u == 1 && !two) break;
+        const int row = r + u * STEP;
+        const uint32_t pa = tile_addr<D>(tile, row, 16 * cp);
+        const uint32_t pb = tile_addr<D>(tile, row, 16 * cp + D);
+        uint4 va = lds_v4(pa), vb = lds_v4(pb);
+        const int k = qq[u] == q0 ? 0 : 1;
+        float2 cs[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float4 c4 = k ? co[1][e] : co[0][e];
+          cs[2 * e] = rope_compose(make_float2(c4.x, c4.y), make_float2(fi[u][e].x, fi[u][e].y));
+          cs[2 * e + 1] =
+              rope_compose(make_float2(c4.z, c4.w), make_float2(fi[u][e].z, fi[u][e].w));
+        }
+        rope_chunk(va, vb, cs);
+        st_shared_v4(pa, va.x, va.y, va.z, va.w);
+        st_shared_v4(pb, vb.x, vb.y, vb.z, vb.w);
+      }
+    }
+  }
+  fence_proxy_async_smem();
+}
+
+// Score of a candidate row against its own key with both rotated to the row's position and
+// rounded to bf16 (the values the pre-pass would store), scaled to log2 units.
+template <int D>
+__device__ __forceinline__ float diag_score_rope(const AttnArgs& a, size_t base, int p) {
+  constexpr int CP = D / 16;
+  const uint4* qp = reinterpret_cast<const uint4*>(a.q + base);
+  const uint4* kp = reinterpret_cast<const uint4*>(a.dk + base);
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+  for (int cp = 0; cp < CP; ++cp) {
+    float2 cs[8];
+    rope_factors<D>(a, p, cp, cs);
+    uint4 qa = ld_global_nc_v4(qp + cp), qb = ld_global_nc_v4(qp + CP + cp);
+    uint4 ka = ld_global_nc_v4(kp + cp), kb = ld_global_nc_v4(kp + CP + cp);
+    rope_chunk(qa, qb, cs);
+    rope_chunk(ka, kb, cs);
+    const uint32_t q4[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+    const uint32_t k4[8] = {ka.x, ka.y, ka.z, ka.w, kb.x, kb.y, kb.z, kb.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      acc0 = fmaf(bf16_lo(q4[e]), bf16_lo(k4[e]), acc0);
+      acc1 = fmaf(bf16_hi(q4[e]), bf16_hi(k4[e]), acc1);
+    }
+  }
+  return (acc0 + acc1) * a.scale_log2;
+}
+
 // Diagonal scores, computed by two warps up to one item ahead of the softmax warps so that no
 // softmax thread waits on the q / k loads: thread t covers rows t, t + 64, t + 128 and t + 192 of
 // each item and deposits the score (-inf for a row without a diagonal term) in the item's slot of
 // a two-slot shared array; it also starts moving each candidate row's own value towards L2 for
 // the epilogue. Slot s is reused for the item after next once all 256 softmax threads have taken
 // the scores out of it.
-template <int D, bool CAUSAL>
-__device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
+template <int D, bool CAUSAL, bool ROPE>
+__device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t sbase, uint32_t bars,
                           volatile int* abort_flag, int t, ItemRing ring) {
   using C = Cfg<D>;
   uint32_t n = 0;
+  uint32_t nq[2] = {0, 0};   // ROPE: Q tiles rotated per query tile (mirrors the producer)
+  uint32_t g = 0;            // ROPE: K tiles rotated
   bool ok = true;
+  // ROPE: rotates the next landed K tile of the item (key tile j).
+  auto rotate_k = [&](const Item& w, int j) -> bool {
+    const int s = (int)(g % C::KVS);
+    if (!mbar_wait(bars + 8 * (C::B_KFULL + s), (g / C::KVS) & 1, abort_flag, a.status))
+      return false;
+    const int valid = min(C::BN, w.kv_len - j * C::BN);
+    rope_tile<D>(a, sbase + C::OFF_K + s * C::TILE_BYTES, a.kv_pos, w.kv_lo + j * C::BN, valid, t);
+    mbar_arrive(bars + 8 * (C::B_KREADY + s));
+    ++g;
+    return true;
+  };
   for (;; ++n) {
     const int it = ring_take(ring, abort_flag, a.status, ok);
     if (!ok || it < 0) return;
     const Item w = decode_item(a.items[it]);
+    if (ROPE && w.n_kv > 0) {
+      // The item's query tiles, then its first key tile, are rotated before anything else: the
+      // tensor core waits on them. The remaining key tiles follow the diagonal scores.
+      const int ntiles = w.nrows > C::BM ? 2 : 1;
+      for (int tt = 0; tt < ntiles; ++tt) {
+        const int slot = tt * C::QS + (int)(nq[tt] % C::QS);
+        if (!mbar_wait(bars + 8 * (C::B_QFULL + slot), (nq[tt] / C::QS) & 1, abort_flag,
+                       a.status))
+          return;
+        rope_tile<D>(a, sbase + C::OFF_Q + slot * C::TILE_BYTES, a.q_pos, w.q_row0 + tt * C::BM,
+                     min(C::BM, w.nrows - tt * C::BM), t);
+        mbar_arrive(bars + 8 * (C::B_QREADY + slot));
+        ++nq[tt];
+      }
+      if (!rotate_k(w, 0)) return;
+    }
     const int slot = n & 1;
     if (!mbar_wait(bars + 8 * (C::B_DIAGEMPTY + slot), ((n >> 1) & 1) ^ 1, abort_flag, a.status))
       return;
@@ -675,12 +861,15 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t bars,
 #pragma unroll
           for (int c = 0; c < D * 2; c += 128)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base + c / 2));
-          sd = diag_score<D>(a, base);
+          sd = ROPE ? diag_score_rope<D>(a, base, a.q_pos[row]) : diag_score<D>(a, base);
         }
       }
       sd_buf[slot * kItemRows + rr] = sd;
     }
     mbar_arrive(bars + 8 * (C::B_DIAGFULL + slot));
+    if (ROPE)
+      for (int j = 1; j < w.n_kv; ++j)
+        if (!rotate_k(w, j)) return;
   }
 }
 
@@ -786,9 +975,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
 
       // Pass 2: p = 2^(scale_log2 * s - m), written back over S_w as bf16 pairs (TMEM column k
       // holds keys 2k, 2k+1) 32 keys at a time; chunks past the last real key are never read
-      // by the trimmed PV and are skipped. Arithmetic runs on key pairs (packed fp32 FMA/add), and
-      // kEmuPairs of every 16 pairs take 2^x on the FMA pipe instead of the special-function
-      // unit, whose 16 results per clock would otherwise set the pace of the softmax.
+      // by the trimmed PV and are skipped. Arithmetic runs on key pairs (packed fp32 FMA/add).
       const float2 sl2v = make_float2(sl2, sl2), negv = make_float2(neg_m, neg_m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
 #pragma unroll
@@ -801,12 +988,8 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
                                                    __uint_as_float(x[32 * c + 2 * i + 1])),
                                        sl2v, negv);
           float2 p;
-          if ((i & 7) >= 8 - kEmuPairs / 2) {
-            p = exp2_fma2(xs);
-          } else {
-            p.x = fast_exp2(xs.x);
-            p.y = fast_exp2(xs.y);
-          }
+          p.x = fast_exp2(xs.x);
+          p.y = fast_exp2(xs.y);
           if ((i & 3) == 0) acc0 = __fadd2_rn(acc0, p);
           if ((i & 3) == 1) acc1 = __fadd2_rn(acc1, p);
           if ((i & 3) == 2) acc2 = __fadd2_rn(acc2, p);
@@ -857,12 +1040,15 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
 // ------------------------------------------------------------------------------------------
 // Kernel
 // ------------------------------------------------------------------------------------------
-template <int D, bool CAUSAL, bool LSE>
+template <int D, bool CAUSAL, bool LSE, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
     jagged_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using C = Cfg<D>;
+  // An empty queue (every user went to the candidate-only streaming kernel, or an error left no
+  // item): nothing to claim, so no CTA touches the queue counters; leave before any setup.
+  if (*a.n_items == 0) return;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -900,6 +1086,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars + 8 * (C::B_RINGFULL + i), 1);
       mbar_init(bars + 8 * (C::B_RINGEMPTY + i), kRingReaders);
     }
+    for (int i = 0; i < 2 * C::QS; ++i) mbar_init(bars + 8 * (C::B_QREADY + i), kDiagThreads);
+    for (int i = 0; i < C::KVS; ++i) mbar_init(bars + 8 * (C::B_KREADY + i), kDiagThreads);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
@@ -926,12 +1114,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane < 2)
         producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag, lane == 1, ring);
     } else if (warp == 1) {
-      if (lane == 0) mma_role<D, CAUSAL>(a, sbase, bars, tmem, abort_flag, ring);
+      if (lane == 0) mma_role<D, CAUSAL, ROPE>(a, sbase, bars, tmem, abort_flag, ring);
     } else if (warp < 10) {
       softmax_role<D, CAUSAL, LSE>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
                       abort_flag, warp, lane, ring);
     } else {
-      diag_role<D, CAUSAL>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), bars, abort_flag,
+      diag_role<D, CAUSAL, ROPE>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), sbase, bars,
+                                 abort_flag,
                    threadIdx.x - 320, ring);
     }
   }
@@ -973,13 +1162,16 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
   {
     std::lock_guard<std::mutex> lock(g_attr_mu);
     if (!g_attr_set[dev][d_index(D)]) {
-      if (cudaFuncSetAttribute(jagged_attn_kernel<D, false, false>,
+      if (cudaFuncSetAttribute(jagged_attn_kernel<D, false, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess ||
-          cudaFuncSetAttribute(jagged_attn_kernel<D, true, false>,
+          cudaFuncSetAttribute(jagged_attn_kernel<D, true, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess ||
-          cudaFuncSetAttribute(jagged_attn_kernel<D, false, true>,
+          cudaFuncSetAttribute(jagged_attn_kernel<D, false, true, false>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               C::SMEM_ALLOC) != cudaSuccess ||
+          cudaFuncSetAttribute(jagged_attn_kernel<D, false, false, true>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess)
         return JCA_ERR_CUDA;
@@ -996,14 +1188,17 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
   // Instantiations: the main path, the causal variant, and the training forward (log-sum-exp
   // output); each mode is compile-time so that the main path carries none of the others' code.
   if (a.causal)
-    jagged_attn_kernel<D, true, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
-                                                                                        tmV, args);
+    jagged_attn_kernel<D, true, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, args);
   else if (a.lse != nullptr)
-    jagged_attn_kernel<D, false, true><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
-                                                                                        tmV, args);
+    jagged_attn_kernel<D, false, true, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, args);
+  else if (a.rope)
+    jagged_attn_kernel<D, false, false, true><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, args);
   else
-    jagged_attn_kernel<D, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(tmQ, tmK,
-                                                                                         tmV, args);
+    jagged_attn_kernel<D, false, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, args);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }
 
@@ -1087,9 +1282,18 @@ extern "C" int jagged_cand_attn_plan(const void* offsets, const void* candidate_
 namespace jca {
 namespace {
 
+// In-kernel RoPE for run_full: positions of the rows and the factor tables (rope_device.cuh).
+struct RopeRun {
+  const int32_t* pos = nullptr;
+  const float2* coarse = nullptr;
+  const float2* fine = nullptr;
+  long long qmax = 0;
+};
+
 int run_full(const void* q, const void* k, const void* v, void* out, int out_fp32, float* lse,
              const int8_t* seg, int64_t B, int64_t T, int H, int d_head, float scale,
-             void* workspace, size_t workspace_bytes, int32_t* status, jca_stream_t stream) {
+             void* workspace, size_t workspace_bytes, int32_t* status, jca_stream_t stream,
+             const RopeRun* rope = nullptr) {
   int rc = check_sizes(32, d_head, B, T, T, H);
   if (rc) return rc;
   if (!status) return JCA_ERR_NULL;
@@ -1118,6 +1322,14 @@ int run_full(const void* q, const void* k, const void* v, void* out, int out_fp3
   a.out_fp32 = out_fp32 ? 1 : 0;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.lse = lse;
+  if (rope != nullptr) {
+    a.rope = 1;
+    a.q_pos = rope->pos;
+    a.kv_pos = rope->pos;
+    a.rope_coarse = rope->coarse;
+    a.rope_fine = rope->fine;
+    a.rope_qmax = rope->qmax;
+  }
   return launch_attention(d_head, a, q, T, k, v, T, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -1313,6 +1525,81 @@ extern "C" int cand_only_attn_fwd(const void* cand_q, const void* own_k, const v
   if (rc) return rc;
   return cand_only_attn_run(cand_q, own_k, own_v, hist_k, hist_v, hist_seg, out, out_fp32, B, Nc,
                             Th, H, d_head, scale, workspace, workspace_bytes, status, stream);
+}
+
+namespace jca {
+namespace {
+
+// Workspace of jagged_cand_attn_rope_fwd: the plan, then the positions and the factor tables.
+struct RopeLayout {
+  WorkspaceLayout base;
+  size_t pos = 0, coarse = 0, fine = 0, total = 0;
+};
+
+RopeLayout rope_layout(int64_t B, int64_t T, int H, int d) {
+  RopeLayout L;
+  L.base = workspace_layout(B, T, H);
+  size_t o = align_up(L.base.total, 256);
+  L.pos = o;
+  o = align_up(o + 4 * (size_t)T, 256);
+  L.coarse = o;
+  o = align_up(o + 8 * (size_t)(d / 2) * (size_t)(T / kRopeFine + 3), 256);
+  L.fine = o;
+  o = align_up(o + 8 * (size_t)(d / 2) * kRopeFine, 256);
+  L.total = o;
+  return L;
+}
+
+}  // namespace
+}  // namespace jca
+
+extern "C" size_t jca_rope_attn_workspace_bytes(int64_t B, int64_t T, int H, int d_head) {
+  if (B < 0 || T < 0 || H < 1 || !head_dim_ok(d_head)) return 0;
+  return rope_layout(B, T, H, d_head).total;
+}
+
+extern "C" int jagged_cand_attn_rope_fwd(const void* q, const void* k, const void* v, void* out,
+                                         int out_fp32, const void* offsets,
+                                         const void* candidate_start, const int8_t* seg, int64_t B,
+                                         int64_t T, int H, int d_head, float scale,
+                                         int64_t history_end, float rope_base, int idx_bits,
+                                         void* workspace, size_t workspace_bytes,
+                                         int32_t* status, jca_stream_t stream) {
+  int rc = check_sizes(idx_bits, d_head, B, T, T, H);
+  if (rc) return rc;
+  if (!(rope_base > 1.f) || history_end > (int64_t)INT_MAX || history_end - T < (int64_t)INT_MIN)
+    return JCA_ERR_SHAPE;
+  if (!status || !offsets) return JCA_ERR_NULL;
+  if (T > 0 && (!q || !k || !v || !out)) return JCA_ERR_NULL;
+  if (B > 0 && !seg && !candidate_start) return JCA_ERR_NULL;
+  if (T > 0 && (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)))
+    return JCA_ERR_ALIGN;
+  if (!workspace) return JCA_ERR_NULL;
+  if (!aligned(workspace, 256)) return JCA_ERR_ALIGN;
+  const RopeLayout L = rope_layout(B, T, H, d_head);
+  if (workspace_bytes < L.total) return JCA_ERR_WORKSPACE;
+  rc = jagged_cand_attn_plan(offsets, candidate_start, seg, B, T, H, d_head, idx_bits, workspace,
+                             workspace_bytes, status, stream);
+  if (rc) return rc;
+  if (T == 0) return JCA_OK;
+  char* ws = static_cast<char*>(workspace);
+  const int8_t* segp = seg ? seg : reinterpret_cast<const int8_t*>(ws + L.base.seg);
+  int32_t* pos = reinterpret_cast<int32_t*>(ws + L.pos);
+  rc = jca_rope_positions(segp, offsets, B, T, history_end, idx_bits, pos, status, stream);
+  if (rc) return rc;
+  const RopeTables tabs = rope_tables(T, history_end);
+  float2* coarse = reinterpret_cast<float2*>(ws + L.coarse);
+  float2* fine = reinterpret_cast<float2*>(ws + L.fine);
+  if (launch_rope_tables(coarse, fine, d_head, tabs, rope_base,
+                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JCA_ERR_CUDA;
+  RopeRun rr;
+  rr.pos = pos;
+  rr.coarse = coarse;
+  rr.fine = fine;
+  rr.qmax = tabs.qmax;
+  return run_full(q, k, v, out, out_fp32, nullptr, seg, B, T, H, d_head, scale, workspace,
+                  workspace_bytes, status, stream, &rr);
 }
 
 extern "C" size_t jca_seqpack_workspace_bytes(int64_t B, int64_t Th, int64_t Nc, int H,

@@ -297,26 +297,11 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// 2^x for two arguments on the FMA pipe, without the special-function unit. Cody-Waite range
-// reduction: x = n + f with n = round(x) and |f| <= 1/2; 2^f from a degree-3 minimax polynomial
-// p(f) = 1 + c1 f + c2 f^2 + c3 f^3 (constant term exactly 1; c1..c3 fitted by
-// exp2_poly_fit.py in the package); 2^n is added to the exponent field of p. The rounding adds
-// 1.5 * 2^23, which leaves round(x) in the low mantissa bits of the sum. Maximum relative error
-// about 1.0e-4 for results of at least 2^-126; arguments at or below -127 (and -inf) give +0.0,
-// arguments in (-127, -126) a non-negative value below 2^-126. Arguments must stay below 127.
-__device__ __forceinline__ float2 exp2_fma2(float2 x) {
-  constexpr float kC1 = 0x1.62f5fap-1f, kC2 = 0x1.f00c4ep-3f, kC3 = 0x1.c2a25cp-5f;
-  constexpr float kRound = 0x1.8p23f;
-  x.x = fmaxf(x.x, -127.f);
-  x.y = fmaxf(x.y, -127.f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 n = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(make_float2(kC3, kC3), f, make_float2(kC2, kC2));
-  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-  p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+// Maximum of three floats in one instruction (max.f32 with three sources, sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -88,6 +88,16 @@ cudaError_t launch_seqpack_plan(const void* hist_off, const void* cand_off, cons
                                 const WorkspaceLayout& L, size_t q_off2, int32_t* status,
                                 cudaStream_t stream);
 
+// Factor tables of the attention kernel's in-tile RoPE rotation (rope_device.cuh): positions lie in
+// [history_end - T, history_end], i.e. 128-position blocks q in [qmax - n_coarse + 1, qmax].
+struct RopeTables {
+  int64_t qmax = 0;
+  int64_t n_coarse = 0;
+};
+RopeTables rope_tables(int64_t T, int64_t history_end);
+cudaError_t launch_rope_tables(float2* coarse, float2* fine, int d, const RopeTables& t,
+                               float base, cudaStream_t stream);
+
 // Workspace of the candidate-packing entry points: workspace_layout(2B, T, H) followed by the
 // 2B + 1 query-run offsets.
 struct SeqpackLayout {

@@ -5,8 +5,9 @@
 //     it ends at history_end - 1 (padding takes the position the next segment-1 token would take,
 //     candidates take history_end);
 //   * rotation: rows of a [T, H, d] bf16 tensor rotated pairwise (element j with j + d/2) by
-//     pos * base^(-2j/d) (angle formed and reduced in fp64, rotation in fp32), rounded once to
-//     bf16. Memory-bound: one read and one write of the tensor, 16-byte accesses.
+//     pos * base^(-2j/d) (cos/sin as rope_device.cuh forms them, rotation in fp32), rounded once
+//     to bf16. Memory-bound: one read and one write of the tensor, 16-byte accesses.
+// and the cos/sin factor tables that the attention kernel's in-tile rotation reads.
 #include <climits>
 #include <cstdint>
 
@@ -14,6 +15,7 @@
 #include <cuda_runtime.h>
 
 #include "jca_internal.h"
+#include "rope_device.cuh"
 
 namespace jca {
 namespace {
@@ -91,8 +93,6 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const __nv_bfloat16* _
                                                           __nv_bfloat16* __restrict__ out,
                                                           const int32_t* __restrict__ pos,
                                                           int64_t T, int H, double log2_base) {
-  constexpr double kTwoPi = 6.283185307179586476925286766559;
-  constexpr double kInvTwoPi = 0.15915494309189533576888376337251;
   constexpr int HALF = D / 2;
   constexpr int UNITS = HALF / 8;   // 8-pair units per (row, head)
   static_assert(256 % UNITS == 0, "stride keeps each thread on one set of frequencies");
@@ -101,12 +101,14 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const __nv_bfloat16* _
   const int j0 = (int)(u0 % UNITS) * 8;
   double inv_freq[8];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) inv_freq[t] = exp2(-(double)(2 * (j0 + t)) / (double)D * log2_base);
+  for (int t = 0; t < 8; ++t) inv_freq[t] = rope_inv_freq(j0 + t, D, log2_base);
   for (int64_t u = u0; u < total; u += (int64_t)gridDim.x * blockDim.x) {
     const int64_t rh = u / UNITS;
     const int64_t row = rh / H;
     const size_t base = (size_t)rh * D;
-    const double p = (double)pos[row];
+    int64_t q;
+    int r;
+    rope_split((int64_t)pos[row], q, r);
     const uint4 va = *reinterpret_cast<const uint4*>(x + base + j0);
     const uint4 vb = *reinterpret_cast<const uint4*>(x + base + HALF + j0);
     const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
@@ -121,16 +123,9 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const __nv_bfloat16* _
       b2[1] = __uint_as_float(wb[k] & 0xffff0000u);
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        // The angle p * base^(-2j/d) reaches thousands of radians at the low frequencies: it is
-        // formed and reduced to [-pi, pi] in fp64, so that the sine and cosine see an argument
-        // accurate to fp32 precision rather than one off by p * 2^-24; on [-pi, pi] the fast
-        // intrinsic is accurate to about 2^-21, far below a bf16 ulp.
-        const double ang = p * inv_freq[2 * k + t];
-        const double red = ang - kTwoPi * rint(ang * kInvTwoPi);
-        float sn, cs;
-        __sincosf((float)red, &sn, &cs);
-        oa[t] = a2[t] * cs - b2[t] * sn;
-        ob[t] = a2[t] * sn + b2[t] * cs;
+        const double f = inv_freq[2 * k + t];
+        const float2 cs = rope_compose(rope_cs((double)(q * kRopeFine), f), rope_cs((double)r, f));
+        rope_rotate(a2[t], b2[t], cs, oa[t], ob[t]);
       }
       __nv_bfloat162 ha = __floats2bfloat162_rn(oa[0], oa[1]);
       __nv_bfloat162 hb = __floats2bfloat162_rn(ob[0], ob[1]);
@@ -139,6 +134,25 @@ __global__ void __launch_bounds__(256) rope_rotate_kernel(const __nv_bfloat16* _
     }
     *reinterpret_cast<uint4*>(out + base + j0) = make_uint4(ra[0], ra[1], ra[2], ra[3]);
     *reinterpret_cast<uint4*>(out + base + HALF + j0) = make_uint4(rb[0], rb[1], rb[2], rb[3]);
+  }
+}
+
+// The factor tables of the in-tile rotation: coarse[i][j] = (cos, sin)(128 (qmax - i) theta_j) for
+// i in [0, n_coarse), fine[r][j] = (cos, sin)(r theta_j) for r in [0, 128); theta_j as above.
+__global__ void __launch_bounds__(256) rope_table_kernel(float2* __restrict__ coarse,
+                                                         float2* __restrict__ fine, int half,
+                                                         int d, int64_t qmax, int64_t n_coarse,
+                                                         double log2_base) {
+  const int64_t n = (n_coarse + kRopeFine) * half;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t i = e / half;
+    const int j = (int)(e - i * half);
+    const double f = rope_inv_freq(j, d, log2_base);
+    if (i < n_coarse)
+      coarse[e] = rope_cs((double)((qmax - i) * kRopeFine), f);
+    else
+      fine[e - n_coarse * half] = rope_cs((double)(i - n_coarse), f);
   }
 }
 
@@ -154,6 +168,28 @@ int sm_count() {
 }
 
 }  // namespace
+
+RopeTables rope_tables(int64_t T, int64_t history_end) {
+  RopeTables t;
+  // Positions lie in [history_end - T, history_end]: a row's segment-1 run is at most T long.
+  auto fl = [](int64_t p) { return p >= 0 ? p / kRopeFine : -((-p + kRopeFine - 1) / kRopeFine); };
+  const int64_t qmax = fl(history_end), qmin = fl(history_end - T);
+  t.qmax = qmax;
+  t.n_coarse = qmax - qmin + 1;
+  return t;
+}
+
+cudaError_t launch_rope_tables(float2* coarse, float2* fine, int d, const RopeTables& t,
+                               float base, cudaStream_t stream) {
+  const int half = d / 2;
+  const int64_t n = (t.n_coarse + kRopeFine) * half;
+  const int64_t want = (n + 255) / 256;
+  const int grid = (int)(want < (int64_t)sm_count() * 8 ? want : (int64_t)sm_count() * 8);
+  rope_table_kernel<<<grid, 256, 0, stream>>>(coarse, fine, half, d, t.qmax, t.n_coarse,
+                                              log2((double)base));
+  return cudaGetLastError();
+}
+
 }  // namespace jca
 
 using namespace jca;

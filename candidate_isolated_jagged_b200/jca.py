@@ -61,6 +61,10 @@ _SIGNATURES = {
     "jagged_cand_attn_bwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
                                      c_i32, c_vp, c_vp, c_vp, c_i64, c_i64, c_i32, c_i32, c_f32,
                                      c_i32, c_vp, c_sz, c_vp, c_vp]),
+    "jca_rope_attn_workspace_bytes": (c_sz, [c_i64, c_i64, c_i32, c_i32]),
+    "jagged_cand_attn_rope_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_i64,
+                                          c_i64, c_i32, c_i32, c_f32, c_i64, c_f32, c_i32, c_vp,
+                                          c_sz, c_vp, c_vp]),
     "jca_seqpack_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i32, c_i32]),
     "jca_seqpack_bwd_workspace_bytes": (c_sz, [c_i64, c_i64, c_i64, c_i32, c_i32]),
     "jagged_cand_attn_seqpack_fwd": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp, c_vp,
@@ -425,6 +429,31 @@ def jagged_cand_attn_bwd(q, k, v, out, dout, lse, dq, dk, dv, offsets, candidate
         _ptr(dv), grad_fp32, _ptr(offsets), _ptr(candidate_start), _ptr(seg), B, T, H, d,
         float(scale), _idx_bits(offsets), _ptr(workspace), workspace.numel(), _ptr(status),
         _stream(stream)), "jagged_cand_attn_bwd")
+
+
+def jca_rope_attn_workspace_bytes(B: int, T: int, H: int, d_head: int) -> int:
+    return int(lib().jca_rope_attn_workspace_bytes(int(B), int(T), int(H), int(d_head)))
+
+
+def jagged_cand_attn_rope_fwd(q, k, v, out, offsets, candidate_start=None, seg=None,
+                              history_end: int = 0, rope_base: float = 10000.0, scale: float = 0.0,
+                              workspace: Optional[torch.Tensor] = None,
+                              status: Optional[torch.Tensor] = None, stream=None) -> int:
+    """Jagged candidate-isolated attention with right-anchored RoPE rotated inside the kernel
+    (q and k unrotated, left unchanged)."""
+    T, H, d = q.shape
+    B = offsets.numel() - 1
+    if workspace is None:
+        workspace = torch.empty(max(1, jca_rope_attn_workspace_bytes(B, T, H, d)),
+                                dtype=torch.uint8, device=q.device)
+    if status is None:
+        status = new_status(q.device)
+    out_fp32 = 1 if out.dtype == torch.float32 else 0
+    return _check(lib().jagged_cand_attn_rope_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), _ptr(candidate_start),
+        _ptr(seg), B, T, H, d, float(scale), int(history_end), float(rope_base),
+        _idx_bits(offsets), _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
+        "jagged_cand_attn_rope_fwd")
 
 
 def jca_seqpack_workspace_bytes(B: int, Th: int, Nc: int, H: int, d_head: int) -> int:

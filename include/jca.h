@@ -326,6 +326,25 @@ int jca_rope_positions(const int8_t* seg, const void* offsets, int64_t B, int64_
 int jca_apply_rope(const void* x, void* out, const int32_t* positions, int64_t T, int H,
                    int d_head, float base, jca_stream_t stream);
 
+/* jagged_cand_attn_fwd with right-anchored RoPE applied inside the attention kernel: q and k are
+ * given UNROTATED and are left unchanged; each Q and K tile is rotated in shared memory, after it
+ * lands and before the tensor core reads it, by the positions jca_rope_positions gives the batch's
+ * segment IDs (history_end as there) and base rope_base. The rotated values are those
+ * jca_apply_rope would store (the same cosines and sines, rotation in fp32, one rounding to bf16),
+ * so the output equals jca_apply_rope on q and k followed by jagged_cand_attn_fwd, up to the
+ * summation order of the candidates' own scores. Saves that pre-pass's read and write of q and k.
+ *   Other arguments as jagged_cand_attn_fwd; rope_base > 1; positions must fit int32
+ *   (history_end <= INT32_MAX and history_end - T >= INT32_MIN, else JCA_ERR_SHAPE).
+ *   workspace >= jca_rope_attn_workspace_bytes(B, T, H, d_head) bytes, 256-byte aligned.
+ * Device errors: as jagged_cand_attn_fwd. */
+size_t jca_rope_attn_workspace_bytes(int64_t B, int64_t T, int H, int d_head);
+
+int jagged_cand_attn_rope_fwd(const void* q, const void* k, const void* v, void* out, int out_fp32,
+                              const void* offsets, const void* candidate_start, const int8_t* seg,
+                              int64_t B, int64_t T, int H, int d_head, float scale,
+                              int64_t history_end, float rope_base, int idx_bits, void* workspace,
+                              size_t workspace_bytes, int32_t* status, jca_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Variant: per-user causal attention on the packed layout (prior art on the pages: the early
  * demo ranker's lower-triangular mask, noted in the FAQ of 候选隔离注意力掩码, and the

@@ -1,6 +1,7 @@
 """GPU parity of cand_only_attn_fwd (candidate queries over frozen history K/V plus their own K/V)
 against the oracle, its equality with the candidate rows of the full op, and the two candidate-only
-workloads at full size on sampled rows."""
+workloads at full size on sampled rows, plus key counts on and around the 128-key tile edges,
+history padding at the ends of a key interval, and many short users over several head counts."""
 
 import numpy as np
 import pytest
@@ -84,3 +85,49 @@ def test_cand_only_bad_history_segment():
     jca.cand_only_attn_fwd(r.cq, r.ck, r.cv, r.coff, r.hk, r.hv, r.hoff, out, r.hseg, status=st)
     assert int(st.item()) == 5
     assert torch.all(out == 3.0)
+
+
+@pytest.mark.parametrize("idx", [torch.int32, torch.int64])
+@pytest.mark.parametrize("d", [16, 32, 64])
+def test_cand_only_key_and_row_boundaries(d, idx):
+    # key counts 0..600 on and around the 128-key tile edges; candidate counts on and around the
+    # 128-row tile edges
+    hist = [1, 2, 15, 16, 17, 127, 128, 129, 255, 256, 257, 0, 600]
+    cands = [129, 1, 300, 128, 5, 256, 3, 127, 140, 700, 9, 4, 130]
+    cb = synth.custom_cand_only(hist, cands, H=3, d=d, seed=30 + d)
+    r = CandOnlyRun(cb, idx=idx)
+    ref = r.reference()
+    out = r.run()
+    assert_close(out, ref, f"cand-only boundaries d={d}")
+    assert_close_bf16(r.run(out_fp32=False), ref, f"cand-only boundaries bf16 d={d}")
+    assert torch.equal(out, r.run())   # the same bits every call
+
+
+@pytest.mark.parametrize("d", [16, 32, 64])
+def test_cand_only_history_holes_at_interval_ends(d):
+    # padding rows inside the key interval are masked; padding at both ends of a 300-row history
+    # shrinks its key interval to 256 keys
+    hist = [40, 256, 200, 300, 3, 130]
+    cands = [300, 77, 1000, 64, 260, 1]
+    cb = synth.custom_cand_only(hist, cands, H=2, d=d, seed=40 + d)
+    rng = np.random.default_rng(d)
+    hseg = (rng.random(cb.Th) > 0.25).astype(np.int8)
+    off = oracle.offsets_from_lengths(hist)
+    s3 = int(off[3])
+    hseg[s3:s3 + 300] = 1
+    hseg[s3:s3 + 20] = 0
+    hseg[s3 + 276:s3 + 300] = 0
+    r = CandOnlyRun(cb, hist_seg=hseg)
+    assert_close(r.run(), r.reference(), f"cand-only with history padding d={d}")
+
+
+@pytest.mark.parametrize("H,d", [(2, 32), (5, 32), (6, 16), (3, 64)])
+def test_cand_only_many_short_users(H, d):
+    # 150 short users with few candidates each: many items of a single key tile and a single
+    # query tile, over several head counts
+    rng = np.random.default_rng(7 + H)
+    hist = rng.integers(1, 257, 150)
+    cands = rng.integers(1, 300, 150)
+    cb = synth.custom_cand_only(hist, cands, H=H, d=d, seed=8)
+    r = CandOnlyRun(cb)
+    assert_close(r.run(), r.reference(), f"cand-only, 150 users, H={H}, d={d}")

@@ -1,6 +1,10 @@
 """GPU parity of the right-anchored RoPE kernels against the oracle (oracle/rope.py): positions
 bit-exact, rotated rows within one bf16 ulp, and attention on rotated queries and keys within the
-usual attention tolerance, plus the candidate-order invariance the pages state."""
+usual attention tolerance, plus the candidate-order invariance the pages state. The fused entry
+point (jagged_cand_attn_rope_fwd, tiles rotated inside the attention kernel) is checked against the
+oracle under the same bars, and against the pre-pass path: history rows bit-identical (the same
+rotated bf16 tiles, the same MMAs), candidate rows within 1e-5 (their own score is summed in
+another order)."""
 
 import numpy as np
 import pytest
@@ -55,15 +59,18 @@ def test_positions_bad_offsets():
 
 
 def _within_one_ulp(got, ref, x):
-    # One bf16 ulp of the result, plus the fp32 rounding of a*cos - b*sin relative to the
-    # inputs' size (which matters only where the two terms cancel).
+    # One bf16 ulp of the result, plus the error of the fp32 cosine and sine relative to the
+    # inputs' size (which matters only where the two terms of a*cos - b*sin cancel). The kernels
+    # compose cos/sin(p theta) from the factors at 128 q and r (p = 128 q + r), each accurate to
+    # about 2^-21 (fast intrinsics on an fp64-reduced argument); with the fp32 products of the
+    # composition and of the rotation the bound is about 3 * 2^-21, under 2^-19.
     got = got.detach().to("cpu", torch.float64).numpy()
     x = x.to(torch.float64).numpy()
     half = x.shape[-1] // 2
     mag = np.abs(x[..., :half]) + np.abs(x[..., half:])
     mag = np.concatenate([mag, mag], axis=-1)
     ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126))) - 7)
-    return np.abs(got - ref) <= ulp + 2.0 ** -22 * mag
+    return np.abs(got - ref) <= ulp + 2.0 ** -19 * mag
 
 
 @pytest.mark.parametrize("d", [16, 32, 64, 128])
@@ -159,3 +166,77 @@ def test_cand_only_with_rope():
     rhk = oracle.round_to_bf16(oracle.apply_rope(cb.hk, hpos_np))
     ref = oracle.cand_only_attn(rq, rk, cb.cv, r.coff_np, rhk, cb.hv, r.hoff_np, None, cb.scale)
     assert_close(out, ref, "cand-only with RoPE")
+
+
+def _fused(b, history_end=1000, idx=torch.int64, out_fp32=True):
+    r = FullRun(b, idx=idx)
+    out = torch.full(b.q.shape, float("nan"), dtype=torch.float32 if out_fp32 else torch.bfloat16,
+                     device=dev())
+    st = jca.new_status(dev())
+    jca.jagged_cand_attn_rope_fwd(r.q, r.k, r.v, out, r.off, r.cs, r.seg, history_end=history_end,
+                                  status=st)
+    torch.cuda.synchronize()
+    jca.check_status(st, "rope fused")
+    return out, r
+
+
+FUSED = {
+    "tiny": lambda: synth.tiny(),
+    "holes_d32": lambda: synth.custom_batch([0, 7, 300, 129, 1], prefix=[2, 0, 4, 1, 0],
+                                            n_cand=[5, 1, 140, 0, 3], H=3, d=32, seed=4,
+                                            pad_hist_to=16),
+    "three_users": lambda: synth.three_users(),
+    "d128_edges": lambda: synth.custom_batch([0, 1, 127, 128, 129, 255, 300], prefix=[0, 1, 2, 0, 4, 1, 3],
+                                             n_cand=[3, 0, 64, 1, 130, 2, 257], H=2, d=128, seed=12),
+}
+
+
+@pytest.mark.parametrize("history_end", [1000, 0, -300])
+@pytest.mark.parametrize("name", list(FUSED))
+def test_fused_rope_matches_oracle_and_prepass(name, history_end):
+    b = FUSED[name]()
+    out, r = _fused(b, history_end)
+    pos_np = oracle.right_anchored_positions(r.off_np, r.seg_np, history_end)
+    q = oracle.round_to_bf16(oracle.apply_rope(b.q, pos_np))
+    k = oracle.round_to_bf16(oracle.apply_rope(b.k, pos_np))
+    ref = oracle.jagged_cand_attn(q, k, b.v, r.off_np, r.seg_np, b.scale)
+    assert_close(out, ref, f"fused rope {name}")
+    # the caller's q and k are left unrotated
+    assert torch.equal(r.q.cpu(), b.q) and torch.equal(r.k.cpu(), b.k)
+    pre, ref2, _ = _rope_full(b, history_end)
+    hist = torch.from_numpy(r.seg_np != -1).to(dev())
+    assert torch.equal(out[hist], pre[hist])
+    assert_close(out, pre.double().cpu().numpy(), f"fused vs pre-pass {name}", max_abs=1e-5,
+                 rel_l2=1e-5)
+
+
+@pytest.mark.parametrize("idx", IDX)
+def test_fused_rope_bf16_output_and_index_types(idx):
+    b = FUSED["holes_d32"]()
+    out, r = _fused(b, 77, idx=idx, out_fp32=False)
+    pos_np = oracle.right_anchored_positions(r.off_np, r.seg_np, 77)
+    q = oracle.round_to_bf16(oracle.apply_rope(b.q, pos_np))
+    k = oracle.round_to_bf16(oracle.apply_rope(b.k, pos_np))
+    from helpers import assert_close_bf16
+    assert_close_bf16(out, oracle.jagged_cand_attn(q, k, b.v, r.off_np, r.seg_np, b.scale),
+                      "fused rope bf16")
+
+
+def test_fused_rope_users256_sampled():
+    """The 256-user workload with in-kernel RoPE (history_end 4096), in the launch configuration
+    the benchmark times, checked on every row of eight users (an empty history, the 4096-token
+    user, the median, the 200th longest and four more): users never interact, so the oracle runs
+    on a batch of just those users."""
+    b = synth.users256()
+    out, r = _fused(b, 4096)
+    order = np.argsort(b.hist_real)
+    users = [0, 1, int(order[128]), int(order[200]), 5, 77, 130, 255]
+    rows = np.concatenate([np.arange(r.off_np[u], r.off_np[u + 1]) for u in users])
+    soff = oracle.offsets_from_lengths(b.row_lengths[users])
+    sseg = r.seg_np[rows]
+    pos_np = oracle.right_anchored_positions(soff, sseg, 4096)
+    rt = torch.from_numpy(rows)
+    q = oracle.round_to_bf16(oracle.apply_rope(b.q[rt], pos_np))
+    k = oracle.round_to_bf16(oracle.apply_rope(b.k[rt], pos_np))
+    ref = oracle.jagged_cand_attn(q, k, b.v[rt], soff, sseg, b.scale)
+    assert_close(out[rt.to(dev())], ref, "fused rope users256 sampled")
