@@ -1046,9 +1046,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
   using C = Cfg<D>;
-  // An empty queue (every user went to the candidate-only streaming kernel, or an error left no
-  // item): nothing to claim, so no CTA touches the queue counters; leave before any setup.
-  if (*a.n_items == 0) return;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;

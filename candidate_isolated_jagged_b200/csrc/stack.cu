@@ -221,9 +221,7 @@ __global__ void __launch_bounds__(256) split_rows_kernel(bf16* __restrict__ x,
 // ---------------------------------------------------------------------------------------------
 // Projections on cuBLASLt: Y[M, N] = X[M, K] W[K, N] (+ R[M, N]), all row-major bf16, fp32
 // accumulation, one rounding to bf16. In cuBLASLt's column-major terms this is
-// Y^T (N x M) = W^T (N x K) * X^T (K x M) with no transposes. With batch > 1 one call computes
-// Y_i = X W_i for `batch` consecutive weight matrices (K x N apart) into consecutive outputs
-// (M x N apart): the query, key and value projections of a layer in one launch.
+// Y^T (N x M) = W^T (N x K) * X^T (K x M) with no transposes.
 // ---------------------------------------------------------------------------------------------
 constexpr size_t kLtWorkspace = size_t(32) << 20;
 constexpr int kMaxDevices = 64;
@@ -247,9 +245,8 @@ struct LtDescs {
 };
 
 int gemm_bf16(const bf16* X, const bf16* W, const bf16* R, bf16* Y, int64_t M, int N, int K,
-              void* lt_ws, cudaStream_t stream, int batch = 1) {
+              void* lt_ws, cudaStream_t stream) {
   if (M == 0) return JCA_OK;
-  if (batch > 1 && R != nullptr) return JCA_ERR_SHAPE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return JCA_ERR_CUDA;
   LtDescs d;
@@ -263,23 +260,6 @@ int gemm_bf16(const bf16* X, const bf16* W, const bf16* R, bf16* Y, int64_t M, i
       cublasLtMatrixLayoutCreate(&d.b, CUDA_R_16BF, K, M, K) != CUBLAS_STATUS_SUCCESS ||
       cublasLtMatrixLayoutCreate(&d.c, CUDA_R_16BF, N, M, N) != CUBLAS_STATUS_SUCCESS)
     return JCA_ERR_CUDA;
-  if (batch > 1) {
-    const int32_t cnt = batch;
-    const int64_t sa = (int64_t)N * K, sb = 0, sc = (int64_t)N * M;
-    if (cublasLtMatrixLayoutSetAttribute(d.a, CUBLASLT_MATRIX_LAYOUT_BATCH_COUNT, &cnt,
-                                         sizeof(cnt)) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutSetAttribute(d.b, CUBLASLT_MATRIX_LAYOUT_BATCH_COUNT, &cnt,
-                                         sizeof(cnt)) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutSetAttribute(d.c, CUBLASLT_MATRIX_LAYOUT_BATCH_COUNT, &cnt,
-                                         sizeof(cnt)) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutSetAttribute(d.a, CUBLASLT_MATRIX_LAYOUT_STRIDED_BATCH_OFFSET, &sa,
-                                         sizeof(sa)) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutSetAttribute(d.b, CUBLASLT_MATRIX_LAYOUT_STRIDED_BATCH_OFFSET, &sb,
-                                         sizeof(sb)) != CUBLAS_STATUS_SUCCESS ||
-        cublasLtMatrixLayoutSetAttribute(d.c, CUBLASLT_MATRIX_LAYOUT_STRIDED_BATCH_OFFSET, &sc,
-                                         sizeof(sc)) != CUBLAS_STATUS_SUCCESS)
-      return JCA_ERR_CUDA;
-  }
   cublasLtHandle_t handle;
   cublasLtMatmulAlgo_t algo;
   {
@@ -290,7 +270,7 @@ int gemm_bf16(const bf16* X, const bf16* W, const bf16* R, bf16* Y, int64_t M, i
       return JCA_ERR_CUDA;
     }
     handle = L.handle;
-    const auto key = std::make_tuple(M, N, K, (R ? 1 : 0) | (batch << 1));
+    const auto key = std::make_tuple(M, N, K, R ? 1 : 0);
     auto it = L.algos.find(key);
     if (it == L.algos.end()) {
       cublasLtMatmulPreference_t pref = nullptr;
@@ -433,8 +413,12 @@ extern "C" int jca_stack_fwd(const void* x, void* x_out, const void* weights, in
   bf16* v = k + (int64_t)T * D;
   for (int l = 0; l < n_full; ++l) {
     const bf16* W = Wt + (int64_t)l * 4 * DD;
-    // Q, K and V in one batched GEMM (the three weights are consecutive, and so are q, k, v).
-    if ((rc = gemm_bf16(cur, W, nullptr, q, T, D, D, lt_ws, st, 3))) return rc;
+    // Q, K and V as three GEMMs: one batched GEMM over the three consecutive weights measured
+    // slower (0.1 ms per layer on users256), cuBLASLt's heuristic picking a slower kernel for it.
+    if ((rc = gemm_bf16(cur, W, nullptr, q, T, D, D, lt_ws, st)) ||
+        (rc = gemm_bf16(cur, W + DD, nullptr, k, T, D, D, lt_ws, st)) ||
+        (rc = gemm_bf16(cur, W + 2 * DD, nullptr, v, T, D, D, lt_ws, st)))
+      return rc;
     // RoPE as a pre-pass over Q and K: each key row is rotated once here, whereas the kernel's
     // in-tile rotation (jagged_cand_attn_rope_fwd) rotates a key tile again for every query block
     // of its user and head, which measured slower on this workload.
@@ -490,8 +474,11 @@ extern "C" int jca_stack_fwd(const void* x, void* x_out, const void* weights, in
   bf16* hv = hk + Th * D;
   for (int l = n_full; l < n_layers; ++l) {
     const bf16* W = Wt + (int64_t)l * 4 * DD;
-    if ((rc = gemm_bf16(xc, W, nullptr, cq, Nc, D, D, lt_ws, st, 3)) ||
-        (rc = gemm_bf16(xh, W + DD, nullptr, hk, Th, D, D, lt_ws, st, 2)))
+    if ((rc = gemm_bf16(xc, W, nullptr, cq, Nc, D, D, lt_ws, st)) ||
+        (rc = gemm_bf16(xc, W + DD, nullptr, ck, Nc, D, D, lt_ws, st)) ||
+        (rc = gemm_bf16(xc, W + 2 * DD, nullptr, cv, Nc, D, D, lt_ws, st)) ||
+        (rc = gemm_bf16(xh, W + DD, nullptr, hk, Th, D, D, lt_ws, st)) ||
+        (rc = gemm_bf16(xh, W + 2 * DD, nullptr, hv, Th, D, D, lt_ws, st)))
       return rc;
     if (rope && ((rc = jca_apply_rope(cq, cq, spos + Th, Nc, H, d_head, rope_base, stream)) ||
                  (rc = jca_apply_rope(ck, ck, spos + Th, Nc, H, d_head, rope_base, stream)) ||
