@@ -80,6 +80,7 @@ _SIGNATURES = {
     "jca_noalloc_scratch_bytes": (c_sz, []),
     "jca_noalloc_prepare": (c_i32, []),
     "jca_user_tile_cost": (c_i64, [c_i64, c_i64]),
+    "jca_selftest_wait_timeout": (c_i32, [c_vp, c_vp]),
     "jca_shard_users": (c_i32, [c_vp, c_vp, c_i64, c_i32, c_vp, c_vp]),
     "jagged_cand_attn_fwd_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i32, c_vp, c_vp, c_vp,
                                              c_i64, c_i64, c_i32, c_i32, c_f32, c_i32, c_vp,
@@ -310,6 +311,13 @@ def jagged_cand_attn_fwd_noalloc(q, k, v, out, offsets, candidate_start=None, se
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), out_fp32, _ptr(offsets), _ptr(candidate_start),
         _ptr(seg), B, T, H, d, float(scale), _idx_bits(offsets), _ptr(status), _stream(stream)),
         "jagged_cand_attn_fwd_noalloc")
+
+
+def jca_selftest_wait_timeout(status, stream=None) -> int:
+    """One block that runs the library's bounded pipeline wait on a barrier nothing completes:
+    *status becomes JCA_STATUS_TIMEOUT (16) after about 2 s, and the context stays usable."""
+    return _check(lib().jca_selftest_wait_timeout(_ptr(status), _stream(stream)),
+                  "jca_selftest_wait_timeout")
 
 
 def shard_users(row_lengths, n_keys, n_shards: int):

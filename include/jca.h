@@ -271,6 +271,13 @@ int jagged_cand_attn_fwd_noalloc(const void* q, const void* k, const void* v, vo
                                  const int8_t* seg, int64_t B, int64_t T, int H, int d_head,
                                  float scale, int idx_bits, int32_t* status, jca_stream_t stream);
 
+/* Self-test of the failure path (no counterpart on the pages): launches one block whose thread runs
+ * the library's bounded pipeline wait on a barrier that nothing completes. After the wait's limit
+ * (2 s) it records JCA_STATUS_TIMEOUT in *status (if *status was 0) and the block returns, as a
+ * kernel whose pipeline stalls does; the context stays usable. Enqueues one kernel on `stream`.
+ * Errors: JCA_ERR_NULL, JCA_ERR_DEVICE, JCA_ERR_CUDA. */
+int jca_selftest_wait_timeout(int32_t* status, jca_stream_t stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Several GPUs: users are independent (no position reads across a user boundary: 候选隔离注意力掩码,
  * section 段 ID：掩码的表达方式; 'HSTU scale' tutorial, section 手算 padding 的浪费与 offset), so one

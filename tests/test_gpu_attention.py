@@ -130,3 +130,21 @@ def test_data_errors_leave_output_untouched():
     jca.jagged_cand_attn_fwd(r.q, r.k, r.v, out, bad_off, r.cs, None, status=st)
     assert int(st.item()) == 2
     assert torch.all(out == 7.0)
+
+
+def test_pipeline_wait_timeout_is_recoverable():
+    """The failure path without a GPU fault: a bounded wait that nothing completes gives up after
+    its limit and records JCA_STATUS_TIMEOUT; the status word then stops later calls that share it,
+    and the context keeps working for calls with a fresh status word."""
+    st = jca.new_status(dev())
+    jca.jca_selftest_wait_timeout(st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 16
+    assert "timed out" in jca.status_string(16)
+    b = synth.tiny()
+    r = FullRun(b)
+    out = torch.full(b.q.shape, 7.0, dtype=torch.float32, device=dev())
+    jca.jagged_cand_attn_fwd(r.q, r.k, r.v, out, r.off, r.cs, r.seg, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 16 and bool((out == 7.0).all())   # nothing written after an error
+    assert_close(r.run(out_fp32=True), r.reference(), "after a timeout")
