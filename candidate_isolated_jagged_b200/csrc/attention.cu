@@ -850,6 +850,22 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t sbase, uint
       if (!rotate_k(w, 0)) return;
     }
     const int slot = n & 1;
+    // Candidate-only layer (every row a candidate) with heads of 64 or more: first every row's own
+    // query, key and value towards L2, so that the score loads below wait about one memory
+    // latency in all instead of one per row (3 % on the 512-candidate workload; on the full
+    // layer, where few rows are candidates, and at d = 32 it measured slightly slower).
+    const bool bulk_prefetch = !CAUSAL && a.q_seg == nullptr && D >= 64;
+    if (bulk_prefetch) {
+      for (int rr = t; rr < w.nrows; rr += kDiagThreads) {
+        const size_t base = ((size_t)(w.q_row0 + rr) * (size_t)a.H + (size_t)w.h) * D;
+#pragma unroll
+        for (int c = 0; c < D * 2; c += 128) {
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.q + base + c / 2));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dk + base + c / 2));
+          asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base + c / 2));
+        }
+      }
+    }
     if (!mbar_wait(bars + 8 * (C::B_DIAGEMPTY + slot), ((n >> 1) & 1) ^ 1, abort_flag, a.status))
       return;
     for (int rr = t; rr < kItemRows; rr += kDiagThreads) {
@@ -858,9 +874,11 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t sbase, uint
         const int row = w.q_row0 + rr;
         if (!CAUSAL && (!a.q_seg || a.q_seg[row] == -1)) {
           const size_t base = ((size_t)row * (size_t)a.H + (size_t)w.h) * D;
+          if (!bulk_prefetch) {
 #pragma unroll
-          for (int c = 0; c < D * 2; c += 128)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base + c / 2));
+            for (int c = 0; c < D * 2; c += 128)
+              asm volatile("prefetch.global.L2 [%0];" ::"l"(a.dv + base + c / 2));
+          }
           sd = ROPE ? diag_score_rope<D>(a, base, a.q_pos[row]) : diag_score<D>(a, base);
         }
       }
