@@ -280,14 +280,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     status = jca.new_status(dev)
     launches_per_step = 4  # offsets, segment IDs + bounds (one pass), work queue, attention
 
-    def step(ev=None):
-        jca.jca_offsets_from_lengths(lengths, offsets, status, stream)
-        jca.jagged_cand_attn_plan(offsets, cand_start, None, T, H, d, ws, status, stream)
+    def step(ev=None, s=stream):
+        jca.jca_offsets_from_lengths(lengths, offsets, status, s)
+        jca.jagged_cand_attn_plan(offsets, cand_start, None, T, H, d, ws, status, s)
         if ev is not None:
-            ev[0].record(stream)
-        jca.jagged_cand_attn_run(q, k, v, out, None, B, ws, status, stream=stream)
+            ev[0].record(s)
+        jca.jagged_cand_attn_run(q, k, v, out, None, B, ws, status, stream=s)
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(s)
 
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
@@ -305,15 +305,36 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize(dev)
         jca.check_status(status, "warm-up")
         assert bool(torch.isfinite(out.float()).all()), "non-finite attention output"
+        # The step's four launches (offsets, segment IDs + bounds, work queue, attention) as one
+        # CUDA graph, replayed once per timed step: the same kernels and work, without the host
+        # launch gaps between them. Every call is capturable (no host synchronisation, no
+        # allocation).
+        graph = None
+        if not args.no_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step(s=torch.cuda.current_stream(dev))
+            graph.replay()
+            torch.cuda.synchronize(dev)
+            jca.check_status(status, "graph warm-up")
         if dist:
             dist.barrier()
         torch.cuda.synchronize(dev)
         sampler.mark()
         t_start.record(stream)
         for i in range(args.steps):
-            step(kev[i])
+            if graph is not None:
+                graph.replay()
+            else:
+                step(kev[i])
         t_end.record(stream)
         torch.cuda.synchronize(dev)
+        if graph is not None:
+            # The attention kernel's own time, with CUDA events around its launch on the stream,
+            # over the same number of steps right after (for the roofline).
+            for i in range(args.steps):
+                step(kev[i])
+            torch.cuda.synchronize(dev)
         if dist:
             dist.barrier()
     jca.check_status(status, "timed region")
@@ -417,6 +438,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "allowed_pairs": pairs, "effective_flops_per_step": flops,
                    "job_effective_flops_per_step": job_flops,
                    "l2": "inputs (Q/K/V 837 MB) larger than L2 (126 MB); no flush",
+                   "step": ("one CUDA graph of the four launches per step, replayed"
+                            if not args.no_graph else "four launches per step"),
                    "parallelism": parallelism},
         "tokens_per_s": job_tokens * args.steps / (elapsed_ms / 1e3),
         "pct_of_bf16_peak": 100.0 * value / (world * peaks["bf16_tflops"]),
@@ -998,6 +1021,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-extras", action="store_true", help="skip the candidate-only workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the step's kernels one by one instead of replaying a CUDA graph")
     ap.add_argument("--cpu-sample-stride", type=int, default=4)
     ap.add_argument("--only", choices=["cand_only", "rope", "stack", "backward", "causal",
                                        "ug_sep", "configs", "seqpack"],
