@@ -94,6 +94,13 @@ struct Cfg {
   static constexpr int KSTEPS_QK = D / 16;
   static constexpr int KSTEPS_PER_BLK = SW / 32;
   static constexpr int KSTEPS_PV = BN / 16;
+  // Heads of up to 32: P of a key tile is released to the MMA thread in two halves (keys 0..63,
+  // then the rest), so the first half of the PV runs while the softmax computes the second. At
+  // d = 32 a PV is eight MMAs of N = 32, whose issue takes about as long as the softmax half
+  // (retrieval 0.358 -> 0.338 ms); at d = 128 the extra barrier round trip costs more than it
+  // hides (users256 0.70 -> 0.76 ms), so larger heads release P whole.
+  static constexpr bool SPLIT_P = D <= 32;
+  static constexpr int PV_FIRST = KSTEPS_PV / 2;                 // k-steps of the first half
   // Ring depths: query-tile buffers per group and K / V stages. Small heads make short items
   // (a few key tiles) whose loads must be issued an item ahead to hide HBM latency; their tiles are
   // small, so the rings are deeper there. D = 128 fills shared memory with one Q buffer per group.
@@ -123,11 +130,13 @@ struct Cfg {
   // instead of the TMA's full barriers).
   static constexpr int B_QREADY = B_RINGEMPTY + kRing;     // [group][QS]
   static constexpr int B_KREADY = B_QREADY + 2 * QS;       // [KVS]
-  static constexpr int NUM_BARS = B_KREADY + KVS;
+  // [group]: keys 0..63 of P_w written (SPLIT_P: the PV may start on them).
+  static constexpr int B_PHALF = B_KREADY + KVS;
+  static constexpr int NUM_BARS = B_PHALF + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // Diagonal scores of the candidate rows: two item slots of kItemRows floats.
-  static constexpr int OFF_RING = OFF_MISC + 16;           // kRing claimed item indices
-  static constexpr int OFF_DIAG = OFF_RING + 4 * kRing;
+  static constexpr int OFF_RING = OFF_MISC + 16;           // kRing claimed item descriptors
+  static constexpr int OFF_DIAG = OFF_RING + 16 * kRing;
   static constexpr int SMEM_USED = OFF_DIAG + 2 * kItemRows * 4;
   static constexpr int SMEM_RAW = SMEM_USED + 1024;                // slack for 1 KB alignment
   // At least 120 KB so that a second CTA never shares the SM (and its TMEM).
@@ -165,39 +174,48 @@ __device__ __forceinline__ Item decode_item(int4 v) {
 
 // Work items are claimed at run time from a global counter, so that a CTA that finishes early
 // takes the next item (the queue is sorted by cost, largest first). The claiming thread (producer
-// lane 0) writes each claimed index, or -1 once the queue is exhausted, into a shared ring; every
-// other role reads the same sequence from the ring and releases each slot after reading it.
+// lane 0) reads each claimed item's descriptor from the queue and writes it (or an end marker once
+// the queue is exhausted) into a shared ring; every other role reads the same sequence of
+// descriptors from the ring and releases each slot after reading it. The claimer runs up to kRing
+// items ahead, so no role waits on the global queue at an item boundary.
 struct ItemRing {
-  volatile int* slot;   // kRing shared entries
+  volatile int* slot;   // kRing shared entries of 4 ints (the item descriptor)
   uint32_t full;        // address of full barrier 0 (kRing consecutive barriers)
   uint32_t empty;       // address of empty barrier 0
   uint32_t k;           // entries taken so far
 };
 
-__device__ __forceinline__ int ring_claim(ItemRing& r, int32_t* head, int n_items,
-                                          volatile int* abort_flag, int32_t* status, bool& ok) {
+constexpr int kEndOfQueue = -1;   // q_row0 of the end marker (real items start at row >= 0)
+
+__device__ __forceinline__ int4 ring_claim(ItemRing& r, const int4* items, int32_t* head,
+                                           int n_items, volatile int* abort_flag, int32_t* status,
+                                           bool& ok) {
   const int s = (int)(r.k % kRing);
   ok = mbar_wait(r.empty + 8 * s, ((r.k / kRing) & 1) ^ 1, abort_flag, status);
-  if (!ok) return -1;
-  int v = atomicAdd(head, 1);
-  if (v >= n_items) v = -1;
-  r.slot[s] = v;
+  if (!ok) return make_int4(kEndOfQueue, 0, 0, 0);
+  const int v = atomicAdd(head, 1);
+  const int4 d = v < n_items ? items[v] : make_int4(kEndOfQueue, 0, 0, 0);
+  r.slot[4 * s + 0] = d.x;
+  r.slot[4 * s + 1] = d.y;
+  r.slot[4 * s + 2] = d.z;
+  r.slot[4 * s + 3] = d.w;
   mbar_arrive(r.full + 8 * s);
   ++r.k;
-  return v;
+  return d;
 }
 
 // Every thread of a consuming role calls this (warps stay converged: `ok` is made warp-uniform
 // by the caller where warp-collective operations follow).
-__device__ __forceinline__ int ring_take(ItemRing& r, volatile int* abort_flag, int32_t* status,
-                                         bool& ok) {
+__device__ __forceinline__ int4 ring_take(ItemRing& r, volatile int* abort_flag, int32_t* status,
+                                          bool& ok) {
   const int s = (int)(r.k % kRing);
   ok = mbar_wait(r.full + 8 * s, (r.k / kRing) & 1, abort_flag, status);
-  if (!ok) return -1;
-  const int v = r.slot[s];
+  if (!ok) return make_int4(kEndOfQueue, 0, 0, 0);
+  const int4 d = make_int4(r.slot[4 * s + 0], r.slot[4 * s + 1], r.slot[4 * s + 2],
+                           r.slot[4 * s + 3]);
   mbar_arrive(r.empty + 8 * s);
   ++r.k;
-  return v;
+  return d;
 }
 
 // ------------------------------------------------------------------------------------------
@@ -218,12 +236,38 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
   bool ok = true;
   for (;;) {
     // Lane 0 claims the CTA's next item; lane 1 reads the claims from the ring.
-    const int it = loads_v ? ring_take(ring, abort_flag, a.status, ok)
-                           : ring_claim(ring, a.queue, n_items, abort_flag, a.status, ok);
-    if (!ok || it < 0) break;
-    const Item w = decode_item(a.items[it]);
+    const int4 desc = loads_v ? ring_take(ring, abort_flag, a.status, ok)
+                              : ring_claim(ring, a.items, a.queue, n_items, abort_flag, a.status, ok);
+    if (!ok || desc.x == kEndOfQueue) break;
+    const Item w = decode_item(desc);
     if (w.n_kv == 0) continue;
+    const int empty = loads_v ? C::B_VEMPTY : C::B_KEMPTY;
+    const int full = loads_v ? C::B_VFULL : C::B_KFULL;
+    const CUtensorMap* map = loads_v ? tmV : tmK;
+    const int off = loads_v ? C::OFF_V : C::OFF_K;
+    auto load_kv = [&](int j) -> bool {
+      const int s = (int)(g % C::KVS);
+      const uint32_t ph = (g / C::KVS) & 1;
+      const int row = w.kv_lo + j * C::BN;
+      if (!mbar_wait(bars + 8 * (empty + s), ph ^ 1, abort_flag, a.status)) return false;
+      mbar_arrive_expect_tx(bars + 8 * (full + s), C::TILE_BYTES);
+#pragma unroll
+      for (int c = 0; c < C::NBLK; ++c)
+        tma_load_3d(sbase + off + s * C::TILE_BYTES + c * C::BLK_BYTES, map,
+                    bars + 8 * (full + s), c * C::BOX_X, w.h, row);
+      ++g;
+      return true;
+    };
+    int j0 = 0;
     if (!loads_v) {
+      // The item's first K tile goes out before its Q tiles: its stage was freed by a QK of the
+      // previous item's second-to-last key tile, while the Q buffers wait for the last, so the
+      // load is issued a key tile earlier and lands before the item's first QK needs it
+      // (users256 0.714 -> 0.702 ms). Every earlier K tile's item had its Q tiles issued by
+      // then, so no release this wait depends on is held up by it.
+      ok = load_kv(0);
+      if (!ok) break;
+      j0 = 1;
       const int ntiles = w.nrows > C::BM ? 2 : 1;
       for (int t = 0; ok && t < ntiles; ++t) {
         // Load n of a buffer waits for the release of load n - 1 (immediate the first time).
@@ -240,21 +284,9 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
       }
       if (!ok) break;
     }
-    const int empty = loads_v ? C::B_VEMPTY : C::B_KEMPTY;
-    const int full = loads_v ? C::B_VFULL : C::B_KFULL;
-    const CUtensorMap* map = loads_v ? tmV : tmK;
-    const int off = loads_v ? C::OFF_V : C::OFF_K;
-    for (int j = 0; j < w.n_kv; ++j, ++g) {
-      const int s = (int)(g % C::KVS);
-      const uint32_t ph = (g / C::KVS) & 1;
-      const int row = w.kv_lo + j * C::BN;
-      ok = mbar_wait(bars + 8 * (empty + s), ph ^ 1, abort_flag, a.status);
+    for (int j = j0; j < w.n_kv; ++j) {
+      ok = load_kv(j);
       if (!ok) break;
-      mbar_arrive_expect_tx(bars + 8 * (full + s), C::TILE_BYTES);
-#pragma unroll
-      for (int c = 0; c < C::NBLK; ++c)
-        tma_load_3d(sbase + off + s * C::TILE_BYTES + c * C::BLK_BYTES, map,
-                    bars + 8 * (full + s), c * C::BOX_X, w.h, row);
     }
   }
   if (!ok) {
@@ -318,6 +350,27 @@ __device__ __forceinline__ void mma_pv(uint32_t o_tmem, uint32_t p_tmem, uint64_
   }
 }
 
+// k-steps [k0, k1) of O_w += P_w V (SPLIT_P halves); a range of N k-steps is straight-line code.
+template <int D, int N>
+__device__ __forceinline__ void mma_pv_range(uint32_t o_tmem, uint32_t p_tmem, uint64_t vb, int k0,
+                                             int k1, bool overwrite) {
+  using C = Cfg<D>;
+  constexpr uint32_t kIdescPV = idesc_bf16_f32(C::BM, D, false, true);
+  constexpr uint32_t kStep = (16 * C::SW) >> 4;   // 16 key rows of V per k-step
+  if (k1 - k0 == N) {
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const int kk = k0 + i;
+      tc_mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u, vb + (uint64_t)(kk * kStep), kIdescPV,
+                (overwrite && i == 0) ? 0u : 1u);
+    }
+  } else {
+    for (int kk = k0; kk < k1; ++kk)
+      tc_mma_ts(o_tmem, p_tmem + (uint32_t)kk * 8u, vb + (uint64_t)(kk * kStep), kIdescPV,
+                (overwrite && kk == k0) ? 0u : 1u);
+  }
+}
+
 // O_w += P_w V for key tile jj of the item (global tile gg: V stage), whose first `valid` keys are
 // real: only ceil(valid / 16) k-steps are issued. P_w is read from the first 64 TMEM columns of
 // S_w (bf16 pairs: 16 keys = 8 columns per k-step). The first PV of an item overwrites O_w, so it
@@ -333,15 +386,28 @@ __device__ __forceinline__ bool issue_pv(int grp, uint32_t gg, int jj, int valid
       return false;
     st.v_seen = gg + 1;
   }
-  if (!mbar_wait(bars + 8 * (C::B_PFULL + grp), st.p_seen[grp] & 1, abort_flag, a.status))
-    return false;
+  const uint32_t par = st.p_seen[grp] & 1;
   ++st.p_seen[grp];
+  if (!mbar_wait(bars + 8 * ((C::SPLIT_P ? C::B_PHALF : C::B_PFULL) + grp), par, abort_flag,
+                 a.status))
+    return false;
   if (jj == 0 && st.o_items[grp] > 0 &&
       !mbar_wait(bars + 8 * (C::B_OFREE + grp), (st.o_items[grp] - 1) & 1, abort_flag, a.status))
     return false;
   tc_fence_after();
-  mma_pv<D>(tmem + (grp ? C::TMEM_O1 : C::TMEM_O0), tmem + (grp ? C::TMEM_S1 : C::TMEM_S0),
-            st.v + (uint64_t)((s * C::TILE_BYTES) >> 4), (valid + 15) >> 4, jj == 0);
+  const uint32_t o_t = tmem + (grp ? C::TMEM_O1 : C::TMEM_O0);
+  const uint32_t p_t = tmem + (grp ? C::TMEM_S1 : C::TMEM_S0);
+  const uint64_t vb = st.v + (uint64_t)((s * C::TILE_BYTES) >> 4);
+  const int ksteps = (valid + 15) >> 4;
+  if (!C::SPLIT_P) {
+    mma_pv<D>(o_t, p_t, vb, ksteps, jj == 0);
+    return true;
+  }
+  const int first = ksteps < C::PV_FIRST ? ksteps : C::PV_FIRST;
+  mma_pv_range<D, C::PV_FIRST>(o_t, p_t, vb, 0, first, jj == 0);
+  if (!mbar_wait(bars + 8 * (C::B_PFULL + grp), par, abort_flag, a.status)) return false;
+  tc_fence_after();
+  mma_pv_range<D, C::KSTEPS_PV - C::PV_FIRST>(o_t, p_t, vb, first, ksteps, false);
   return true;
 }
 
@@ -391,9 +457,9 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     return true;
   };
   for (;;) {
-    const int it = ring_take(ring, abort_flag, a.status, ok);
-    if (!ok || it < 0) break;
-    const Item w = decode_item(a.items[it]);
+    const int4 desc = ring_take(ring, abort_flag, a.status, ok);
+    if (!ok || desc.x == kEndOfQueue) break;
+    const Item w = decode_item(desc);
     if (w.n_kv == 0) continue;
     const bool has_b = w.nrows > C::BM;
     // This item's Q buffers (one per query tile) in the per-group rings.
@@ -830,9 +896,9 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t sbase, uint
     return true;
   };
   for (;; ++n) {
-    const int it = ring_take(ring, abort_flag, a.status, ok);
-    if (!ok || it < 0) return;
-    const Item w = decode_item(a.items[it]);
+    const int4 desc = ring_take(ring, abort_flag, a.status, ok);
+    if (!ok || desc.x == kEndOfQueue) return;
+    const Item w = decode_item(desc);
     if (ROPE && w.n_kv > 0) {
       // The item's query tiles, then its first key tile, are rotated before anything else: the
       // tensor core waits on them. The remaining key tiles follow the diagonal scores.
@@ -908,10 +974,10 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
   bool ok = true;
   uint32_t n = 0;                             // items walked (diagonal-score slot sequence)
   for (;; ++n) {
-    const int it = ring_take(ring, abort_flag, a.status, ok);
+    const int4 desc = ring_take(ring, abort_flag, a.status, ok);
     ok = __all_sync(0xffffffffu, ok);
-    if (!ok || it < 0) break;
-    const Item w = decode_item(a.items[it]);
+    if (!ok || desc.x == kEndOfQueue) break;
+    const Item w = decode_item(desc);
     const int slot = n & 1;
     if (grp == 1 && w.nrows <= C::BM) {
       // The item has no tile B; its diagonal-score slot is still released (after it was filled,
@@ -994,11 +1060,22 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       // Pass 2: p = 2^(scale_log2 * s - m), written back over S_w as bf16 pairs (TMEM column k
       // holds keys 2k, 2k+1) 32 keys at a time; chunks past the last real key are never read
       // by the trimmed PV and are skipped. Arithmetic runs on key pairs (packed fp32 FMA/add).
+      // TMEM loads and stores are warp-collective: the warp rescales O_w (after pass 2) when any
+      // of its rows must. With SPLIT_P such a warp releases the first half of P only after the
+      // rescale, since the first PV k-step already adds into every row of O_w.
+      const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
+      const bool warp_rescale = __any_sync(0xffffffffu, rescale && j >= 1);
       const float2 sl2v = make_float2(sl2, sl2), negv = make_float2(neg_m, neg_m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0, acc2 = acc0, acc3 = acc0;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        if (c >= nchunks) break;
+        if (C::SPLIT_P && 32 * c == 16 * C::PV_FIRST && !warp_rescale) {
+          // Keys 0..63 of P_w are written: the PV may start on them.
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bars + 8 * (C::B_PHALF + grp));
+        }
+        if (c >= nchunks) continue;
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -1019,14 +1096,13 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       const float2 acc01 = __fadd2_rn(acc0, acc1), acc23 = __fadd2_rn(acc2, acc3);
       const float tile_sum = (acc01.x + acc01.y) + (acc23.x + acc23.y);
       // O_w is stable here: its last PV was issued before the QK that filled S_w, and that
-      // QK's commit fired only after every earlier MMA completed. TMEM loads/stores are
-      // warp-collective: the warp rescales when any of its rows must.
-      const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
-      if (__any_sync(0xffffffffu, rescale && j >= 1)) rescale_o_row<D>(t_o, alpha);
+      // QK's commit fired only after every earlier MMA completed.
+      if (warp_rescale) rescale_o_row<D>(t_o, alpha);
       l = l * alpha + tile_sum;
       m = m_use;
       tmem_wait_st();
       tc_fence_before();
+      if (C::SPLIT_P && warp_rescale) mbar_arrive(bars + 8 * (C::B_PHALF + grp));
       mbar_arrive(bars + 8 * (C::B_PFULL + grp));
     }
     if (!ok) break;
@@ -1103,6 +1179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2 * C::QS; ++i) mbar_init(bars + 8 * (C::B_QREADY + i), kDiagThreads);
     for (int i = 0; i < C::KVS; ++i) mbar_init(bars + 8 * (C::B_KREADY + i), kDiagThreads);
+    for (int i = 0; i < 2; ++i) mbar_init(bars + 8 * (C::B_PHALF + i), kSoftmaxThreads / 2);
     *abort_flag = 0;
     mbar_fence_init();
     fence_proxy_async_smem();
