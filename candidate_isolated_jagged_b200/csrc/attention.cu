@@ -29,8 +29,11 @@
 // done and O_w may be rescaled in place.
 // Work items (user, head, 256-row query block) come from the cost-sorted queue and are claimed at
 // run time from a global counter, so the longest items start first and a CTA that finishes early
-// takes the next one. The kernel is instantiated per mode: the main path, the per-user causal
-// variant (CAUSAL) and the training forward that also writes each row's log-sum-exp (LSE).
+// takes the next one; the claiming thread passes each item's descriptor to every role through a
+// shared ring. Heads of up to 32 release each key tile's P to the MMA thread in two halves, so
+// that the first half of the PV overlaps the softmax of the second. The kernel is instantiated
+// per mode: the main path, the per-user causal variant (CAUSAL), the training forward that also
+// writes each row's log-sum-exp (LSE) and the in-kernel RoPE rotation (ROPE).
 #include <climits>
 #include <cmath>
 #include <cstdint>
