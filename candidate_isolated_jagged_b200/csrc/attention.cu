@@ -33,7 +33,12 @@
 // shared ring. Heads of up to 32 release each key tile's P to the MMA thread in two halves, so
 // that the first half of the PV overlaps the softmax of the second. The kernel is instantiated
 // per mode: the main path, the per-user causal variant (CAUSAL), the training forward that also
-// writes each row's log-sum-exp (LSE) and the in-kernel RoPE rotation (ROPE).
+// writes each row's log-sum-exp (LSE), the in-kernel RoPE rotation (ROPE), and the candidate-only
+// layer with heads of 64 or more (DT), where every row is a candidate: there each query tile's own
+// keys and values arrive as TMA tiles and go through the tensor core as one more "diagonal" key
+// step after the history tiles (QK against the own keys, of which each row keeps its own score;
+// P zero off the diagonal; PV against the own values), instead of per-row loads on CUDA cores;
+// the diagonal warps then only follow the item ring.
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -227,10 +232,12 @@ __device__ __forceinline__ int4 ring_take(ItemRing& r, volatile int* abort_flag,
 // Two producer threads in warp 0 walk the same item sequence: lane 0 loads the Q tiles (a ring of
 // QS buffers per query tile, each refilled once the last QK of the item that used it completed)
 // and the K tiles (stages freed by QK completions), lane 1 loads the V tiles (stages freed by PV
-// completions), so a slow PV never holds back the next K.
-template <int D>
+// completions), so a slow PV never holds back the next K. With DT each item also gets its query
+// tiles' own keys (lane 0) and values (lane 1), one stage per query tile, after its key tiles.
+template <int D, bool DT>
 __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
-                              const CUtensorMap* tmV, const AttnArgs& a, uint32_t sbase,
+                              const CUtensorMap* tmV, const CUtensorMap* tmDK,
+                              const CUtensorMap* tmDV, const AttnArgs& a, uint32_t sbase,
                               uint32_t bars, int n_items, volatile int* abort_flag, bool loads_v,
                               ItemRing ring) {
   using C = Cfg<D>;
@@ -243,7 +250,7 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
                               : ring_claim(ring, a.items, a.queue, n_items, abort_flag, a.status, ok);
     if (!ok || desc.x == kEndOfQueue) break;
     const Item w = decode_item(desc);
-    if (w.n_kv == 0) continue;
+    if (!DT && w.n_kv == 0) continue;
     const int empty = loads_v ? C::B_VEMPTY : C::B_KEMPTY;
     const int full = loads_v ? C::B_VFULL : C::B_KFULL;
     const CUtensorMap* map = loads_v ? tmV : tmK;
@@ -268,9 +275,11 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
       // load is issued a key tile earlier and lands before the item's first QK needs it
       // (users256 0.714 -> 0.702 ms). Every earlier K tile's item had its Q tiles issued by
       // then, so no release this wait depends on is held up by it.
-      ok = load_kv(0);
-      if (!ok) break;
-      j0 = 1;
+      if (!DT || w.n_kv > 0) {
+        ok = load_kv(0);
+        if (!ok) break;
+        j0 = 1;
+      }
       const int ntiles = w.nrows > C::BM ? 2 : 1;
       for (int t = 0; ok && t < ntiles; ++t) {
         // Load n of a buffer waits for the release of load n - 1 (immediate the first time).
@@ -290,6 +299,24 @@ __device__ void producer_role(const CUtensorMap* tmQ, const CUtensorMap* tmK,
     for (int j = j0; j < w.n_kv; ++j) {
       ok = load_kv(j);
       if (!ok) break;
+    }
+    if (DT && ok) {
+      // Diagonal step: each query tile's own keys (lane 0) or values (lane 1), one stage each,
+      // in the order the MMA thread consumes the stages (tile A's, then tile B's).
+      const CUtensorMap* dmap = loads_v ? tmDV : tmDK;
+      const int ntiles = w.nrows > C::BM ? 2 : 1;
+      for (int t = 0; t < ntiles; ++t) {
+        const int s = (int)(g % C::KVS);
+        const uint32_t ph = (g / C::KVS) & 1;
+        ok = mbar_wait(bars + 8 * (empty + s), ph ^ 1, abort_flag, a.status);
+        if (!ok) break;
+        mbar_arrive_expect_tx(bars + 8 * (full + s), C::TILE_BYTES);
+#pragma unroll
+        for (int c = 0; c < C::NBLK; ++c)
+          tma_load_3d(sbase + off + s * C::TILE_BYTES + c * C::BLK_BYTES, dmap,
+                      bars + 8 * (full + s), c * C::BOX_X, w.h, w.q_row0 + t * C::BM);
+        ++g;
+      }
     }
   }
   if (!ok) {
@@ -426,7 +453,7 @@ struct PendingPV {
   bool last;     // the item's last key tile: its completion makes O ready
 };
 
-template <int D, bool CAUSAL, bool ROPE>
+template <int D, bool CAUSAL, bool ROPE, bool DT>
 __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint32_t tmem,
                          volatile int* abort_flag, ItemRing ring) {
   using C = Cfg<D>;
@@ -463,7 +490,7 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     const int4 desc = ring_take(ring, abort_flag, a.status, ok);
     if (!ok || desc.x == kEndOfQueue) break;
     const Item w = decode_item(desc);
-    if (w.n_kv == 0) continue;
+    if (!DT && w.n_kv == 0) continue;
     const bool has_b = w.nrows > C::BM;
     // This item's Q buffers (one per query tile) in the per-group rings.
     const int qslot_a = (int)(st.q_seen[0] % C::QS);
@@ -478,7 +505,8 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
     for (int j = 0; j < w.n_kv; ++j, ++g) {
       const int s = (int)(g % C::KVS);
       const uint32_t ph = (g / C::KVS) & 1;
-      const bool last = j == w.n_kv - 1;
+      // With the diagonal step the item's last QK and PV come after its key tiles.
+      const bool last = !DT && j == w.n_kv - 1;
       // Causal variant: an item's key tiles end at its last row, which tile B holds; tile A's
       // rows end 128 rows earlier and see none of the last key tile, so A stops one tile early.
       const bool a_skips = CAUSAL && has_b && last;
@@ -525,6 +553,45 @@ __device__ void mma_role(const AttnArgs& a, uint32_t sbase, uint32_t bars, uint3
         }
       }
       if (has_b) pend = PendingPV{g, j, valid, last};
+    }
+    if (DT) {
+      if (!ok) break;
+      // Diagonal step: S_w = Q_w K_own,w^T against the query tile's own keys (only the diagonal
+      // is used), then O_w += P_w V_own,w with P_w zero off the diagonal. Group A's own keys and
+      // values occupy one K / V stage, group B's the next.
+      const int sa = (int)(g % C::KVS), sb = (int)((g + 1) % C::KVS);
+      ok = mbar_wait(bars + 8 * (KF + sa), (g / C::KVS) & 1, abort_flag, a.status);
+      if (!ok) break;
+      tc_fence_after();
+      mma_qk<D>(tmem + C::TMEM_S0, qa, st.k + (uint64_t)((sa * C::TILE_BYTES) >> 4), kIdescQKFull);
+      tc_commit(bars + 8 * C::B_SFULL);
+      tc_commit(bars + 8 * (C::B_QEMPTY + qslot_a));
+      tc_commit(bars + 8 * (C::B_KEMPTY + sa));
+      ok = flush_b();
+      if (!ok) break;
+      if (has_b) {
+        if (w.n_kv == 0) {
+          ok = mbar_wait(bars + 8 * (QF + qslot_b), (st.q_seen[1] / C::QS) & 1, abort_flag,
+                         a.status);
+          if (!ok) break;
+          ++st.q_seen[1];
+        }
+        ok = mbar_wait(bars + 8 * (KF + sb), ((g + 1) / C::KVS) & 1, abort_flag, a.status);
+        if (!ok) break;
+        tc_fence_after();
+        mma_qk<D>(tmem + C::TMEM_S1, qb, st.k + (uint64_t)((sb * C::TILE_BYTES) >> 4),
+                  kIdescQKFull);
+        tc_commit(bars + 8 * (C::B_SFULL + 1));
+        tc_commit(bars + 8 * (C::B_QEMPTY + qslot_b));
+        tc_commit(bars + 8 * (C::B_KEMPTY + sb));
+      }
+      ok = issue_pv<D>(0, g, w.n_kv == 0 ? 0 : 1, C::BN, st, bars, tmem, a, abort_flag);
+      if (!ok) break;
+      tc_commit(bars + 8 * (C::B_VEMPTY + sa));
+      tc_commit(bars + 8 * C::B_OREADY);
+      ++st.o_items[0];
+      if (has_b) pend = PendingPV{g + 1, w.n_kv == 0 ? 0 : 1, C::BN, true};
+      g += has_b ? 2u : 1u;
     }
   }
   if (ok) ok = flush_b();
@@ -879,10 +946,18 @@ __device__ __forceinline__ float diag_score_rope(const AttnArgs& a, size_t base,
 // a two-slot shared array; it also starts moving each candidate row's own value towards L2 for
 // the epilogue. Slot s is reused for the item after next once all 256 softmax threads have taken
 // the scores out of it.
-template <int D, bool CAUSAL, bool ROPE>
+template <int D, bool CAUSAL, bool ROPE, bool DT>
 __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t sbase, uint32_t bars,
                           volatile int* abort_flag, int t, ItemRing ring) {
   using C = Cfg<D>;
+  if (DT) {
+    // The diagonal terms go through the tensor core: these warps only follow the item ring.
+    bool ok = true;
+    for (;;) {
+      const int4 desc = ring_take(ring, abort_flag, a.status, ok);
+      if (!ok || desc.x == kEndOfQueue) return;
+    }
+  }
   uint32_t n = 0;
   uint32_t nq[2] = {0, 0};   // ROPE: Q tiles rotated per query tile (mirrors the producer)
   uint32_t g = 0;            // ROPE: K tiles rotated
@@ -960,7 +1035,7 @@ __device__ void diag_role(const AttnArgs& a, float* sd_buf, uint32_t sbase, uint
   }
 }
 
-template <int D, bool CAUSAL, bool LSE>
+template <int D, bool CAUSAL, bool LSE, bool DT>
 __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
                              const float* sd_buf, volatile int* abort_flag, int warp, int lane,
                              ItemRing ring) {
@@ -982,6 +1057,7 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
     if (!ok || desc.x == kEndOfQueue) break;
     const Item w = decode_item(desc);
     const int slot = n & 1;
+    if (DT && grp == 1 && w.nrows <= C::BM) continue;
     if (grp == 1 && w.nrows <= C::BM) {
       // The item has no tile B; its diagonal-score slot is still released (after it was filled,
       // so that this release cannot count toward the slot's previous use).
@@ -1109,6 +1185,57 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       mbar_arrive(bars + 8 * (C::B_PFULL + grp));
     }
     if (!ok) break;
+    if (DT) {
+      // Diagonal step: S holds this tile's rows against their own keys; each row keeps only its
+      // own score (column r), merged like a key tile's, and P is zero off the diagonal.
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bars + 8 * (C::B_SFULL + grp), lt & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      ++lt;
+      uint32_t xs[32];
+      tmem_ld_x32(t_s + (uint32_t)(quarter * 32), xs);
+      tmem_wait_ld();
+      reg_fence16(xs);
+      reg_fence16(xs + 16);
+      float sraw = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) sraw = c == lane ? __uint_as_float(xs[c]) : sraw;
+      const float s2 = sraw * sl2;
+      const float m_new = fmaxf(m, s2);
+      const bool rescale = m_new > m + 8.0f;
+      const float m_use = rescale ? m_new : m;
+      const float alpha = (rescale && m != -INFINITY) ? fast_exp2(m - m_use) : 1.f;
+      const uint32_t pb = pack_bf16x2(fast_exp2(s2 - m_use), 0.f) & 0xFFFFu;
+      // The row sum takes the weight exactly as the PV applies it (bf16), so that a row whose own
+      // term dominates is normalised by that same weight.
+      const float p = __uint_as_float(pb << 16);
+      const uint32_t pw = (r & 1) ? (pb << 16) : pb;
+      const int pcol = r >> 1;   // TMEM column of P holding keys 2 pcol, 2 pcol + 1
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = (16 * c + i == pcol) ? pw : 0u;
+        tmem_st_x16(t_s + 16 * c, pk);
+      }
+      // O_w is stable here (as for a key tile); the item's first step needs no rescale.
+      if (__any_sync(0xffffffffu, rescale && w.n_kv > 0)) rescale_o_row<D>(t_o, alpha);
+      l = l * alpha + p;
+      m = m_use;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bars + 8 * (C::B_PFULL + grp));
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(bars + 8 * (C::B_OREADY + grp), oi & 1, abort_flag, a.status));
+      if (!ok) break;
+      tc_fence_after();
+      ++oi;
+      const uint4 vz[D / 8] = {};
+      finish_row<D, LSE>(a, row_ok, row_ok ? 1 : 0, base, t_o, true, m, l, -INFINITY, vz,
+                         bars + 8 * (C::B_OFREE + grp));
+      continue;
+    }
     // The row's own value is fetched while the item's last PV runs.
     uint4 vv[D / 8];
     {
@@ -1137,11 +1264,13 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
 // ------------------------------------------------------------------------------------------
 // Kernel
 // ------------------------------------------------------------------------------------------
-template <int D, bool CAUSAL, bool LSE, bool ROPE>
+template <int D, bool CAUSAL, bool LSE, bool ROPE, bool DT>
 __global__ void __launch_bounds__(kThreads, 1)
     jagged_attn_kernel(const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmDK,
+                       const __grid_constant__ CUtensorMap tmDV, const AttnArgs a) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -1191,6 +1320,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_map(&tmQ);
     tma_prefetch_map(&tmK);
     tma_prefetch_map(&tmV);
+    if (DT) {
+      tma_prefetch_map(&tmDK);
+      tma_prefetch_map(&tmDV);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -1207,14 +1340,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!*skip) {
     if (warp == 0) {
       if (lane < 2)
-        producer_role<D>(&tmQ, &tmK, &tmV, a, sbase, bars, n_items, abort_flag, lane == 1, ring);
+        producer_role<D, DT>(&tmQ, &tmK, &tmV, &tmDK, &tmDV, a, sbase, bars, n_items, abort_flag,
+                             lane == 1, ring);
     } else if (warp == 1) {
-      if (lane == 0) mma_role<D, CAUSAL, ROPE>(a, sbase, bars, tmem, abort_flag, ring);
+      if (lane == 0) mma_role<D, CAUSAL, ROPE, DT>(a, sbase, bars, tmem, abort_flag, ring);
     } else if (warp < 10) {
-      softmax_role<D, CAUSAL, LSE>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
+      softmax_role<D, CAUSAL, LSE, DT>(a, bars, tmem, reinterpret_cast<const float*>(smem + C::OFF_DIAG),
                       abort_flag, warp, lane, ring);
     } else {
-      diag_role<D, CAUSAL, ROPE>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), sbase, bars,
+      diag_role<D, CAUSAL, ROPE, DT>(a, reinterpret_cast<float*>(smem + C::OFF_DIAG), sbase, bars,
                                  abort_flag,
                    threadIdx.x - 320, ring);
     }
@@ -1257,18 +1391,21 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
   {
     std::lock_guard<std::mutex> lock(g_attr_mu);
     if (!g_attr_set[dev][d_index(D)]) {
-      if (cudaFuncSetAttribute(jagged_attn_kernel<D, false, false, false>,
+      if (cudaFuncSetAttribute(jagged_attn_kernel<D, false, false, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess ||
-          cudaFuncSetAttribute(jagged_attn_kernel<D, true, false, false>,
+          cudaFuncSetAttribute(jagged_attn_kernel<D, true, false, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess ||
-          cudaFuncSetAttribute(jagged_attn_kernel<D, false, true, false>,
+          cudaFuncSetAttribute(jagged_attn_kernel<D, false, true, false, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                C::SMEM_ALLOC) != cudaSuccess ||
-          cudaFuncSetAttribute(jagged_attn_kernel<D, false, false, true>,
+          cudaFuncSetAttribute(jagged_attn_kernel<D, false, false, true, false>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               C::SMEM_ALLOC) != cudaSuccess)
+                               C::SMEM_ALLOC) != cudaSuccess ||
+          (D >= 64 && cudaFuncSetAttribute(jagged_attn_kernel<D, false, false, false, true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           C::SMEM_ALLOC) != cudaSuccess))
         return JCA_ERR_CUDA;
       g_attr_set[dev][d_index(D)] = true;
     }
@@ -1280,20 +1417,31 @@ int launch_attention_d(const AttnArgs& a, const void* q, int64_t Tq, const void*
     return JCA_ERR_CUDA;
   AttnArgs args = a;
   args.out_v8 = aligned(a.out, 32) ? 1 : 0;
-  // Instantiations: the main path, the causal variant, and the training forward (log-sum-exp
-  // output); each mode is compile-time so that the main path carries none of the others' code.
+  // Candidate-only layer with heads of 64 or more: the rows' own keys and values go through the
+  // tensor core as a diagonal step (two more maps over them); elsewhere those maps are unused.
+  const bool dt = D >= 64 && a.q_seg == nullptr && !a.causal && a.lse == nullptr && !a.rope;
+  CUtensorMap tmDK = tmK, tmDV = tmV;
+  if (dt && (!make_rows_map_bf16(&tmDK, a.dk, Tq, a.H, D, C::BM) ||
+             !make_rows_map_bf16(&tmDV, a.dv, Tq, a.H, D, C::BM)))
+    return JCA_ERR_CUDA;
+  // Instantiations: the main path, the causal variant, the training forward (log-sum-exp
+  // output), the in-kernel RoPE rotation and the candidate-only diagonal step; each mode is
+  // compile-time so that the main path carries none of the others' code.
   if (a.causal)
-    jagged_attn_kernel<D, true, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
-        tmQ, tmK, tmV, args);
+    jagged_attn_kernel<D, true, false, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, tmDK, tmDV, args);
   else if (a.lse != nullptr)
-    jagged_attn_kernel<D, false, true, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
-        tmQ, tmK, tmV, args);
+    jagged_attn_kernel<D, false, true, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, tmDK, tmDV, args);
   else if (a.rope)
-    jagged_attn_kernel<D, false, false, true><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
-        tmQ, tmK, tmV, args);
+    jagged_attn_kernel<D, false, false, true, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, tmDK, tmDV, args);
+  else if (dt)
+    jagged_attn_kernel<D, false, false, false, (D >= 64)><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, tmDK, tmDV, args);
   else
-    jagged_attn_kernel<D, false, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
-        tmQ, tmK, tmV, args);
+    jagged_attn_kernel<D, false, false, false, false><<<sms, kThreads, C::SMEM_ALLOC, stream>>>(
+        tmQ, tmK, tmV, tmDK, tmDV, args);
   return cudaGetLastError() == cudaSuccess ? JCA_OK : JCA_ERR_CUDA;
 }
 
