@@ -59,7 +59,8 @@ def test_cand_only_equals_full_candidate_rows(d):
         # candidate-only layer (its weight rounded to bf16 as a PV operand, like every other
         # weight), the full layer on CUDA cores in fp32: the same within the parity bar, and both
         # against the oracle.
-        assert_close(got, out_full[ci], f"cand-only vs full candidate rows d={d}")
+        assert_close(got, out_full[ci].cpu().double().numpy(),
+                     f"cand-only vs full candidate rows d={d}")
         ref = full.reference()
         assert_close(got, np.asarray(ref)[cand_idx], f"cand-only d={d}")
 
