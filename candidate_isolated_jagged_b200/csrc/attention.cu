@@ -1225,6 +1225,9 @@ __device__ void softmax_role(const AttnArgs& a, uint32_t bars, uint32_t tmem,
       m = m_use;
       tmem_wait_st();
       tc_fence_before();
+      // The whole diagonal P is written at once: with SPLIT_P (heads of up to 32, where the host
+      // does not select this step) both of its releases go out here.
+      if (C::SPLIT_P) mbar_arrive(bars + 8 * (C::B_PHALF + grp));
       mbar_arrive(bars + 8 * (C::B_PFULL + grp));
       ok = __all_sync(0xffffffffu,
                       mbar_wait(bars + 8 * (C::B_OREADY + grp), oi & 1, abort_flag, a.status));
