@@ -203,7 +203,10 @@ int jagged_cand_attn_run(const void* q, const void* k, const void* v, void* out,
  * Candidate-only attention layer (候选隔离注意力掩码, section 只更新候选的末尾层; the arguments mirror
  * the page's operator inputs candidate_q, history_k, history_v, own_k, own_v): each candidate of
  * user b attends to the frozen history keys/values of user b and to its own key/value only.
- * Its result equals the candidate rows of jagged_cand_attn_fwd on the same K/V.
+ * Its result equals the candidate rows of jagged_cand_attn_fwd on the same K/V: bit for bit at
+ * d_head <= 32; at d_head 64 and 128 the candidate's own key and value go through the tensor core
+ * (its own weight rounded to bf16 like every other weight), and the two agree within the parity
+ * tolerance (max-abs 1e-2, rel-L2 5e-3).
  *   cand_q, own_k, own_v [Nc, H, d_head] bf16, read; cand_offsets [B+1] (idx_bits type).
  *   hist_k, hist_v [Th, H, d_head] bf16, read; hist_offsets [B+1] (idx_bits type).
  *   hist_seg [Th] int8 or NULL: 1 = valid history row, 0 = padding (NULL = all valid).
